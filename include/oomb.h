@@ -1,0 +1,224 @@
+/*
+ * oomb.h — C ABI of the paged chunk-attention library (liboomb.so).
+ *
+ * One chunk's queries attend to a paged KV cache that holds every earlier
+ * chunk plus the chunk itself (causal), on one NVIDIA B200 (sm_100a).  The
+ * method is the one summarised in "Out of the Memory Barrier: A Highly Memory
+ * Efficient Training System for LLMs with Million-Token Contexts"
+ * (gist.science/{pt,es,it}/paper/2602.02108):
+ *   - chunk-recurrent training, activations recomputed in the backward
+ *     ([pt] §2A, [es] §2A, [it] §2A);
+ *   - KV cache AND its gradients in non-contiguous pages, no reallocation or
+ *     copy on append ([pt] §2B, [es] §2B "Gestión de Memoria Paginada",
+ *     [it] §2B);
+ *   - custom forward/backward operators on the paged cache that add gradients
+ *     in place with atomic adds, outside autograd ([pt] §2B "Kernels
+ *     Personalizados", [es] §2B, [it] §2B);
+ *   - page-level Top-K sparse attention by a mean representative vector
+ *     ([pt] §2C, [es] §2B "Atención Escasa a Nivel de Página", [it] §2D);
+ *   - asynchronous CPU offload of KV and gradients with pinned memory and
+ *     dedicated streams ([pt] §2D, [es] §2B "Descarga Asíncrona", [it] §2C).
+ *
+ * Conventions
+ *   - Every call returns an oomb_status; nothing throws across the ABI.
+ *   - Argument errors are detected on the host before any launch and leave
+ *     all buffers untouched.
+ *   - Work is stream-ordered on the stream passed (a cudaStream_t given as
+ *     void*; NULL = the legacy default stream).  Asynchronous CUDA errors
+ *     surface at a later call as OOMB_ERR_CUDA.
+ *   - Kernels never trap or assert.  A kernel that finds an invalid page id
+ *     skips the access and sets the pool's device status word; a kernel whose
+ *     internal wait runs past its limit sets it too and returns.  Read it with
+ *     oomb_get_device_status().
+ *   - Caller-owned buffers (q, o, lse, dO, dq, page lists, workspaces) are
+ *     plain device pointers; the library keeps no caller pointer past a call.
+ *   - The library owns pool memory; a page id stays valid until freed.
+ *
+ * Layouts (row-major, innermost last)
+ *   KV pool     [num_pages][num_kv_heads][2][page_size][head_dim] bf16
+ *               (index 0 of the size-2 axis = K, 1 = V)
+ *   grad pool   same shape, fp32 (dK, dV)
+ *   summaries   [num_pages][num_kv_heads][head_dim] fp32 (mean key of a page)
+ *   q, o, dO, dq  [chunk_len][num_q_heads][head_dim] bf16 (token-major)
+ *   lse, delta  [num_q_heads][chunk_len] fp32, natural log
+ *   query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *
+ * Supported shapes: head_dim 64 or 128; page_size 16, 32, 64 or 128;
+ * chunk_len a positive multiple of page_size; num_q_heads a multiple of
+ * num_kv_heads.
+ */
+#ifndef OOMB_H
+#define OOMB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum oomb_status {
+  OOMB_OK = 0,
+  OOMB_ERR_INVALID_ARG = 1,   /* bad pointer, size, shape or combination       */
+  OOMB_ERR_OUT_OF_PAGES = 2,  /* alloc_page on an exhausted pool               */
+  OOMB_ERR_BAD_PAGE = 3,      /* page id out of range, or freeing a free page  */
+  OOMB_ERR_CUDA = 4,          /* a CUDA runtime call failed                    */
+  OOMB_ERR_TIMEOUT = 5,       /* oomb_wait ran past its limit                  */
+  OOMB_ERR_UNSUPPORTED = 6,   /* shape outside the supported set               */
+  OOMB_ERR_DEVICE_CHECK = 7   /* a kernel recorded a bounds or wait failure    */
+} oomb_status;
+
+typedef enum oomb_location {
+  OOMB_LOC_DEVICE = 0,       /* HBM of desc.device (cudaMalloc)               */
+  OOMB_LOC_PINNED_HOST = 1,  /* page-locked host memory (cudaHostAlloc)       */
+  OOMB_LOC_HOST = 2          /* ordinary host memory; needs no GPU            */
+} oomb_location;
+
+typedef struct oomb_pool oomb_pool; /* opaque, owned by the library */
+
+typedef struct oomb_pool_desc {
+  int32_t num_pages;    /* > 0 */
+  int32_t page_size;    /* tokens per page: 16, 32, 64 or 128 */
+  int32_t num_kv_heads; /* > 0 */
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t location;     /* oomb_location */
+  int32_t with_grad;    /* non-zero: allocate the fp32 gradient pool too */
+  uint64_t alloc_seed;  /* 0: pages handed out ascending; otherwise in the order of
+                           a Fisher-Yates shuffle driven by SplitMix64(alloc_seed) */
+  int32_t device;       /* CUDA device ordinal (ignored for OOMB_LOC_HOST) */
+} oomb_pool_desc;
+
+/* ---------------------------------------------------------------- pools
+ * Paged memory for the KV cache and its gradients ([pt] §2B, [it] §2B: pages
+ * are non-contiguous, so appending needs no reallocation or copy).
+ * The free list is a stack: pages freed are handed out again first (LIFO).
+ * Pool buffers are zero-filled at creation. */
+oomb_status oomb_pool_create(const oomb_pool_desc* desc, oomb_pool** out_pool);
+oomb_status oomb_pool_destroy(oomb_pool* pool); /* NULL is accepted */
+/* Pops the next free page id; OOMB_ERR_OUT_OF_PAGES when none is left. */
+oomb_status oomb_pool_alloc_page(oomb_pool* pool, int32_t* out_page_id);
+/* Returns a page to the free list; OOMB_ERR_BAD_PAGE if out of range or already free. */
+oomb_status oomb_pool_free_page(oomb_pool* pool, int32_t page_id);
+oomb_status oomb_pool_num_free(const oomb_pool* pool, int32_t* out_num_free);
+/* Borrowed views of the pool's buffers (any output may be NULL; grad is NULL
+ * without with_grad).  Valid until oomb_pool_destroy. */
+oomb_status oomb_pool_buffers(const oomb_pool* pool, void** kv, float** grad, float** summary);
+oomb_status oomb_pool_get_desc(const oomb_pool* pool, oomb_pool_desc* out_desc);
+
+/* ---------------------------------------------------------------- append
+ * Writes one chunk's keys and values into pages of a device pool, computes each
+ * written page's fp32 mean key per KV head (the page representative, [es] §2B)
+ * and zero-fills the written pages' gradient blocks.
+ *   d_page_ids  device int32[n_pages]: physical page of the chunk's i-th page
+ *   d_k, d_v    device bf16 [n_pages*page_size][num_kv_heads][head_dim] */
+oomb_status oomb_kv_append(oomb_pool* pool, const int32_t* d_page_ids, int32_t n_pages,
+                           const void* d_k, const void* d_v, void* stream);
+
+/* ---------------------------------------------------------------- attention
+ * Row i of the chunk (query head h, KV head g = h / G) attends to every token
+ * of the past pages listed for group g (unmasked) and to the chunk's own keys
+ * at local positions <= i (causal):
+ *   S_ij = scale q_i.k_j,  LSE_i = ln sum_j exp(S_ij),  O_i = sum_j exp(S_ij - LSE_i) v_j.
+ * Dense attention lists every past page for every group; page-sparse lists
+ * the pages oomb_page_topk kept. */
+typedef struct oomb_attn_args {
+  const void* q;      /* device bf16 [chunk_len][num_q_heads][head_dim]            */
+  void* o;            /* device bf16, same layout: fwd output, bwd input           */
+  float* lse;         /* device fp32 [num_q_heads][chunk_len]: fwd output, bwd input */
+  const void* d_o;    /* device bf16, layout of q: bwd input (dL/dO)               */
+  void* dq;           /* device bf16, layout of q: bwd output (overwritten)        */
+  float* delta_ws;    /* device fp32 [num_q_heads][chunk_len]: bwd workspace       */
+  int32_t chunk_len;
+  int32_t num_q_heads;
+  const int32_t* past_pages;  /* device int32 [num_kv_heads][max_past] physical ids  */
+  const int32_t* past_counts; /* device int32 [num_kv_heads], each in [0, max_past]   */
+  int32_t max_past;           /* row stride of past_pages; 0 for the first chunk     */
+  const int32_t* cur_pages;   /* device int32 [chunk_len/page_size] physical ids      */
+  float softmax_scale;        /* usually 1/sqrt(head_dim)                             */
+} oomb_attn_args;
+
+/* Forward with online softmax; writes o and lse. */
+oomb_status oomb_chunk_attn_fwd(oomb_pool* pool, const oomb_attn_args* args, void* stream);
+
+/* Backward of sum(O * dO): writes dq and ADDS dK, dV into the pool's gradient
+ * blocks of every page read (fp32 atomic adds, in place; [it] §2B).  Needs o
+ * and lse from the forward of the same chunk, and delta_ws as workspace. */
+oomb_status oomb_chunk_attn_bwd(oomb_pool* pool, const oomb_attn_args* args, void* stream);
+
+/* The backward's three launches, for timing them separately; running
+ * PREPROCESS, DKDV and DQ in this order equals oomb_chunk_attn_bwd. */
+typedef enum oomb_bwd_step {
+  OOMB_BWD_PREPROCESS = 0, /* delta_ws = rowsum(dO * O)                          */
+  OOMB_BWD_DKDV = 1,       /* grad pool += dK, dV (needs delta_ws)                */
+  OOMB_BWD_DQ = 2          /* dq (needs delta_ws)                                 */
+} oomb_bwd_step;
+oomb_status oomb_chunk_attn_bwd_step(oomb_pool* pool, const oomb_attn_args* args, int32_t step,
+                                     void* stream);
+
+/* ---------------------------------------------------------------- Top-K
+ * Page-level selection for one chunk ([pt] §2C, [es] §2B, [it] §2D):
+ *   q_bar_g   = fp32 mean of the chunk's rows over the G query heads of group g
+ *   score_p,g = q_bar_g . (summary of page p, KV head g)          (fp32)
+ * Candidates are logical pages [0, n_past - n_recent); the top_k highest
+ * scores are kept (ties: lower logical id first), together with the n_recent
+ * most recent pages [n_past - n_recent, n_past).  Output per group: the kept
+ * logical ids in ascending order, their physical ids, and the count
+ * min(top_k, n_past - n_recent) + min(n_recent, n_past).
+ *   d_q              device bf16 [chunk_len][num_q_heads][head_dim]
+ *   d_page_table     device int32 [n_past]: logical -> physical page id
+ *   d_out_logical    device int32 [num_kv_heads][top_k + n_recent]
+ *   d_out_physical   device int32 [num_kv_heads][top_k + n_recent] (may be NULL)
+ *   d_out_count      device int32 [num_kv_heads]
+ *   d_out_scores     device fp32 [num_kv_heads][n_past] (may be NULL)
+ *   d_workspace      device memory of oomb_page_topk_workspace_size() bytes
+ * Limits: n_past <= 65536; top_k + n_recent <= 4096. */
+size_t oomb_page_topk_workspace_size(int32_t chunk_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                     int32_t head_dim, int32_t n_past);
+oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk_len,
+                           int32_t num_q_heads, const int32_t* d_page_table, int32_t n_past,
+                           int32_t top_k, int32_t n_recent, int32_t* d_out_logical,
+                           int32_t* d_out_physical, int32_t* d_out_count, float* d_out_scores,
+                           void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- offload
+ * A block is the K and V of one page and one KV head: block id = page *
+ * num_kv_heads + head, contiguous in both pools ([pt] §2D, [it] §2C: KV and
+ * its gradients move between pinned host memory and the GPU on dedicated
+ * streams, overlapped with compute).
+ *
+ * oomb_page_prefetch: host (pinned) pool -> device pool, one cudaMemcpyAsync
+ * per run of consecutive blocks, on `stream`; records `done_event` (a
+ * cudaEvent_t given as void*, may be NULL) after the last copy.  The two pools
+ * must share page_size, num_kv_heads and head_dim. */
+oomb_status oomb_page_prefetch(const oomb_pool* host_pool, oomb_pool* device_pool,
+                               const int32_t* h_src_blocks, const int32_t* h_dst_blocks,
+                               int32_t n_blocks, void* stream, void* done_event);
+
+/* oomb_grad_writeback: adds the device pool's gradient blocks into the host
+ * pool's gradient blocks.  The blocks are copied device -> host into a
+ * library-owned pinned staging area on `stream`; a host function enqueued on
+ * the same stream then adds them into the host pool with several CPU
+ * threads.  The device blocks are then zero-filled on the stream, ready for
+ * the next chunk's contributions.  Later work on `stream` is ordered after
+ * the add. */
+oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* host_pool,
+                                const int32_t* h_src_blocks, const int32_t* h_dst_blocks,
+                                int32_t n_blocks, void* stream);
+
+/* ---------------------------------------------------------------- status
+ * Waits for a cudaEvent_t (given as void*) by polling, for at most timeout_us
+ * microseconds; OOMB_ERR_TIMEOUT instead of blocking forever. */
+oomb_status oomb_wait(void* event, int64_t timeout_us);
+/* Synchronises with the pool's device, reads and clears its device status
+ * word: OOMB_OK, or OOMB_ERR_DEVICE_CHECK if a kernel recorded a failure.
+ * *out_word (may be NULL) receives the raw bits:
+ *   bit 0 invalid page id, bit 1 wait limit reached, bit 2 bad count. */
+oomb_status oomb_get_device_status(oomb_pool* pool, uint32_t* out_word);
+const char* oomb_status_string(oomb_status status);
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t oomb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* OOMB_H */

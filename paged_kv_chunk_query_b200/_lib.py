@@ -1,0 +1,318 @@
+"""ctypes binding of liboomb.so: argument marshalling only.
+
+Every function here forwards to the C ABI declared in include/oomb.h, taking
+torch tensors for device buffers (their data pointers are passed) and raising
+:class:`OombError` on a non-OK status.  No step of the computation runs here;
+if the shared library is missing or fails to load, importing the package fails
+loudly — there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liboomb.so")
+
+STATUS = {
+    0: "OOMB_OK", 1: "OOMB_ERR_INVALID_ARG", 2: "OOMB_ERR_OUT_OF_PAGES", 3: "OOMB_ERR_BAD_PAGE",
+    4: "OOMB_ERR_CUDA", 5: "OOMB_ERR_TIMEOUT", 6: "OOMB_ERR_UNSUPPORTED",
+    7: "OOMB_ERR_DEVICE_CHECK",
+}
+OK, ERR_INVALID_ARG, ERR_OUT_OF_PAGES, ERR_BAD_PAGE, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED, \
+    ERR_DEVICE_CHECK = range(8)
+LOC_DEVICE, LOC_PINNED_HOST, LOC_HOST = 0, 1, 2
+BWD_PREPROCESS, BWD_DKDV, BWD_DQ = 0, 1, 2
+
+# Every exported symbol of include/oomb.h.
+EXPORTS = (
+    "oomb_pool_create", "oomb_pool_destroy", "oomb_pool_alloc_page", "oomb_pool_free_page",
+    "oomb_pool_num_free", "oomb_pool_buffers", "oomb_pool_get_desc", "oomb_kv_append",
+    "oomb_chunk_attn_fwd", "oomb_chunk_attn_bwd", "oomb_chunk_attn_bwd_step",
+    "oomb_page_topk_workspace_size", "oomb_page_topk", "oomb_page_prefetch",
+    "oomb_grad_writeback", "oomb_wait", "oomb_get_device_status", "oomb_status_string",
+    "oomb_version",
+)
+
+
+class OombError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class PoolDesc(ctypes.Structure):
+    _fields_ = [("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("location", ctypes.c_int32), ("with_grad", ctypes.c_int32),
+                ("alloc_seed", ctypes.c_uint64), ("device", ctypes.c_int32)]
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("d_o", ctypes.c_void_p), ("dq", ctypes.c_void_p),
+                ("delta_ws", ctypes.c_void_p), ("chunk_len", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("past_pages", ctypes.c_void_p),
+                ("past_counts", ctypes.c_void_p), ("max_past", ctypes.c_int32),
+                ("cur_pages", ctypes.c_void_p), ("softmax_scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m paged_kv_chunk_query_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, u64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_float
+    sig = {
+        "oomb_pool_create": [ctypes.POINTER(PoolDesc), ctypes.POINTER(vp)],
+        "oomb_pool_destroy": [vp],
+        "oomb_pool_alloc_page": [vp, ctypes.POINTER(i32)],
+        "oomb_pool_free_page": [vp, i32],
+        "oomb_pool_num_free": [vp, ctypes.POINTER(i32)],
+        "oomb_pool_buffers": [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp)],
+        "oomb_pool_get_desc": [vp, ctypes.POINTER(PoolDesc)],
+        "oomb_kv_append": [vp, vp, i32, vp, vp, vp],
+        "oomb_chunk_attn_fwd": [vp, ctypes.POINTER(AttnArgs), vp],
+        "oomb_chunk_attn_bwd": [vp, ctypes.POINTER(AttnArgs), vp],
+        "oomb_chunk_attn_bwd_step": [vp, ctypes.POINTER(AttnArgs), i32, vp],
+        "oomb_page_topk": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp,
+                           ctypes.c_size_t, vp],
+        "oomb_page_prefetch": [vp, vp, vp, vp, i32, vp, vp],
+        "oomb_grad_writeback": [vp, vp, vp, vp, i32, vp],
+        "oomb_wait": [vp, ctypes.c_int64],
+        "oomb_get_device_status": [vp, ctypes.POINTER(ctypes.c_uint32)],
+    }
+    for name, args in sig.items():
+        if not hasattr(lib, name):  # completeness is checked by the export test
+            continue
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    if hasattr(lib, "oomb_page_topk_workspace_size"):
+        lib.oomb_page_topk_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        lib.oomb_page_topk_workspace_size.restype = ctypes.c_size_t
+    lib.oomb_status_string.argtypes = [ctypes.c_int]
+    lib.oomb_status_string.restype = ctypes.c_char_p
+    lib.oomb_version.argtypes = []
+    lib.oomb_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise OombError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dev_tensor(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+# ------------------------------------------------------------------- pools
+def pool_create(num_pages, page_size, num_kv_heads, head_dim, location=LOC_DEVICE,
+                with_grad=True, alloc_seed=0, device=0) -> int:
+    d = PoolDesc(num_pages, page_size, num_kv_heads, head_dim, location, int(bool(with_grad)),
+                 alloc_seed, device)
+    h = ctypes.c_void_p()
+    _check(load().oomb_pool_create(ctypes.byref(d), ctypes.byref(h)), "oomb_pool_create")
+    return h.value
+
+
+def pool_destroy(pool: int):
+    _check(load().oomb_pool_destroy(pool), "oomb_pool_destroy")
+
+
+def pool_alloc_page(pool: int) -> int:
+    out = ctypes.c_int32()
+    _check(load().oomb_pool_alloc_page(pool, ctypes.byref(out)), "oomb_pool_alloc_page")
+    return out.value
+
+
+def pool_free_page(pool: int, page_id: int):
+    _check(load().oomb_pool_free_page(pool, page_id), "oomb_pool_free_page")
+
+
+def pool_num_free(pool: int) -> int:
+    out = ctypes.c_int32()
+    _check(load().oomb_pool_num_free(pool, ctypes.byref(out)), "oomb_pool_num_free")
+    return out.value
+
+
+def pool_get_desc(pool: int) -> PoolDesc:
+    d = PoolDesc()
+    _check(load().oomb_pool_get_desc(pool, ctypes.byref(d)), "oomb_pool_get_desc")
+    return d
+
+
+def pool_buffers(pool: int):
+    """(kv, grad, summary) raw pointers (0 where absent)."""
+    kv, grad, summ = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    _check(load().oomb_pool_buffers(pool, ctypes.byref(kv), ctypes.byref(grad),
+                                    ctypes.byref(summ)), "oomb_pool_buffers")
+    return kv.value or 0, grad.value or 0, summ.value or 0
+
+
+class _CudaArray:
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"data": (ptr, False), "shape": tuple(shape),
+                                         "typestr": typestr, "version": 3, "strides": None}
+
+
+def pool_views(pool: int):
+    """Torch views (kv, grad, summary) of a device pool's buffers, borrowed: they
+    are valid until pool_destroy.  Host pools give CPU tensors."""
+    d = pool_get_desc(pool)
+    kv, grad, summ = pool_buffers(pool)
+    shape = (d.num_pages, d.num_kv_heads, 2, d.page_size, d.head_dim)
+    sshape = (d.num_pages, d.num_kv_heads, d.head_dim)
+    if d.location == LOC_DEVICE:
+        dev = torch.device("cuda", d.device)
+        t_kv = torch.as_tensor(_CudaArray(kv, shape, "<i2"), device=dev).view(torch.bfloat16)
+        t_g = torch.as_tensor(_CudaArray(grad, shape, "<f4"), device=dev) if grad else None
+        t_s = torch.as_tensor(_CudaArray(summ, sshape, "<f4"), device=dev)
+        return t_kv, t_g, t_s
+
+    def host(ptr, shp, ctype, dt):
+        n = 1
+        for x in shp:
+            n *= x
+        buf = (ctype * n).from_address(ptr)
+        return torch.frombuffer(buf, dtype=dt).view(shp)
+
+    t_kv = host(kv, shape, ctypes.c_int16, torch.int16).view(torch.bfloat16)
+    t_g = host(grad, shape, ctypes.c_float, torch.float32) if grad else None
+    t_s = host(summ, sshape, ctypes.c_float, torch.float32)
+    return t_kv, t_g, t_s
+
+
+# ------------------------------------------------------------------- compute
+def kv_append(pool: int, page_ids: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None):
+    n = page_ids.numel()
+    _check(load().oomb_kv_append(pool, _dev_tensor(page_ids, torch.int32, "page_ids"), n,
+                                 _dev_tensor(k, torch.bfloat16, "k"),
+                                 _dev_tensor(v, torch.bfloat16, "v"), _stream(stream)),
+           "oomb_kv_append")
+
+
+def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o=None, dq=None,
+               delta_ws=None):
+    C, Hq, _ = q.shape
+    max_past = past_pages.shape[1] if past_pages is not None and past_pages.numel() else 0
+    return AttnArgs(
+        _dev_tensor(q, torch.bfloat16, "q"), _dev_tensor(o, torch.bfloat16, "o"),
+        _dev_tensor(lse, torch.float32, "lse"),
+        _dev_tensor(d_o, torch.bfloat16, "d_o") if d_o is not None else None,
+        _dev_tensor(dq, torch.bfloat16, "dq") if dq is not None else None,
+        _dev_tensor(delta_ws, torch.float32, "delta_ws") if delta_ws is not None else None,
+        C, Hq,
+        _dev_tensor(past_pages, torch.int32, "past_pages") if max_past else None,
+        _dev_tensor(past_counts, torch.int32, "past_counts") if max_past else None,
+        max_past, _dev_tensor(cur_pages, torch.int32, "cur_pages"), softmax_scale)
+
+
+def chunk_attn_fwd(pool, q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
+                   stream=None):
+    a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale)
+    _check(load().oomb_chunk_attn_fwd(pool, ctypes.byref(a), _stream(stream)),
+           "oomb_chunk_attn_fwd")
+
+
+def chunk_attn_bwd(pool, q, o, lse, d_o, dq, delta_ws, past_pages, past_counts, cur_pages,
+                   softmax_scale, stream=None, step=None):
+    a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o, dq,
+                   delta_ws)
+    if step is None:
+        _check(load().oomb_chunk_attn_bwd(pool, ctypes.byref(a), _stream(stream)),
+               "oomb_chunk_attn_bwd")
+    else:
+        _check(load().oomb_chunk_attn_bwd_step(pool, ctypes.byref(a), step, _stream(stream)),
+               "oomb_chunk_attn_bwd_step")
+
+
+def page_topk_workspace_size(chunk_len, num_q_heads, num_kv_heads, head_dim, n_past) -> int:
+    return load().oomb_page_topk_workspace_size(chunk_len, num_q_heads, num_kv_heads, head_dim,
+                                                n_past)
+
+
+def page_topk(pool, q, page_table, n_past, top_k, n_recent, out_logical, out_physical,
+              out_count, workspace, out_scores=None, stream=None):
+    C, Hq, _ = q.shape
+    _check(load().oomb_page_topk(
+        pool, _dev_tensor(q, torch.bfloat16, "q"), C, Hq,
+        _dev_tensor(page_table, torch.int32, "page_table") if n_past else None, n_past, top_k,
+        n_recent, _dev_tensor(out_logical, torch.int32, "out_logical"),
+        _dev_tensor(out_physical, torch.int32, "out_physical") if out_physical is not None
+        else None, _dev_tensor(out_count, torch.int32, "out_count"),
+        _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
+        _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "oomb_page_topk")
+
+
+def _host_i32(blocks):
+    t = torch.as_tensor(blocks, dtype=torch.int32).contiguous()
+    return t, t.data_ptr()
+
+
+def page_prefetch(host_pool, device_pool, src_blocks, dst_blocks, stream=None, done_event=None):
+    s, sp = _host_i32(src_blocks)
+    d, dp = _host_i32(dst_blocks)
+    ev = done_event.cuda_event if done_event is not None else None
+    _check(load().oomb_page_prefetch(host_pool, device_pool, sp, dp, s.numel(), _stream(stream),
+                                     ev), "oomb_page_prefetch")
+
+
+def grad_writeback(device_pool, host_pool, src_blocks, dst_blocks, stream=None):
+    s, sp = _host_i32(src_blocks)
+    d, dp = _host_i32(dst_blocks)
+    _check(load().oomb_grad_writeback(device_pool, host_pool, sp, dp, s.numel(),
+                                      _stream(stream)), "oomb_grad_writeback")
+
+
+def wait(event, timeout_us: int):
+    _check(load().oomb_wait(event.cuda_event, timeout_us), "oomb_wait")
+
+
+def get_device_status(pool) -> int:
+    w = ctypes.c_uint32()
+    st = load().oomb_get_device_status(pool, ctypes.byref(w))
+    if st not in (OK, ERR_DEVICE_CHECK):
+        raise OombError(st, "oomb_get_device_status")
+    return w.value
+
+
+def status_string(status: int) -> str:
+    return load().oomb_status_string(status).decode()
+
+
+def version() -> int:
+    return load().oomb_version()

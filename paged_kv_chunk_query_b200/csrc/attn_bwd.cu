@@ -1,0 +1,748 @@
+// Chunk attention backward over the paged KV cache (tcgen05 + TMA, sm_100a).
+//
+// "Out of the Memory Barrier" ([pt] §2B "Kernels Personalizados": gradients
+// accumulated in place, outside autograd; [es] §2B: the operators are opaque
+// to autograd and need no intermediate buffers; [it] §2B: in-place
+// accumulation with atomic_add).  For the loss sum(O * dO):
+//   D_i  = dO_i . O_i                         (preprocess)
+//   P_ij = exp(S_ij - LSE_i),  dS_ij = P_ij (dO_i . v_j - D_i)
+//   dK_j += scale sum_i dS_ij q_i,  dV_j += sum_i P_ij dO_i   (KV-major kernel,
+//           summed over every query head of the group, then added into the
+//           fp32 gradient pool with vector atomics)
+//   dQ_i  = scale sum_j dS_ij k_j                               (Q-major kernel)
+// The dQ kernel recomputes S and dP rather than reducing dQ across KV tiles:
+// the chunk's rows are few (C * G per group) and the keys many, so a KV-major
+// dQ would need a large reduction per chunk.
+#include "internal.h"
+#include "ptx.cuh"
+#include "tiles.cuh"
+#include "tmap.h"
+
+namespace {
+
+using namespace oomb;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+  const __nv_bfloat16* o;
+  const __nv_bfloat16* d_o;
+  const float* lse;
+  float* delta;
+  __nv_bfloat16* dq;
+  float* grad;
+  const int32_t* past_pages;
+  const int32_t* past_counts;
+  const int32_t* cur_pages;
+  uint32_t* status;
+  int max_past, C, Hq, Hkv, G, P, num_pool_pages, max_past_tiles;
+  float scale, scale_log2;
+};
+
+// ------------------------------------------------------------------ preprocess
+// delta[h][q] = sum_d dO[q][h][d] * O[q][h][d], fp32; D/8 lanes per row, 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) {
+  constexpr int LPR = D / 8;
+  constexpr int RPB = 256 / LPR;  // rows per block per pass
+  const int t = threadIdx.x;
+  const int row = blockIdx.x * RPB + t / LPR;
+  const int sub = t % LPR;
+  const int rows = p.C * p.Hq;
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p.o + static_cast<size_t>(row) * D + sub * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(p.d_o + static_cast<size_t>(row) * D + sub * 8);
+    const __nv_bfloat16* av = reinterpret_cast<const __nv_bfloat16*>(&a);
+    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc += __bfloat162float(av[e]) * __bfloat162float(bv[e]);
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && sub == 0) {
+    const int q = row / p.Hq, h = row % p.Hq;
+    p.delta[static_cast<size_t>(h) * p.C + q] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ dK / dV
+// One CTA per (KV tile of 128 keys, KV head g); loops over the group's query
+// tiles (G heads x 128-row tiles; for the chunk's own keys only the causally
+// reachable tiles).  Thread r of warps 0-3 owns key r (TMEM lane r).
+// TMEM: S^T [0,128) (then P^T bf16 in [0,64)), dP^T [128,256) (then dS^T in
+// [128,192)), dV [256,256+D), dK [256+D, 256+2D).
+template <int D>
+struct KvCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kNS = 2;
+  static constexpr int kStageBytes = 2 * kTileBytes + 1024;  // Q, dO, LSE[128], delta[128]
+  static constexpr int kSmem = 2 * kTileBytes + kNS * kStageBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dkdv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap domap,
+                    const __grid_constant__ CUtensorMap kvmap) {
+  using Cfg = KvCfg<D>;
+  const int g = blockIdx.y;
+  const KvSchedule sch = kv_schedule(p.past_counts, g, p.max_past, p.P, p.status);
+  const bool is_past = static_cast<int>(blockIdx.x) < p.max_past_tiles;
+  if (is_past && static_cast<int>(blockIdx.x) >= sch.n_past_tiles) return;  // beyond the list
+  const int u = is_past ? 0 : static_cast<int>(blockIdx.x) - p.max_past_tiles;  // current tile
+  const int j = is_past ? static_cast<int>(blockIdx.x) : sch.n_past_tiles + u;    // schedule index
+  const int n_qtiles = (p.C + kTile - 1) / kTile;
+  const int t0 = is_past ? 0 : u;  // first query tile that can see these keys
+  const int n_qt = n_qtiles - t0;
+  const int n_iter = p.G * n_qt;
+  const int n_cur_pages = p.C / p.P;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + Cfg::kTileBytes;
+  uint8_t* sStage = sV + Cfg::kTileBytes;
+  auto sQ = [&](int s) { return sStage + s * Cfg::kStageBytes; };
+  auto sDO = [&](int s) { return sStage + s * Cfg::kStageBytes + Cfg::kTileBytes; };
+  auto sL = [&](int s) {
+    return reinterpret_cast<float*>(sStage + s * Cfg::kStageBytes + 2 * Cfg::kTileBytes);
+  };
+  auto sDl = [&](int s) {
+    return reinterpret_cast<float*>(sStage + s * Cfg::kStageBytes + 2 * Cfg::kTileBytes + 512);
+  };
+
+  __shared__ uint64_t bar_kv, bar_qf[Cfg::kNS], bar_qe[Cfg::kNS];
+  __shared__ uint64_t bar_st, bar_dpt, bar_p, bar_ds, bar_acc, bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh, q_issued_sh, q_used_sh, kv_issued_sh;
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    q_issued_sh = q_used_sh = kv_issued_sh = 0;
+    mbar_init(&bar_kv, 1);
+    for (int i = 0; i < Cfg::kNS; ++i) {
+      mbar_init(&bar_qf[i], 1);
+      mbar_init(&bar_qe[i], 1);
+    }
+    mbar_init(&bar_st, 1);
+    mbar_init(&bar_dpt, 1);
+    mbar_init(&bar_p, 4);
+    mbar_init(&bar_ds, 4);
+    mbar_init(&bar_acc, 1);
+    mbar_init(&bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int32_t* past_list = p.past_pages ? p.past_pages + static_cast<size_t>(g) * p.max_past
+                                          : nullptr;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&domap);
+      prefetch_tensormap(&kvmap);
+      const int per = kTile / p.P;
+      mbar_arrive_expect_tx(&bar_kv, 2 * Cfg::kTileBytes);
+      for (int s = 0; s < per; ++s) {
+        const int pg = tile_page(j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
+                                 p.num_pool_pages, p.status);
+        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+          tma_load_4d(sK + hf * kTile * 128 + s * p.P * 128, &kvmap, &bar_kv, hf * 64, 0, 2 * g,
+                      pg);
+          tma_load_4d(sV + hf * kTile * 128 + s * p.P * 128, &kvmap, &bar_kv, hf * 64, 0,
+                      2 * g + 1, pg);
+        }
+      }
+      kv_issued_sh = 1;
+      int issued = 0;
+      for (int i = 0; i < n_iter; ++i) {
+        const int s = i % Cfg::kNS;
+        const int head = g * p.G + i / n_qt, t = t0 + i % n_qt;
+        const int nvalid = min(kTile, p.C - t * kTile);
+        if (!mbar_wait(&bar_qe[s], ((i / Cfg::kNS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bar_qf[s], 2 * Cfg::kTileBytes + 2 * nvalid * 4);
+        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+          tma_load_3d(sQ(s) + hf * kTile * 128, &qmap, &bar_qf[s], hf * 64, head, t * kTile);
+          tma_load_3d(sDO(s) + hf * kTile * 128, &domap, &bar_qf[s], hf * 64, head, t * kTile);
+        }
+        const size_t row0 = static_cast<size_t>(head) * p.C + t * kTile;
+        bulk_load(sL(s), p.lse + row0, nvalid * 4, &bar_qf[s]);
+        bulk_load(sDl(s), p.delta + row0, nvalid * 4, &bar_qf[s]);
+        ++issued;
+      }
+      if (*abort_flag) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+      q_issued_sh = issued;
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      int used = 0;
+      bool ok = mbar_wait(&bar_kv, 0, abort_flag);
+      for (int i = 0; ok && i < n_iter; ++i) {
+        const int s = i % Cfg::kNS;
+        if (!(ok = mbar_wait(&bar_qf[s], (i / Cfg::kNS) & 1, abort_flag))) break;
+        ++used;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ(s)), do_addr = smem_u32(sDO(s));
+        // S^T_i = K Q_i^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+          umma_ss(tmem + Cfg::kColST, sw128_desc(k_addr + off, 16, 1024),
+                  sw128_desc(q_addr + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&bar_st);
+        if (i > 0) {
+          // dK += dS^T_{i-1} Q_{i-1}
+          if (!(ok = mbar_wait(&bar_ds, (i - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const int sp = (i - 1) % Cfg::kNS;
+          const uint32_t qp = smem_u32(sQ(sp));
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPT + kk * 8,
+                    sw128_desc(qp + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
+                    (i - 1 > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bar_qe[sp]);
+        }
+        // dP^T_i = V dO_i^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+          umma_ss(tmem + Cfg::kColDPT, sw128_desc(v_addr + off, 16, 1024),
+                  sw128_desc(do_addr + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&bar_dpt);
+        // dV += P^T_i dO_i
+        if (!(ok = mbar_wait(&bar_p, i & 1, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColST + kk * 8,
+                  sw128_desc(do_addr + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      if (ok && n_iter > 0) {
+        const int i = n_iter;
+        if ((ok = mbar_wait(&bar_ds, (i - 1) & 1, abort_flag))) {
+          tc_fence_after();
+          const int sp = (i - 1) % Cfg::kNS;
+          const uint32_t qp = smem_u32(sQ(sp));
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPT + kk * 8,
+                    sw128_desc(qp + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
+                    (i - 1 > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bar_qe[sp]);
+          umma_commit(&bar_acc);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+      }
+      umma_commit(&bar_drain);
+      mbar_wait_drain(&bar_drain, 0);
+      q_used_sh = used;
+    }
+  } else {
+    const int r = threadIdx.x;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    bool key_valid;
+    if (is_past) key_valid = j * kTile + r < sch.n_past_pages * p.P;
+    else key_valid = u * kTile + r < p.C;
+    const int key_local = u * kTile + r;  // causal position (current tiles only)
+    bool ok = true;
+    for (int i = 0; i < n_iter; ++i) {
+      const int s = i % Cfg::kNS;
+      const int t = t0 + i % n_qt;
+      if (!(ok = warp_wait(&bar_st, i & 1, abort_flag))) break;
+      if (!(ok = warp_wait(&bar_qf[s], (i / Cfg::kNS) & 1, abort_flag))) break;
+      tc_fence_after();
+      float pr[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c)
+        tmem_ld32(tmem + lane_off + Cfg::kColST + c * 32, reinterpret_cast<uint32_t*>(pr + c * 32));
+      tmem_ld_wait();
+      const float* L = sL(s);
+      // query column c is valid if inside the chunk and (current tile) causally after the key
+      int cmax = min(kTile, p.C - t * kTile);  // columns [0, cmax) are inside the chunk
+      int cmin = 0;
+      if (!is_past) cmin = key_local - t * kTile;  // q_local >= key_local
+      uint32_t pk[kTile / 2];
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const bool v = key_valid && c < cmax && c >= cmin;
+        const float e = fast_exp2(fmaf(pr[c], p.scale_log2, -L[c] * kLog2e));
+        pr[c] = v ? e : 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < kTile / 2; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+#pragma unroll
+      for (int c = 0; c < kTile / 2 / 16; ++c)
+        tmem_st16(tmem + lane_off + Cfg::kColST + c * 16, pk + c * 16);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p);
+
+      if (!(ok = warp_wait(&bar_dpt, i & 1, abort_flag))) break;
+      tc_fence_after();
+      const float* Dl = sDl(s);
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c) {
+        uint32_t dp[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColDPT + c * 32, dp);
+        tmem_ld_wait();
+        uint32_t dk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = c * 32 + 2 * e;
+          float a = pr[c0] * (__uint_as_float(dp[2 * e]) - Dl[c0]);
+          float b = pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - Dl[c0 + 1]);
+          a = pr[c0] != 0.f ? a : 0.f;
+          b = pr[c0 + 1] != 0.f ? b : 0.f;
+          dk[e] = pack_bf16(a, b);
+        }
+        tmem_st16(tmem + lane_off + Cfg::kColDPT + c * 16, dk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_ds);
+    }
+    if (ok && n_iter > 0) ok = warp_wait(&bar_acc, 0, abort_flag);
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+    } else if (n_iter > 0) {
+      tc_fence_after();
+      int page = -1;
+      if (key_valid)
+        page = tile_page(j, r / p.P, sch, past_list, p.cur_pages, n_cur_pages, p.P,
+                         p.num_pool_pages, p.status);
+      const bool write = key_valid && page >= 0 && page < p.num_pool_pages;
+      const size_t blk = (static_cast<size_t>(write ? page : 0) * p.Hkv + g) * 2;
+      float* gk = p.grad + (blk * p.P + r % p.P) * D;
+      float* gv = p.grad + ((blk + 1) * p.P + r % p.P) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColDK + c * 32, a);
+        tmem_ld32(tmem + lane_off + Cfg::kColDV + c * 32, b);
+        tmem_ld_wait();
+        if (write) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            atomicAdd(reinterpret_cast<float4*>(gk + c * 32 + 4 * e),
+                      make_float4(__uint_as_float(a[4 * e]) * p.scale,
+                                  __uint_as_float(a[4 * e + 1]) * p.scale,
+                                  __uint_as_float(a[4 * e + 2]) * p.scale,
+                                  __uint_as_float(a[4 * e + 3]) * p.scale));
+            atomicAdd(reinterpret_cast<float4*>(gv + c * 32 + 4 * e),
+                      make_float4(__uint_as_float(b[4 * e]), __uint_as_float(b[4 * e + 1]),
+                                  __uint_as_float(b[4 * e + 2]), __uint_as_float(b[4 * e + 3])));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4 && lane == 0) {
+    // Loads that were issued but never consumed must land before the CTA exits.
+    if (kv_issued_sh && (abort_sh || n_iter == 0)) mbar_wait_drain(&bar_kv, 0);
+    if (abort_sh)
+      for (int i = q_used_sh; i < q_issued_sh; ++i)
+        mbar_wait_drain(&bar_qf[i % Cfg::kNS], (i / Cfg::kNS) & 1);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+// One CTA per (128-row query tile, head).  TMEM: S0 [0,128), S1 [128,256),
+// dP [256,384) (then dS bf16 in [256,320)), dQ [384, 384+D).
+template <int D>
+struct QCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kNK = 2, kNV = 2;
+  static constexpr int kSmem = kTileBytes * (2 + kNK + kNV) + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColDP = 256, kColDQ = 384;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap qmap,
+                  const __grid_constant__ CUtensorMap domap,
+                  const __grid_constant__ CUtensorMap kvmap) {
+  using Cfg = QCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = sQ + Cfg::kTileBytes;
+  uint8_t* sK = sDO + Cfg::kTileBytes;
+  uint8_t* sV = sK + Cfg::kNK * Cfg::kTileBytes;
+
+  __shared__ uint64_t bar_q, bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV],
+      bar_ve[Cfg::kNV];
+  __shared__ uint64_t bar_s[2], bar_dp, bar_ds, bar_fin, bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh, k_issued_sh, v_issued_sh, k_used_sh, v_used_sh;
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = blockIdx.x, h = blockIdx.y, g = h / p.G;
+  const KvSchedule sch = kv_schedule(p.past_counts, g, p.max_past, p.P, p.status);
+  const int T = sch.n_past_tiles + qt + 1;
+  const int n_cur_pages = p.C / p.P;
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    k_issued_sh = v_issued_sh = k_used_sh = v_used_sh = 0;
+    mbar_init(&bar_q, 1);
+    for (int i = 0; i < Cfg::kNK; ++i) {
+      mbar_init(&bar_kf[i], 1);
+      mbar_init(&bar_ke[i], 1);
+    }
+    for (int i = 0; i < Cfg::kNV; ++i) {
+      mbar_init(&bar_vf[i], 1);
+      mbar_init(&bar_ve[i], 1);
+    }
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
+    mbar_init(&bar_dp, 1);
+    mbar_init(&bar_ds, 4);
+    mbar_init(&bar_fin, 1);
+    mbar_init(&bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&domap);
+      prefetch_tensormap(&kvmap);
+      const int32_t* past_list =
+          p.past_pages ? p.past_pages + static_cast<size_t>(g) * p.max_past : nullptr;
+      const int per = kTile / p.P;
+      mbar_arrive_expect_tx(&bar_q, 2 * Cfg::kTileBytes);
+      for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+        tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
+        tma_load_3d(sDO + hf * kTile * 128, &domap, &bar_q, hf * 64, h, qt * kTile);
+      }
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < T; ++j) {
+        int pg[8];
+        for (int s = 0; s < per; ++s)
+          pg[s] = tile_page(j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
+                            p.num_pool_pages, p.status);
+        const int ks = j % Cfg::kNK;
+        if (!mbar_wait(&bar_ke[ks], ((j / Cfg::kNK) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bar_kf[ks], Cfg::kTileBytes);
+        for (int s = 0; s < per; ++s)
+          for (int hf = 0; hf < Cfg::kHalves; ++hf)
+            tma_load_4d(sK + ks * Cfg::kTileBytes + hf * kTile * 128 + s * p.P * 128, &kvmap,
+                        &bar_kf[ks], hf * 64, 0, 2 * g, pg[s]);
+        ++k_issued;
+        const int vs = j % Cfg::kNV;
+        if (!mbar_wait(&bar_ve[vs], ((j / Cfg::kNV) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bar_vf[vs], Cfg::kTileBytes);
+        for (int s = 0; s < per; ++s)
+          for (int hf = 0; hf < Cfg::kHalves; ++hf)
+            tma_load_4d(sV + vs * Cfg::kTileBytes + hf * kTile * 128 + s * p.P * 128, &kvmap,
+                        &bar_vf[vs], hf * 64, 0, 2 * g + 1, pg[s]);
+        ++v_issued;
+      }
+      if (*abort_flag) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+      k_issued_sh = k_issued;
+      v_issued_sh = v_issued;
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      int k_used = 0, v_used = 0;
+      auto issue_s = [&](int j) -> bool {
+        const int ks = j % Cfg::kNK;
+        if (!mbar_wait(&bar_kf[ks], (j / Cfg::kNK) & 1, abort_flag)) return false;
+        ++k_used;
+        tc_fence_after();
+        const uint32_t kb = k_addr + ks * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+          umma_ss(tmem + (j & 1) * 128, sw128_desc(q_addr + off, 16, 1024),
+                  sw128_desc(kb + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&bar_s[j & 1]);
+        return true;
+      };
+      auto issue_dp = [&](int j) -> bool {
+        const int vs = j % Cfg::kNV;
+        if (!mbar_wait(&bar_vf[vs], (j / Cfg::kNV) & 1, abort_flag)) return false;
+        ++v_used;
+        tc_fence_after();
+        const uint32_t vb = v_addr + vs * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+          umma_ss(tmem + Cfg::kColDP, sw128_desc(do_addr + off, 16, 1024),
+                  sw128_desc(vb + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&bar_ve[vs]);
+        umma_commit(&bar_dp);
+        return true;
+      };
+      bool ok = mbar_wait(&bar_q, 0, abort_flag);
+      ok = ok && issue_s(0) && issue_dp(0);
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T && !(ok = issue_s(j + 1))) break;
+        if (!(ok = mbar_wait(&bar_ds, j & 1, abort_flag))) break;
+        tc_fence_after();
+        const int ks = j % Cfg::kNK;
+        const uint32_t kb = k_addr + ks * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * 8,
+                  sw128_desc(kb + kk * 16 * 128, kTile * 128, 1024), idesc_dq,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bar_ke[ks]);
+        if (j + 1 < T && !(ok = issue_dp(j + 1))) break;
+      }
+      if (ok) umma_commit(&bar_fin);
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+      }
+      umma_commit(&bar_drain);
+      mbar_wait_drain(&bar_drain, 0);
+      k_used_sh = k_used;
+      v_used_sh = v_used;
+    }
+  } else {
+    const int r = threadIdx.x;
+    const int q_local = qt * kTile + r;
+    const bool row_valid = q_local < p.C;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float lse2 = row_valid ? p.lse[static_cast<size_t>(h) * p.C + q_local] * kLog2e : 0.f;
+    const float dl = row_valid ? p.delta[static_cast<size_t>(h) * p.C + q_local] : 0.f;
+    const int n_past_keys = sch.n_past_pages * p.P;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int b = j & 1;
+      if (!(ok = warp_wait(&bar_s[b], (j >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      float pr[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c)
+        tmem_ld32(tmem + lane_off + b * 128 + c * 32, reinterpret_cast<uint32_t*>(pr + c * 32));
+      tmem_ld_wait();
+      int lim;
+      if (j < sch.n_past_tiles) lim = n_past_keys - j * kTile;
+      else lim = min(p.C, q_local + 1) - (j - sch.n_past_tiles) * kTile;
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const float e = fast_exp2(fmaf(pr[c], p.scale_log2, -lse2));
+        pr[c] = (c < lim && row_valid) ? e : 0.f;
+      }
+      if (!(ok = warp_wait(&bar_dp, j & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c) {
+        uint32_t dp[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + c * 32, dp);
+        tmem_ld_wait();
+        uint32_t ds[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = c * 32 + 2 * e;
+          ds[e] = pack_bf16(pr[c0] * (__uint_as_float(dp[2 * e]) - dl),
+                            pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - dl));
+        }
+        tmem_st16(tmem + lane_off + Cfg::kColDP + c * 16, ds);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_ds);
+    }
+    if (ok) ok = warp_wait(&bar_fin, 0, abort_flag);
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+    } else {
+      tc_fence_after();
+      __nv_bfloat16* row = p.dq + (static_cast<size_t>(q_local) * p.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColDQ + c * 32, a);
+        tmem_ld_wait();
+        if (row_valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16(__uint_as_float(a[2 * e]) * p.scale,
+                              __uint_as_float(a[2 * e + 1]) * p.scale);
+          uint4* dst = reinterpret_cast<uint4*>(row + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_sh && warp == 4 && lane == 0) {
+    for (int i = k_used_sh; i < k_issued_sh; ++i)
+      mbar_wait_drain(&bar_kf[i % Cfg::kNK], (i / Cfg::kNK) & 1);
+    for (int i = v_used_sh; i < v_issued_sh; ++i)
+      mbar_wait_drain(&bar_vf[i % Cfg::kNV], (i / Cfg::kNV) & 1);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host
+bool make_row_map(CUtensorMap* m, const void* base, int D, int Hq, int C) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(Hq),
+                            static_cast<uint64_t>(C)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hq) * D * 2};
+  const uint32_t box[3] = {64, 1, kTile};
+  return make_bf16_map(m, base, 3, dims, strides, box);
+}
+
+bool make_pool_map(CUtensorMap* m, const oomb_pool* pool) {
+  const oomb_pool_desc& d = pool->desc;
+  const int D = d.head_dim;
+  const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(d.page_size),
+                            static_cast<uint64_t>(2 * d.num_kv_heads),
+                            static_cast<uint64_t>(d.num_pages)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2,
+                               static_cast<uint64_t>(d.page_size) * D * 2,
+                               static_cast<uint64_t>(2 * d.num_kv_heads) * d.page_size * D * 2};
+  const uint32_t box[4] = {64, static_cast<uint32_t>(d.page_size), 1, 1};
+  return make_bf16_map(m, pool->kv, 4, dims, strides, box);
+}
+
+template <int D>
+oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape& s, int step,
+                       cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             KvCfg<D>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             QCfg<D>::kSmem) != cudaSuccess)
+      return OOMB_ERR_CUDA;
+    attr_set = true;
+  }
+  BwdParams p;
+  p.o = static_cast<const __nv_bfloat16*>(a->o);
+  p.d_o = static_cast<const __nv_bfloat16*>(a->d_o);
+  p.lse = a->lse;
+  p.delta = a->delta_ws;
+  p.dq = static_cast<__nv_bfloat16*>(a->dq);
+  p.grad = pool->grad;
+  p.past_pages = a->past_pages;
+  p.past_counts = a->past_counts;
+  p.cur_pages = a->cur_pages;
+  p.status = pool->d_status;
+  p.max_past = a->max_past;
+  p.C = s.C;
+  p.Hq = s.Hq;
+  p.Hkv = s.Hkv;
+  p.G = s.G;
+  p.P = s.P;
+  p.num_pool_pages = pool->desc.num_pages;
+  p.max_past_tiles = (a->max_past * s.P + kTile - 1) / kTile;
+  p.scale = a->softmax_scale;
+  p.scale_log2 = a->softmax_scale * kLog2e;
+
+  if (step < 0 || step == OOMB_BWD_PREPROCESS) {
+    constexpr int RPB = 256 / (D / 8);
+    const int rows = s.C * s.Hq;
+    bwd_preprocess_kernel<D><<<(rows + RPB - 1) / RPB, 256, 0, stream>>>(p);
+    if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+  }
+  if (step < 0 || step == OOMB_BWD_DKDV || step == OOMB_BWD_DQ) {
+    CUtensorMap qmap, domap, kvmap;
+    if (!make_row_map(&qmap, a->q, D, s.Hq, s.C) || !make_row_map(&domap, a->d_o, D, s.Hq, s.C) ||
+        !make_pool_map(&kvmap, pool))
+      return OOMB_ERR_CUDA;
+    if (step < 0 || step == OOMB_BWD_DKDV) {
+      dim3 grid(p.max_past_tiles + s.n_qtiles, s.Hkv);
+      bwd_dkdv_kernel<D><<<grid, 192, KvCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
+      if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+    }
+    if (step < 0 || step == OOMB_BWD_DQ) {
+      dim3 grid(s.n_qtiles, s.Hq);
+      bwd_dq_kernel<D><<<grid, 192, QCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
+      if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+    }
+  }
+  return OOMB_OK;
+}
+
+oomb_status bwd_entry(oomb_pool* pool, const oomb_attn_args* args, int step, void* stream) {
+  AttnShape s;
+  oomb_status st = validate_attn(pool, args, true, &s);
+  if (st != OOMB_OK) return st;
+  if (!aligned16(args->lse) || !aligned16(args->delta_ws)) return OOMB_ERR_INVALID_ARG;
+  DeviceGuard guard(pool->desc.device);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return s.D == 128 ? launch_bwd<128>(pool, args, s, step, cs)
+                    : launch_bwd<64>(pool, args, s, step, cs);
+}
+
+}  // namespace
+
+extern "C" oomb_status oomb_chunk_attn_bwd(oomb_pool* pool, const oomb_attn_args* args,
+                                           void* stream) {
+  return bwd_entry(pool, args, -1, stream);
+}
+
+extern "C" oomb_status oomb_chunk_attn_bwd_step(oomb_pool* pool, const oomb_attn_args* args,
+                                                int32_t step, void* stream) {
+  if (step < OOMB_BWD_PREPROCESS || step > OOMB_BWD_DQ) return OOMB_ERR_INVALID_ARG;
+  return bwd_entry(pool, args, step, stream);
+}

@@ -1,0 +1,381 @@
+// Chunk attention forward over the paged KV cache (tcgen05 + TMA, sm_100a).
+//
+// "Out of the Memory Barrier" ([pt] §2B "Kernels Personalizados"; [es] §2B;
+// [it] §2B): attention runs directly on the paged cache.  One CTA owns 128
+// query rows of one head and walks the KV tiles of its group: the listed past
+// pages (all visible) and then the chunk's own pages (causal).
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Reads S from
+//              TMEM, keeps the running max / sum, writes P (bf16) back into the
+//              same TMEM columns, rescales O when the max grows, and finally
+//              normalises O and writes O and the LSE.
+//   warp 4     TMA producer: Q once, then K and V tiles page by page through
+//              a 4-D tensor map over the pool (page id = outermost coordinate).
+//   warp 5     UMMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
+//              buffers, O += P_j V_j with P read from TMEM (A operand) and V
+//              from shared memory (MN-major B operand).
+// TMEM: S0 [0,128), S1 [128,256), O [256, 256+D).
+//
+// Online softmax in base 2: s2 = S * scale * log2(e).  The running maximum is
+// only moved when a tile's maximum exceeds it by more than 8 (a factor 256),
+// so O is rescaled rarely; the final O / l and LSE = ln2 * (m + log2 l) are
+// exact whichever maximum was used.
+#include "internal.h"
+#include "ptx.cuh"
+#include "tiles.cuh"
+#include "tmap.h"
+
+namespace {
+
+using namespace oomb;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  const int32_t* past_pages;
+  const int32_t* past_counts;
+  const int32_t* cur_pages;
+  uint32_t* status;
+  int max_past, C, Hq, G, P, num_pool_pages;
+  float scale_log2;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kTile * D * 2;  // Q, K or V tile
+  static constexpr int kNK = 3;
+  static constexpr int kNV = 2;
+  static constexpr int kSmem = kTileBytes * (1 + kNK + kNV) + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColO = 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap kvmap) {
+  using Cfg = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + Cfg::kTileBytes;
+  uint8_t* sV = sK + Cfg::kNK * Cfg::kTileBytes;
+
+  __shared__ uint64_t bar_q, bar_drain, bar_o, bar_fin;
+  __shared__ uint64_t bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV], bar_ve[Cfg::kNV];
+  __shared__ uint64_t bar_s[2], bar_p[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ int k_issued_sh, v_issued_sh, k_used_sh, v_used_sh;
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = blockIdx.x, h = blockIdx.y, g = h / p.G;
+  const KvSchedule sch = kv_schedule(p.past_counts, g, p.max_past, p.P, p.status);
+  const int T = sch.n_past_tiles + qt + 1;  // past tiles + current tiles up to the diagonal
+  const int n_cur_pages = p.C / p.P;
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    k_issued_sh = v_issued_sh = k_used_sh = v_used_sh = 0;
+    mbar_init(&bar_q, 1);
+    mbar_init(&bar_drain, 1);
+    mbar_init(&bar_o, 1);
+    mbar_init(&bar_fin, 1);
+    for (int i = 0; i < Cfg::kNK; ++i) {
+      mbar_init(&bar_kf[i], 1);
+      mbar_init(&bar_ke[i], 1);
+    }
+    for (int i = 0; i < Cfg::kNV; ++i) {
+      mbar_init(&bar_vf[i], 1);
+      mbar_init(&bar_ve[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&kvmap);
+      const int32_t* past_list = p.past_pages + static_cast<size_t>(g) * p.max_past;
+      const int per = kTile / p.P;
+      mbar_arrive_expect_tx(&bar_q, Cfg::kTileBytes);
+      for (int hf = 0; hf < Cfg::kHalves; ++hf)
+        tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < T; ++j) {
+        int pg[8];
+        for (int s = 0; s < per; ++s)
+          pg[s] = tile_page(j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
+                            p.num_pool_pages, p.status);
+        const int ks = j % Cfg::kNK;
+        if (!mbar_wait(&bar_ke[ks], ((j / Cfg::kNK) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bar_kf[ks], Cfg::kTileBytes);
+        uint8_t* kdst = sK + ks * Cfg::kTileBytes;
+        for (int s = 0; s < per; ++s)
+          for (int hf = 0; hf < Cfg::kHalves; ++hf)
+            tma_load_4d(kdst + hf * kTile * 128 + s * p.P * 128, &kvmap, &bar_kf[ks], hf * 64, 0,
+                        2 * g, pg[s]);
+        ++k_issued;
+        const int vs = j % Cfg::kNV;
+        if (!mbar_wait(&bar_ve[vs], ((j / Cfg::kNV) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bar_vf[vs], Cfg::kTileBytes);
+        uint8_t* vdst = sV + vs * Cfg::kTileBytes;
+        for (int s = 0; s < per; ++s)
+          for (int hf = 0; hf < Cfg::kHalves; ++hf)
+            tma_load_4d(vdst + hf * kTile * 128 + s * p.P * 128, &kvmap, &bar_vf[vs], hf * 64, 0,
+                        2 * g + 1, pg[s]);
+        ++v_issued;
+      }
+      if (*abort_flag) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+      k_issued_sh = k_issued;
+      v_issued_sh = v_issued;
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      int k_used = 0, v_used = 0;
+      bool ok = mbar_wait(&bar_q, 0, abort_flag);
+      for (int j = 0; ok && j <= T; ++j) {
+        if (j < T) {
+          const int ks = j % Cfg::kNK;
+          if (!(ok = mbar_wait(&bar_kf[ks], (j / Cfg::kNK) & 1, abort_flag))) break;
+          ++k_used;
+          tc_fence_after();
+          const uint32_t sd = tmem + (j & 1) * 128;
+          const uint32_t kb = k_addr + ks * Cfg::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+            umma_ss(sd, sw128_desc(q_addr + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+                    idesc_s, kk > 0);
+          }
+          umma_commit(&bar_ke[ks]);
+          umma_commit(&bar_s[j & 1]);
+        }
+        if (j >= 1) {
+          const int jp = j - 1, b = jp & 1, vs = jp % Cfg::kNV;
+          if (!(ok = mbar_wait(&bar_p[b], (jp >> 1) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&bar_vf[vs], (jp / Cfg::kNV) & 1, abort_flag))) break;
+          ++v_used;
+          tc_fence_after();
+          const uint32_t vb = v_addr + vs * Cfg::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tmem + Cfg::kColO, tmem + b * 128 + kk * 8,
+                    sw128_desc(vb + kk * 16 * 128, kTile * 128, 1024), idesc_pv,
+                    (jp > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bar_ve[vs]);
+          umma_commit(&bar_o);
+          if (jp == T - 1) umma_commit(&bar_fin);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+      }
+      // every UMMA of this CTA has completed once bar_drain fires
+      umma_commit(&bar_drain);
+      mbar_wait_drain(&bar_drain, 0);
+      k_used_sh = k_used;
+      v_used_sh = v_used;
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = threadIdx.x;  // 0..127
+    const int q_local = qt * kTile + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int n_past_keys = sch.n_past_pages * p.P;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int b = j & 1;
+      if (!(ok = warp_wait(&bar_s[b], (j >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      float s[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c)
+        tmem_ld32(tmem + lane_off + b * 128 + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
+      tmem_ld_wait();
+      int lim;
+      if (j < sch.n_past_tiles) {
+        lim = n_past_keys - j * kTile;
+      } else {
+        const int key0 = (j - sch.n_past_tiles) * kTile;
+        lim = min(p.C, q_local + 1) - key0;
+      }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const float x = c < lim ? s[c] * p.scale_log2 : -INFINITY;
+        s[c] = x;
+        mt = fmaxf(mt, x);
+      }
+      const bool need = mt > m_used + kRescaleThreshold;
+      const float m_new = need ? mt : m_used;
+      const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds sum_{<j} 2^(s - m_used) v; PV_{j-1} must land before rescaling.
+        // S_j's commit implies PV_{j-2} completed and PV_j waits for P_j, so
+        // bar_o is in phase j-1 or j here and the parity names PV_{j-1}.
+        if (!(ok = warp_wait(&bar_o, (j - 1) & 1, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tmem + lane_off + Cfg::kColO + c * 32, o);
+        }
+        tmem_st_wait();
+      }
+      l *= alpha;
+      m_used = m_new;
+      const float mref = m_used == -INFINITY ? 0.f : m_used;
+      uint32_t pk[kTile / 2];
+#pragma unroll
+      for (int c = 0; c < kTile / 2; ++c) {
+        const float p0 = fast_exp2(s[2 * c] - mref);
+        const float p1 = fast_exp2(s[2 * c + 1] - mref);
+        l += p0 + p1;
+        pk[c] = pack_bf16(p0, p1);
+      }
+#pragma unroll
+      for (int c = 0; c < kTile / 2 / 16; ++c)
+        tmem_st16(tmem + lane_off + b * 128 + c * 16, pk + c * 16);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p[b]);
+    }
+    if (ok) ok = warp_wait(&bar_fin, 0, abort_flag);
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
+    } else {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const bool valid = q_local < p.C;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
+        tmem_ld_wait();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      if (valid) p.lse[static_cast<size_t>(h) * p.C + q_local] = kLn2 * (m_used + log2f(l));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // After an abort, wait (bounded) for TMA loads still landing in shared memory.
+  if (abort_sh && warp == 4 && lane == 0) {
+    for (int i = k_used_sh; i < k_issued_sh; ++i)
+      mbar_wait_drain(&bar_kf[i % Cfg::kNK], (i / Cfg::kNK) & 1);
+    for (int i = v_used_sh; i < v_issued_sh; ++i)
+      mbar_wait_drain(&bar_vf[i % Cfg::kNV], (i / Cfg::kNV) & 1);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+template <int D>
+oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape& s,
+                       cudaStream_t stream) {
+  using Cfg = FwdCfg<D>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmem) != cudaSuccess)
+      return OOMB_ERR_CUDA;
+    attr_set = true;
+  }
+  CUtensorMap qmap, kvmap;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(s.Hq),
+                              static_cast<uint64_t>(s.C)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
+                                 static_cast<uint64_t>(s.Hq) * D * 2};
+    const uint32_t box[3] = {64, 1, kTile};
+    if (!make_bf16_map(&qmap, a->q, 3, dims, strides, box)) return OOMB_ERR_CUDA;
+  }
+  {
+    const oomb_pool_desc& d = pool->desc;
+    const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(d.page_size),
+                              static_cast<uint64_t>(2 * d.num_kv_heads),
+                              static_cast<uint64_t>(d.num_pages)};
+    const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2,
+                                 static_cast<uint64_t>(d.page_size) * D * 2,
+                                 static_cast<uint64_t>(2 * d.num_kv_heads) * d.page_size * D * 2};
+    const uint32_t box[4] = {64, static_cast<uint32_t>(d.page_size), 1, 1};
+    if (!make_bf16_map(&kvmap, pool->kv, 4, dims, strides, box)) return OOMB_ERR_CUDA;
+  }
+  FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(a->o);
+  p.lse = a->lse;
+  p.past_pages = a->past_pages;
+  p.past_counts = a->past_counts;
+  p.cur_pages = a->cur_pages;
+  p.status = pool->d_status;
+  p.max_past = a->max_past;
+  p.C = s.C;
+  p.Hq = s.Hq;
+  p.G = s.G;
+  p.P = s.P;
+  p.num_pool_pages = pool->desc.num_pages;
+  p.scale_log2 = a->softmax_scale * kLog2e;
+  dim3 grid(s.n_qtiles, s.Hq);
+  attn_fwd_kernel<D><<<grid, 192, Cfg::kSmem, stream>>>(p, qmap, kvmap);
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" oomb_status oomb_chunk_attn_fwd(oomb_pool* pool, const oomb_attn_args* args,
+                                           void* stream) {
+  oomb::AttnShape s;
+  oomb_status st = oomb::validate_attn(pool, args, false, &s);
+  if (st != OOMB_OK) return st;
+  oomb::DeviceGuard guard(pool->desc.device);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return s.D == 128 ? launch_fwd<128>(pool, args, s, cs) : launch_fwd<64>(pool, args, s, cs);
+}
