@@ -101,7 +101,9 @@ oomb_status oomb_pool_alloc_page(oomb_pool* pool, int32_t* out_page_id);
 oomb_status oomb_pool_free_page(oomb_pool* pool, int32_t page_id);
 oomb_status oomb_pool_num_free(const oomb_pool* pool, int32_t* out_num_free);
 /* Borrowed views of the pool's buffers (any output may be NULL; grad is NULL
- * without with_grad).  Valid until oomb_pool_destroy. */
+ * without with_grad).  Valid until oomb_pool_destroy.  The summaries of a
+ * pinned-host pool are in device memory (Top-K reads them on the GPU); its KV
+ * and gradients are in pinned host memory. */
 oomb_status oomb_pool_buffers(const oomb_pool* pool, void** kv, float** grad, float** summary);
 oomb_status oomb_pool_get_desc(const oomb_pool* pool, oomb_pool_desc* out_desc);
 
@@ -171,7 +173,8 @@ oomb_status oomb_chunk_attn_bwd_step(oomb_pool* pool, const oomb_attn_args* args
  *   d_out_count      device int32 [num_kv_heads]
  *   d_out_scores     device fp32 [num_kv_heads][n_past] (may be NULL)
  *   d_workspace      device memory of oomb_page_topk_workspace_size() bytes
- * Limits: n_past <= 65536; top_k + n_recent <= 4096. */
+ * The pool may be a device pool or a pinned-host pool (its summaries are on
+ * the device).  Limits: n_past <= 65536; 1 <= top_k + n_recent <= 4096. */
 size_t oomb_page_topk_workspace_size(int32_t chunk_len, int32_t num_q_heads, int32_t num_kv_heads,
                                      int32_t head_dim, int32_t n_past);
 oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk_len,
@@ -186,21 +189,26 @@ oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk
  * its gradients move between pinned host memory and the GPU on dedicated
  * streams, overlapped with compute).
  *
- * oomb_page_prefetch: host (pinned) pool -> device pool, one cudaMemcpyAsync
- * per run of consecutive blocks, on `stream`; records `done_event` (a
- * cudaEvent_t given as void*, may be NULL) after the last copy.  The two pools
- * must share page_size, num_kv_heads and head_dim. */
-oomb_status oomb_page_prefetch(const oomb_pool* host_pool, oomb_pool* device_pool,
+ * oomb_page_prefetch: copies KV blocks from src_pool to dst_pool, one
+ * cudaMemcpyAsync per run of blocks consecutive in both pools, on `stream`,
+ * then records `done_event` (a cudaEvent_t given as void*, may be NULL).
+ * Pinned host -> device is the prefetch of selected pages; device -> pinned
+ * host stores freshly appended pages, and then also copies each block's page
+ * representative into the host pool's (device-resident) summaries.  The pools
+ * must share page_size, num_kv_heads and head_dim; OOMB_LOC_HOST pools are
+ * not accepted; block ids are checked on the host (OOMB_ERR_BAD_PAGE). */
+oomb_status oomb_page_prefetch(const oomb_pool* src_pool, oomb_pool* dst_pool,
                                const int32_t* h_src_blocks, const int32_t* h_dst_blocks,
                                int32_t n_blocks, void* stream, void* done_event);
 
-/* oomb_grad_writeback: adds the device pool's gradient blocks into the host
- * pool's gradient blocks.  The blocks are copied device -> host into a
- * library-owned pinned staging area on `stream`; a host function enqueued on
- * the same stream then adds them into the host pool with several CPU
- * threads.  The device blocks are then zero-filled on the stream, ready for
- * the next chunk's contributions.  Later work on `stream` is ordered after
- * the add. */
+/* oomb_grad_writeback: adds the device pool's gradient blocks h_src_blocks
+ * into the pinned host pool's gradient blocks h_dst_blocks (same order), then
+ * zero-fills the device blocks.  The blocks are copied device -> host into a
+ * pinned staging area owned by the device pool, and a host function enqueued
+ * on `stream` adds them with up to 16 CPU threads; later work on `stream` is
+ * ordered after the add.  Calls for one device pool must be ordered (same
+ * stream), since they share the staging area.  Destination blocks should be
+ * distinct within one call. */
 oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* host_pool,
                                 const int32_t* h_src_blocks, const int32_t* h_dst_blocks,
                                 int32_t n_blocks, void* stream);

