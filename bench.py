@@ -1,0 +1,562 @@
+"""Throughput of paged chunk attention (fwd+bwd) on one B200 per rank.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over a 256K-token context of the
+Qwen2.5-7B attention shape (Hq=28, Hkv=4, d=128, 64-token pages, 64 chunks of
+4096, shuffled page table): for every chunk, append K/V into its pages, the
+forward, and the backward (preprocess, dK/dV added in place into the gradient
+pool, dQ).  The headline value is the dense run's algorithmic TFLOP/s; the
+same line carries the Top-K sparse run (Top-64 + 2 recent pages per chunk and
+KV-head group, Top-K selection included in the timed step), tokens/s for
+both, an end-to-end figure with host buffers, the roofline of the dominant
+kernel and the CPU oracle's throughput on a bounded sample.
+
+Inputs are synthetic (seeded), drawn on the device before timing; the
+working set (Q, dO, KV pool, gradient pool) is far larger than L2.  Under
+torchrun each rank runs the same workload on its own GPU (independent
+replicas, weak scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk-attn fwd+bwd TFLOP/s and context tokens/s at 256K (dense; Top-K sparse)"
+
+
+# ------------------------------------------------------------------ helpers
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16": d.get("bf16_tflops", 1590.0),
+                "bf16_sustained": d.get("bf16_tflops_sustained", 1400.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def pairs_of_chunk(C, n_past_keys):
+    """(query row, key) pairs of one head of one chunk: every past key plus the
+    causal part of the chunk itself."""
+    return C * n_past_keys + C * (C + 1) // 2
+
+
+class Clocks:
+    """Samples nvidia-smi every 200 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        return self.summary()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ our path
+class Run:
+    """All device state of one workload: pool, page tables, inputs, outputs."""
+
+    def __init__(self, w, sparse, device):
+        import paged_kv_chunk_query_b200 as pk
+        from paged_kv_chunk_query_b200 import synth
+        self.pk, self.w, self.sparse, self.dev = pk, w, sparse, device
+        N, C, P, Hq, Hkv, d = (w.num_chunks, w.chunk_len, w.page_size, w.num_q_heads,
+                               w.num_kv_heads, w.head_dim)
+        self.pool = pk.pool_create(w.num_pages, P, Hkv, d, pk.LOC_DEVICE, True, w.alloc_seed,
+                                   device.index or 0)
+        ppc = w.pages_per_chunk
+        self.page_table = [pk.pool_alloc_page(self.pool) for _ in range(N * ppc)]
+        pt = torch.tensor(self.page_table, dtype=torch.int32, device=device)
+        self.page_table_dev = pt
+        self.cur = [pt[c * ppc:(c + 1) * ppc].contiguous() for c in range(N)]
+        self.inputs = [synth.device_chunk_inputs(w, c, device) for c in range(N)]
+        self.o = [torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device) for _ in range(N)]
+        self.dq = [torch.empty_like(x) for x in self.o]
+        self.lse = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(N)]
+        self.delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        self.dense_past = [None] + [pt[:c * ppc].repeat(Hkv, 1).contiguous() for c in range(1, N)]
+        self.dense_cnt = [None] + [torch.full((Hkv,), c * ppc, dtype=torch.int32, device=device)
+                                   for c in range(1, N)]
+        if sparse:
+            ms = w.top_k + w.n_recent
+            self.sel_l = [torch.zeros((Hkv, ms), dtype=torch.int32, device=device) for _ in range(N)]
+            self.sel_p = [torch.zeros((Hkv, ms), dtype=torch.int32, device=device) for _ in range(N)]
+            self.sel_n = [torch.zeros((Hkv,), dtype=torch.int32, device=device) for _ in range(N)]
+            ws = pk.page_topk_workspace_size(C, Hq, Hkv, d, (N - 1) * ppc)
+            self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        # algorithmic FLOPs per chunk (per kernel class) and per step
+        self.flops = {"fwd": [], "dkdv": [], "dq": []}
+        for c in range(N):
+            if sparse and c:
+                n_keys = (min(w.top_k, max(0, c * ppc - w.n_recent)) + min(w.n_recent, c * ppc)) * P
+            else:
+                n_keys = c * C
+            pairs = pairs_of_chunk(C, n_keys) * Hq
+            self.flops["fwd"].append(4.0 * pairs * d)
+            self.flops["dkdv"].append(8.0 * pairs * d)
+            self.flops["dq"].append(2.0 * pairs * d)
+        self.step_flops = sum(sum(v) for v in self.flops.values())
+        self.launches_per_step = N * 5 + ((N - 1) * 2 if sparse else 0)
+
+    def step(self, timers=None):
+        pk, w = self.pk, self.w
+        stream = torch.cuda.current_stream()
+
+        def timed(name, fn):
+            if timers is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            timers.setdefault(name, []).append((a, b))
+
+        ppc = w.pages_per_chunk
+        for c in range(w.num_chunks):
+            x = self.inputs[c]
+            timed("append", lambda: pk.kv_append(self.pool, self.cur[c], x["k"], x["v"], stream))
+            if c == 0:
+                past, cnt = None, None
+            elif self.sparse:
+                n_past = c * ppc
+                timed("topk", lambda: pk.page_topk(
+                    self.pool, x["q"], self.page_table_dev[:n_past], n_past, w.top_k, w.n_recent,
+                    self.sel_l[c], self.sel_p[c], self.sel_n[c], self.ws, stream=stream))
+                past, cnt = self.sel_p[c], self.sel_n[c]
+            else:
+                past, cnt = self.dense_past[c], self.dense_cnt[c]
+            o, lse, dq = self.o[c], self.lse[c], self.dq[c]
+            s = w.softmax_scale
+            timed("fwd", lambda: pk.chunk_attn_fwd(self.pool, x["q"], o, lse, past, cnt,
+                                                   self.cur[c], s, stream))
+            for name, st in (("preprocess", pk.BWD_PREPROCESS), ("dkdv", pk.BWD_DKDV),
+                             ("dq", pk.BWD_DQ)):
+                timed(name, lambda st=st: pk.chunk_attn_bwd(
+                    self.pool, x["q"], o, lse, x["do"], dq, self.delta, past, cnt, self.cur[c],
+                    s, stream, step=st))
+
+    def close(self):
+        self.pk.pool_destroy(self.pool)
+
+
+def _barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x, dist_on, device):
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(run, steps, warmup, dist_on, device, kernel_timers=True):
+    for _ in range(warmup):
+        run.step()
+    torch.cuda.synchronize()
+    _barrier(dist_on)
+    torch.cuda.synchronize()
+    timers = {} if kernel_timers else None
+    stream = torch.cuda.current_stream()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        run.step(timers)
+    b.record(stream)
+    torch.cuda.synchronize()
+    _barrier(dist_on)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    per_kernel = {}
+    if timers:
+        for name, ev in timers.items():
+            per_kernel[name] = sum(x.elapsed_time(y) for x, y in ev) / steps  # ms per step
+    return _max_over_ranks(ms, dist_on, device), per_kernel
+
+
+def e2e_dense(w, steps, device):
+    """Same dense workload through the public API with host buffers: every
+    chunk's Q, K, V, dO are copied from pinned host memory and O, LSE, dQ plus
+    the final gradient pool are read back, inside the timed region.  Copies run
+    on a copy stream, overlapped with the previous chunk's compute."""
+    import paged_kv_chunk_query_b200 as pk
+    from paged_kv_chunk_query_b200 import synth
+    N, C, Hq, Hkv, d, P = (w.num_chunks, w.chunk_len, w.num_q_heads, w.num_kv_heads,
+                           w.head_dim, w.page_size)
+    ppc = w.pages_per_chunk
+    pool = pk.pool_create(w.num_pages, P, Hkv, d, pk.LOC_DEVICE, True, w.alloc_seed,
+                          device.index or 0)
+    try:
+        table = [pk.pool_alloc_page(pool) for _ in range(N * ppc)]
+        pt = torch.tensor(table, dtype=torch.int32, device=device)
+        host_in = []
+        for c in range(N):
+            x = synth.device_chunk_inputs(w, c, device)
+            host_in.append({k: v.cpu().pin_memory() for k, v in x.items()})
+        host_o = [torch.empty((C, Hq, d), dtype=torch.bfloat16).pin_memory() for _ in range(N)]
+        host_dq = [torch.empty_like(t) for t in host_o]
+        host_dq = [t.pin_memory() for t in host_dq]
+        host_lse = [torch.empty((Hq, C), dtype=torch.float32).pin_memory() for _ in range(N)]
+        _, grad, _ = pk.pool_views(pool)
+        host_grad = torch.empty(grad.shape, dtype=torch.float32).pin_memory()
+        dev_in = [{k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in host_in[0].items()}
+                  for _ in range(2)]
+        dev_out = [(torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device),
+                    torch.empty((Hq, C), dtype=torch.float32, device=device),
+                    torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device)) for _ in range(2)]
+        delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        past = [None] + [pt[:c * ppc].repeat(Hkv, 1).contiguous() for c in range(1, N)]
+        cnt = [None] + [torch.full((Hkv,), c * ppc, dtype=torch.int32, device=device)
+                        for c in range(1, N)]
+        comp = torch.cuda.current_stream()
+        copy = torch.cuda.Stream(device=device)
+        h2d = sum(t.numel() * t.element_size() for t in host_in[0].values()) * N
+        d2h = (sum(t.numel() * t.element_size() for t in (host_o[0], host_lse[0], host_dq[0])) * N
+               + host_grad.numel() * 4)
+
+        def one_step():
+            in_ready = [torch.cuda.Event() for _ in range(N)]
+            out_ready = [torch.cuda.Event() for _ in range(N)]
+            out_free = [torch.cuda.Event() for _ in range(N)]
+            with torch.cuda.stream(copy):
+                for k, v in host_in[0].items():
+                    dev_in[0][k].copy_(v, non_blocking=True)
+                in_ready[0].record(copy)
+            for c in range(N):
+                buf = c % 2
+                if c + 1 < N:
+                    with torch.cuda.stream(copy):
+                        if c >= 1:
+                            copy.wait_event(out_ready[c - 1])  # inputs buffer (c+1)%2 was chunk c-1's
+                        for k, v in host_in[c + 1].items():
+                            dev_in[(c + 1) % 2][k].copy_(v, non_blocking=True)
+                        in_ready[c + 1].record(copy)
+                comp.wait_event(in_ready[c])
+                if c >= 2:
+                    comp.wait_event(out_free[c - 2])
+                x = dev_in[buf]
+                o, lse, dq = dev_out[buf]
+                cur = pt[c * ppc:(c + 1) * ppc]
+                pk.kv_append(pool, cur, x["k"], x["v"], comp)
+                pk.chunk_attn_fwd(pool, x["q"], o, lse, past[c], cnt[c], cur, w.softmax_scale, comp)
+                pk.chunk_attn_bwd(pool, x["q"], o, lse, x["do"], dq, delta, past[c], cnt[c], cur,
+                                  w.softmax_scale, comp)
+                out_ready[c].record(comp)
+                with torch.cuda.stream(copy):
+                    copy.wait_event(out_ready[c])
+                    host_o[c].copy_(o, non_blocking=True)
+                    host_lse[c].copy_(lse, non_blocking=True)
+                    host_dq[c].copy_(dq, non_blocking=True)
+                    out_free[c].record(copy)
+            comp.wait_stream(copy)
+            host_grad.copy_(grad, non_blocking=True)
+
+        one_step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        for _ in range(steps):
+            one_step()
+        b.record(comp)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps, h2d, d2h
+    finally:
+        pk.pool_destroy(pool)
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, rows, seed_chunk=None):
+    """Bounded sample of the same workload for the CPU oracle: the first `rows`
+    query rows of chunk N/2 (all heads), as a chunk of their own, against every
+    past key of that chunk, forward and backward.  Returns (seconds,
+    algorithmic FLOPs, threads used, description)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle.attention import chunk_backward, chunk_forward
+    from paged_kv_chunk_query_b200 import synth
+    c = w.num_chunks // 2 if seed_chunk is None else seed_chunk
+    C, P = w.chunk_len, w.page_size
+    ch = synth.chunk_inputs(w, c)
+    q = ch["q"][:rows].float().numpy().astype(np.float64)
+    do = ch["do"][:rows].float().numpy().astype(np.float64)
+    kc, vc = ch["k"][:rows].float().numpy(), ch["v"][:rows].float().numpy()
+    past_k, past_v = [], []
+    for cc in range(c):  # past keys of chunk c, drawn chunk by chunk (not timed)
+        x = synth.chunk_inputs(w, cc, which=("k", "v"))
+        past_k.append(x["k"].float().numpy())
+        past_v.append(x["v"].float().numpy())
+    pk_ = np.concatenate(past_k).astype(np.float64)
+    pv_ = np.concatenate(past_v).astype(np.float64)
+    Hkv = w.num_kv_heads
+    kp = [pk_[:, g, :] for g in range(Hkv)]
+    vp = [pv_[:, g, :] for g in range(Hkv)]
+    t0 = time.perf_counter()
+    chunk_forward(q, kp, vp, kc, vc, w.softmax_scale)
+    chunk_backward(q, kp, vp, kc, vc, do, w.softmax_scale)
+    dt = time.perf_counter() - t0
+    pairs = pairs_of_chunk(rows, c * C) * w.num_q_heads
+    flops = 14.0 * pairs * w.head_dim
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    desc = (f"{w.name}: first {rows} rows of chunk {c} (all {w.num_q_heads} heads) against its "
+            f"{c * C} past keys + causal self, fp64 numpy fwd+bwd")
+    return dt, flops, threads, desc
+
+
+# ------------------------------------------------------------------ roofline bits
+def _traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != e["sha256"]:
+        return None
+    return e
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen256k")
+    ap.add_argument("--sparse-workload", default=None,
+                    help="sparse run's workload (default: the Top-K variant of --workload)")
+    ap.add_argument("--no-sparse", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0: auto)")
+    a = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from paged_kv_chunk_query_b200 import synth
+    w = synth.WORKLOADS[a.workload]
+    ws_name = a.sparse_workload or (a.workload + "_topk" if a.workload + "_topk" in synth.WORKLOADS
+                                    else a.workload)
+
+    if a.impl == "reference":
+        # The reference arm is the CPU oracle as it stands, rank 0 only.
+        if rank != 0:
+            return
+        rows = a.cpu_rows or 32
+        for _ in range(a.warmup):
+            oracle_sample(w, rows)
+        secs, flops = [], 0.0
+        threads, desc = 1, ""
+        for _ in range(a.steps):
+            dt, flops, threads, desc = oracle_sample(w, rows)
+            secs.append(dt)
+        dt = sum(secs) / len(secs)
+        val = flops / dt / 1e12
+        line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 0, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": w.name, "sample": desc},
+                "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads,
+                                 "kind": "oracle", "sample": desc},
+                "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import paged_kv_chunk_query_b200 as pk  # noqa: F401  (fails loudly without the library)
+
+    clocks = Clocks(local)
+    dense = Run(w, False, device)
+    clocks.start()
+    ms, kt = time_steps(dense, a.steps, a.warmup, dist_on, device)
+    clk = clocks.stop()
+    dense_status = pk.get_device_status(dense.pool)
+    step_flops = dense.step_flops
+    value = step_flops * world / (ms / 1e3) / 1e12
+    tokens = w.context * world / (ms / 1e3)
+    kernel_flops = {k: sum(v) for k, v in dense.flops.items()}
+    dense.close()
+    del dense
+    torch.cuda.empty_cache()
+
+    peaks = _peaks()
+    # dominant kernel: the largest share of the step's time
+    dom = max(kt, key=kt.get)
+    dom_ms = kt[dom]
+    tr = _traffic(dom)
+    if dom in kernel_flops:
+        achieved = kernel_flops[dom] / (dom_ms / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_sustained"],
+                "frac_of_burst": achieved / peaks["bf16"],
+                "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                "traffic": tr["bytes_per_launch"] if tr else None,
+                "launch_share": dom_ms / ms}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": tr["bytes_per_launch"] if tr else None}
+    kernels = {k: {"ms_per_step": v, "share": v / ms,
+                   "tflops": (kernel_flops[k] / (v / 1e3) / 1e12) if k in kernel_flops else None}
+               for k, v in kt.items()}
+
+    sparse_obj = None
+    if not a.no_sparse:
+        ws = synth.WORKLOADS[ws_name]
+        sp = Run(ws, True, device)
+        ms_s, kt_s = time_steps(sp, a.steps, a.warmup, dist_on, device)
+        sparse_status = pk.get_device_status(sp.pool)
+        topk_bytes = 0.0
+        C, Hq, Hkv, d, P = ws.chunk_len, ws.num_q_heads, ws.num_kv_heads, ws.head_dim, ws.page_size
+        for c in range(1, ws.num_chunks):
+            n_past = c * ws.pages_per_chunk
+            topk_bytes += C * Hq * d * 2 + n_past * (Hkv * d * 4 + 4) + Hkv * (ws.top_k + ws.n_recent) * 8
+        topk_ms = kt_s.get("topk", 0.0)
+        sparse_obj = {"workload": ws.name, "value": sp.step_flops * world / (ms_s / 1e3) / 1e12,
+                      "unit": "TFLOP/s", "ms_per_step": ms_s,
+                      "tokens_per_s": ws.context * world / (ms_s / 1e3),
+                      "dense_over_sparse_time": ms / ms_s,
+                      "kernels": {k: {"ms_per_step": v, "share": v / ms_s} for k, v in kt_s.items()},
+                      "topk_hbm": {"bound": "hbm", "achieved": topk_bytes / (topk_ms / 1e3) / 1e9
+                                   if topk_ms else None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": (topk_bytes / (topk_ms / 1e3) / 1e9) / peaks["hbm_gbs"]
+                                   if topk_ms else None,
+                                   "note": "per-chunk launches (query mean + select), launch-bound"},
+                      "device_status": sparse_status}
+        sp.close()
+        del sp
+        torch.cuda.empty_cache()
+
+    e2e = None
+    if not a.no_e2e:
+        ms_e, h2d, d2h = e2e_dense(w, max(1, min(a.steps, 2)), device)
+        e2e = {"value": step_flops * world / (ms_e / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu:
+        rows = a.cpu_rows or 32
+        dt, fl, threads, desc = oracle_sample(w, rows)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "seconds": dt}
+
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "context": w.context, "chunk_len": w.chunk_len,
+                   "num_chunks": w.num_chunks, "page_size": w.page_size,
+                   "heads": f"{w.num_q_heads}q/{w.num_kv_heads}kv", "head_dim": w.head_dim,
+                   "page_table": "shuffled" if w.shuffle_pages else "identity",
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (Q+dO 3.5 GiB, KV pool 512 MiB, grad pool 1 GiB)"},
+        "tokens_per_s": tokens,
+        "kernels": kernels,
+        "roofline": roof,
+        "sparse": sparse_obj,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": w.num_chunks * 5 * a.steps
+        + ((w.num_chunks * 5 + (w.num_chunks - 1) * 2) * a.steps if sparse_obj else 0),
+        "clocks": clk,
+        "device_status": dense_status,
+        "peaks": peaks,
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -78,6 +78,9 @@ class Workload:
 WORKLOADS = {
     "tiny": Workload("tiny", 4, 1, 64, 16, 64, 8, seed=1000),
     "qwen32k": Workload("qwen32k", 28, 4, 128, 64, 4096, 8, seed=1001, do_std=1e-2),
+    # profiling-sized sparse case (not a headline configuration)
+    "qwen32k_topk": Workload("qwen32k_topk", 28, 4, 128, 64, 4096, 8, seed=1005,
+                             shuffle_pages=True, page_direction=0.5, top_k=64, n_recent=2),
     "qwen256k": Workload("qwen256k", 28, 4, 128, 64, 4096, 64, seed=1002,
                          shuffle_pages=True),
     "qwen256k_topk": Workload("qwen256k_topk", 28, 4, 128, 64, 4096, 64, seed=1003,
@@ -100,26 +103,29 @@ def _randn(shape, gen) -> torch.Tensor:
     return torch.randn(shape, generator=gen, dtype=torch.float32)
 
 
-def chunk_inputs(w: Workload, c: int) -> dict[str, torch.Tensor]:
-    """Q, K, V, dO of chunk ``c`` as bf16 CPU tensors.
+def chunk_inputs(w: Workload, c: int, which=("q", "k", "v", "do")) -> dict[str, torch.Tensor]:
+    """Q, K, V, dO of chunk ``c`` as bf16 CPU tensors (only those named in
+    ``which``; each tensor has its own generator, so skipping some does not
+    change the others).
 
     Layouts: q, do ``[C][Hq][d]``; k, v ``[C][Hkv][d]`` (token-major, as a
     projection would write them).
     """
     C, Hq, Hkv, d, P = w.chunk_len, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size
-    q = _randn((C, Hq, d), _generator(w.seed, c, 0))
-    k = _randn((C, Hkv, d), _generator(w.seed, c, 1))
-    v = _randn((C, Hkv, d), _generator(w.seed, c, 2))
-    do = _randn((C, Hq, d), _generator(w.seed, c, 3)) * w.do_std
-    if w.page_direction:
-        u = _randn((C // P, Hkv, d), _generator(w.seed, c, 4)) * w.page_direction
-        k = k + u.repeat_interleave(P, dim=0)
-    return {
-        "q": q.to(torch.bfloat16),
-        "k": k.to(torch.bfloat16),
-        "v": v.to(torch.bfloat16),
-        "do": do.to(torch.bfloat16),
-    }
+    out = {}
+    if "q" in which:
+        out["q"] = _randn((C, Hq, d), _generator(w.seed, c, 0)).to(torch.bfloat16)
+    if "k" in which:
+        k = _randn((C, Hkv, d), _generator(w.seed, c, 1))
+        if w.page_direction:
+            u = _randn((C // P, Hkv, d), _generator(w.seed, c, 4)) * w.page_direction
+            k = k + u.repeat_interleave(P, dim=0)
+        out["k"] = k.to(torch.bfloat16)
+    if "v" in which:
+        out["v"] = _randn((C, Hkv, d), _generator(w.seed, c, 2)).to(torch.bfloat16)
+    if "do" in which:
+        out["do"] = (_randn((C, Hq, d), _generator(w.seed, c, 3)) * w.do_std).to(torch.bfloat16)
+    return out
 
 
 def sequence_inputs(w: Workload) -> dict[str, torch.Tensor]:
