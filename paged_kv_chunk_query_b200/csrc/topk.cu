@@ -10,58 +10,73 @@
 // ties going to the lower logical id; pages [n_past - R, n_past) are always
 // kept; the output lists ascending logical ids.
 //
-// Kernel 1 (qmean_partial): grid (splits, Hkv); each CTA streams a slice of the
-//   chunk's rows with 16-byte loads and writes one fp32 partial sum per d.
-// Kernel 2 (select): one CTA per group; reduces the partials in a fixed order,
-//   scores every past page (one warp per page, float4 loads of the summary),
-//   finds the K-th largest 64-bit key (ordered score, inverted id) with an
-//   8-pass radix select, then compacts the kept ids in ascending order.
+// Kernel 1 (qmean_partial): grid (64 slices, Hkv); each CTA streams a slice of
+//   the chunk's rows with 16-byte loads, 4 in flight per thread, and writes one
+//   fp32 partial sum per d.
+// Kernel 2 (page_score): grid (pages / 64, Hkv); each CTA reduces the partials
+//   in a fixed order into q_bar, then each warp scores 8 pages (float4 loads of
+//   the summaries, shuffle reduction).
+// Kernel 3 (select): one CTA per group; finds the K-th largest 64-bit key
+//   (ordered score, inverted id) by 8-bit radix passes from the top with a
+//   parallel bin scan, stopping once the boundary bin is kept whole, then
+//   compacts the kept ids in ascending order.
 #include <cuda_bf16.h>
 
 #include "internal.h"
 
 namespace {
 
+constexpr int kSplits = 64;          // query-mean slices per group
+constexpr int kMeanThreads = 512;
+constexpr int kScoreThreads = 256;   // 8 warps x 8 pages per CTA
+constexpr int kPagesPerScoreCta = 64;
 constexpr int kSelectThreads = 1024;
-
-int topk_splits(int C) {
-  int s = C / 32;
-  if (s < 1) s = 1;
-  if (s > 128) s = 128;
-  return s;
-}
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// ---------------------------------------------------------------- query mean
+// grid (kSplits, Hkv): CTA (s, g) sums rows (token, head in g) of token slice s.
 template <int D>
-__global__ void __launch_bounds__(256) qmean_partial_kernel(const __nv_bfloat16* __restrict__ q,
-                                                            float* __restrict__ partial, int C,
-                                                            int Hq, int G, int splits) {
-  constexpr int VPR = D / 8;      // 16-byte vectors per row
-  constexpr int RG = 256 / VPR;   // rows in flight per pass
+__global__ void __launch_bounds__(kMeanThreads) qmean_partial_kernel(
+    const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, int C, int Hq, int G) {
+  constexpr int VPR = D / 8;               // 16-byte vectors per row
+  constexpr int RG = kMeanThreads / VPR;   // rows per pass
+  constexpr int U = 4;                     // loads in flight per thread
   __shared__ float red[RG][D];
   const int split = blockIdx.x, g = blockIdx.y, t = threadIdx.x;
   const int vec = t % VPR, rg = t / VPR;
-  const int per = (C + splits - 1) / splits;
+  const int per = (C + kSplits - 1) / kSplits;
   const int tok0 = split * per, tok1 = min(C, tok0 + per);
-  const int rows = max(0, tok1 - tok0) * G;  // rows (token, head in group) of this slice
+  const int rows = max(0, tok1 - tok0) * G;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int rr = rg; rr < rows; rr += RG) {
-    const int tok = tok0 + rr / G, hh = g * G + rr % G;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-        q + (static_cast<size_t>(tok) * Hq + hh) * D + vec * 8));
-    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+  for (int base = rg; base < rows; base += RG * U) {
+    uint4 v[U];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(b[e]);
+    for (int u = 0; u < U; ++u) {
+      const int rr = base + u * RG;
+      if (rr < rows) {
+        const int tok = tok0 + rr / G, hh = g * G + rr % G;
+        v[u] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<size_t>(tok) * Hq + hh) * D +
+                                                    vec * 8));
+      } else {
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(b[e]);
+    }
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[rg][vec * 8 + e] = acc[e];
   __syncthreads();
   if (t < D) {
     float s = 0.f;
-    for (int r = 0; r < RG; ++r) s += red[r][t];
+    for (int r = 0; r < RG; ++r) s += red[r][t];  // fixed order: deterministic
     partial[(static_cast<size_t>(split) * gridDim.y + g) * D + t] = s;
   }
 }
@@ -72,102 +87,162 @@ __device__ __forceinline__ uint32_t order_f32(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// ---------------------------------------------------------------- page scores
+// grid (ceil(n_past / 64), Hkv).  Every CTA reduces the kSplits partials of its
+// group in the same fixed order (so all CTAs use the identical q_bar), then
+// each warp scores 8 pages.  Key = (ordered score << 32) | (~logical id).
 template <int D>
-__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
-    const float* __restrict__ partial, int splits, const float* __restrict__ summary,
-    const int32_t* __restrict__ page_table, int n_past, int top_k, int n_recent, int Hkv,
-    int num_pool_pages, float inv_rows, unsigned long long* __restrict__ keys,
-    int32_t* __restrict__ out_logical, int32_t* __restrict__ out_physical,
-    int32_t* __restrict__ out_count, float* __restrict__ out_scores, uint32_t* status) {
+__global__ void __launch_bounds__(kScoreThreads) page_score_kernel(
+    const float* __restrict__ partial, const float* __restrict__ summary,
+    const int32_t* __restrict__ page_table, int n_past, int Hkv, int num_pool_pages,
+    float inv_rows, unsigned long long* __restrict__ keys, float* __restrict__ out_scores,
+    uint32_t* status) {
+  constexpr int kParts = kScoreThreads / D;  // threads per d in the q_bar reduction
+  __shared__ float part_sum[kParts][D];
   __shared__ float qbar[D];
+  const int g = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  {
+    constexpr int PER = kSplits / kParts;  // partials per thread, all loads in flight
+    const int d = t % D, part = t / D;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      v[i] = __ldg(partial + (static_cast<size_t>(part * PER + i) * Hkv + g) * D + d);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) s += v[i];
+    part_sum[part][d] = s;
+    __syncthreads();
+    if (t < D) {
+      float s2 = 0.f;
+#pragma unroll
+      for (int i = 0; i < kParts; ++i) s2 += part_sum[i][t];
+      qbar[t] = s2 * inv_rows;
+    }
+    __syncthreads();
+  }
+  constexpr int PW = kPagesPerScoreCta / (kScoreThreads / 32);  // pages per warp
+  const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
+  constexpr int EPL = D / 32;  // elements per lane
+  float qv[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) qv[e] = qbar[lane * EPL + e];
+  float acc[PW];
+#pragma unroll
+  for (int i = 0; i < PW; ++i) {
+    const int p = p0 + i;
+    acc[i] = 0.f;
+    if (p < n_past) {
+      int phys = __ldg(page_table + p);
+      if (phys < 0 || phys >= num_pool_pages) {
+        if (lane == 0) atomicOr(status, OOMB_DEV_BAD_PAGE);
+        phys = 0;
+      }
+      const float* srow = summary + (static_cast<size_t>(phys) * Hkv + g) * D + lane * EPL;
+      if (EPL == 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(srow));
+        acc[i] = a.x * qv[0] + a.y * qv[1] + a.z * qv[2] + a.w * qv[3];
+      } else {
+        const float2 a = __ldg(reinterpret_cast<const float2*>(srow));
+        acc[i] = a.x * qv[0] + a.y * qv[1];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < PW; ++i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+  }
+  if (lane < PW) {
+    float mine = 0.f;
+#pragma unroll
+    for (int i = 0; i < PW; ++i)
+      if (lane == i) mine = acc[i];
+    const int p = p0 + lane;
+    if (p < n_past) {
+      if (out_scores) out_scores[static_cast<size_t>(g) * n_past + p] = mine;
+      keys[static_cast<size_t>(g) * n_past + p] =
+          (static_cast<unsigned long long>(order_f32(mine)) << 32) |
+          static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
+    }
+  }
+}
+
+// ---------------------------------------------------------------- select
+// One CTA per group: the K-th largest candidate key by 8-bit radix passes from
+// the top, each with a parallel suffix scan over the 256 bins; stops early once
+// the boundary bin is taken whole.  Then compacts kept ids in ascending order.
+__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
+    const unsigned long long* __restrict__ keys_all, const int32_t* __restrict__ page_table,
+    int n_past, int top_k, int n_recent, int num_pool_pages, int32_t* __restrict__ out_logical,
+    int32_t* __restrict__ out_physical, int32_t* __restrict__ out_count) {
   __shared__ unsigned int hist[256];
+  __shared__ unsigned int warp_tot[8];
   __shared__ unsigned long long kth_sh;
-  __shared__ int need_sh;
+  __shared__ int need_sh, done_sh;
   __shared__ int warp_sum[kSelectThreads / 32];
   __shared__ int running_sh;
   const int g = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int max_sel = top_k + n_recent;
   const int n_cand = max(0, n_past - n_recent);
   const int k_eff = min(top_k, n_cand);
+  const unsigned long long* keys = keys_all + static_cast<size_t>(g) * n_past;
 
-  if (t < D) {
-    float s = 0.f;
-    for (int i = 0; i < splits; ++i) s += partial[(static_cast<size_t>(i) * Hkv + g) * D + t];
-    qbar[t] = s * inv_rows;
-  }
-  __syncthreads();
-
-  // scores: one warp per page
-  unsigned long long* gkeys = keys + static_cast<size_t>(g) * n_past;
-  for (int p = warp; p < n_past; p += kSelectThreads / 32) {
-    int phys = page_table[p];
-    if (phys < 0 || phys >= num_pool_pages) {
-      if (lane == 0) atomicOr(status, OOMB_DEV_BAD_PAGE);
-      phys = 0;
-    }
-    const float* srow = summary + (static_cast<size_t>(phys) * Hkv + g) * D;
-    float acc = 0.f;
-    if (D == 128) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(srow) + lane);
-      acc = a.x * qbar[4 * lane] + a.y * qbar[4 * lane + 1] + a.z * qbar[4 * lane + 2] +
-            a.w * qbar[4 * lane + 3];
-    } else {
-      const float2 a = __ldg(reinterpret_cast<const float2*>(srow) + lane);
-      acc = a.x * qbar[2 * lane] + a.y * qbar[2 * lane + 1];
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      if (out_scores) out_scores[static_cast<size_t>(g) * n_past + p] = acc;
-      gkeys[p] = (static_cast<unsigned long long>(order_f32(acc)) << 32) |
-                 static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
-    }
-  }
-  __syncthreads();
-
-  // K-th largest candidate key (keys are unique: ids differ)
   if (t == 0) {
     kth_sh = 0ull;  // with k_eff >= n_cand every candidate is kept
     need_sh = k_eff;
+    done_sh = 0;
   }
   __syncthreads();
   if (k_eff > 0 && k_eff < n_cand) {
     unsigned long long prefix = 0ull, mask = 0ull;
     for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int i = t; i < 256; i += kSelectThreads) hist[i] = 0u;
+      if (t < 256) hist[t] = 0u;
       __syncthreads();
       for (int p = t; p < n_cand; p += kSelectThreads) {
-        const unsigned long long k = gkeys[p];
+        const unsigned long long k = keys[p];
         if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255ull], 1u);
       }
       __syncthreads();
-      if (t == 0) {
-        int need = need_sh, cum = 0, sel = 0;
-        for (int d = 255; d >= 0; --d) {
-          if (cum + static_cast<int>(hist[d]) >= need) {
-            sel = d;
-            need -= cum;
-            break;
-          }
-          cum += hist[d];
+      // inclusive suffix sum over bins 255..0: thread t < 256 owns bin 255 - t
+      unsigned int incl = 0;
+      if (t < 256) {
+        const unsigned int v = hist[255 - t];
+        incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
         }
-        need_sh = need;
-        kth_sh = prefix | (static_cast<unsigned long long>(sel) << shift);
+        if (lane == 31) warp_tot[warp] = incl;
+      }
+      __syncthreads();
+      if (t < 256) {
+        for (int w = 0; w < warp; ++w) incl += warp_tot[w];
+        const int bin = 255 - t;
+        const unsigned int v = hist[bin];
+        const unsigned int excl = incl - v;
+        const int need = need_sh;
+        if (excl < static_cast<unsigned>(need) && static_cast<unsigned>(need) <= incl) {
+          kth_sh = prefix | (static_cast<unsigned long long>(bin) << shift);
+          need_sh = need - static_cast<int>(excl);
+          if (v == static_cast<unsigned>(need) - excl) done_sh = 1;  // bin taken whole
+        }
       }
       __syncthreads();
       prefix = kth_sh;
       mask |= 255ull << shift;
+      if (done_sh) break;
     }
   }
   const unsigned long long kth = kth_sh;
 
-  // compaction in ascending logical id
   if (t == 0) running_sh = 0;
   __syncthreads();
   for (int base = 0; base < n_past; base += kSelectThreads) {
     const int p = base + t;
     int keep = 0;
-    if (p < n_cand) keep = (k_eff >= n_cand) || (k_eff > 0 && gkeys[p] >= kth);
+    if (p < n_cand) keep = (k_eff >= n_cand) || (k_eff > 0 && keys[p] >= kth);
     else if (p < n_past) keep = 1;
     const unsigned ballot = __ballot_sync(0xffffffffu, keep);
     if (lane == 0) warp_sum[warp] = __popc(ballot);
@@ -178,7 +253,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
     if (keep && before < max_sel) {
       out_logical[static_cast<size_t>(g) * max_sel + before] = p;
       if (out_physical) {
-        int phys = page_table[p];
+        const int phys = page_table[p];
         out_physical[static_cast<size_t>(g) * max_sel + before] =
             (phys >= 0 && phys < num_pool_pages) ? phys : 0;
       }
@@ -201,7 +276,7 @@ extern "C" size_t oomb_page_topk_workspace_size(int32_t chunk_len, int32_t num_q
                                                 int32_t n_past) {
   (void)num_q_heads;
   if (chunk_len <= 0 || num_kv_heads <= 0 || head_dim <= 0 || n_past < 0) return 0;
-  const size_t partial = static_cast<size_t>(topk_splits(chunk_len)) * num_kv_heads * head_dim * 4;
+  const size_t partial = static_cast<size_t>(kSplits) * num_kv_heads * head_dim * 4;
   const size_t keys = static_cast<size_t>(num_kv_heads) * (n_past > 0 ? n_past : 1) * 8;
   return align256(partial) + align256(keys);
 }
@@ -227,26 +302,28 @@ extern "C" oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, in
     return OOMB_ERR_INVALID_ARG;
   oomb::DeviceGuard guard(d.device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int splits = topk_splits(chunk_len);
   float* partial = static_cast<float*>(d_workspace);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(
-      static_cast<uint8_t*>(d_workspace) +
-      align256(static_cast<size_t>(splits) * Hkv * D * 4));
+      static_cast<uint8_t*>(d_workspace) + align256(static_cast<size_t>(kSplits) * Hkv * D * 4));
   const int G = num_q_heads / Hkv;
   const float inv_rows = 1.0f / (static_cast<float>(chunk_len) * static_cast<float>(G));
-  dim3 g1(splits, Hkv);
+  const auto* q = static_cast<const __nv_bfloat16*>(d_q);
+  dim3 g1(kSplits, Hkv), g2((n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv);
   if (D == 128) {
-    qmean_partial_kernel<128><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(d_q), partial,
-                                                 chunk_len, num_q_heads, G, splits);
-    topk_select_kernel<128><<<Hkv, kSelectThreads, 0, s>>>(
-        partial, splits, pool->summary, d_page_table, n_past, top_k, n_recent, Hkv, d.num_pages,
-        inv_rows, keys, d_out_logical, d_out_physical, d_out_count, d_out_scores, pool->d_status);
+    qmean_partial_kernel<128><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
+    if (n_past > 0)
+      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
+                                                          n_past, Hkv, d.num_pages, inv_rows,
+                                                          keys, d_out_scores, pool->d_status);
   } else {
-    qmean_partial_kernel<64><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(d_q), partial,
-                                                chunk_len, num_q_heads, G, splits);
-    topk_select_kernel<64><<<Hkv, kSelectThreads, 0, s>>>(
-        partial, splits, pool->summary, d_page_table, n_past, top_k, n_recent, Hkv, d.num_pages,
-        inv_rows, keys, d_out_logical, d_out_physical, d_out_count, d_out_scores, pool->d_status);
+    qmean_partial_kernel<64><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
+    if (n_past > 0)
+      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
+                                                         n_past, Hkv, d.num_pages, inv_rows, keys,
+                                                         d_out_scores, pool->d_status);
   }
+  topk_select_kernel<<<Hkv, kSelectThreads, 0, s>>>(keys, d_page_table, n_past, top_k, n_recent,
+                                                     d.num_pages, d_out_logical, d_out_physical,
+                                                     d_out_count);
   return oomb::check_launch();
 }
