@@ -282,16 +282,26 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld_wait();
       const float* L = sL(s);
       // query column c is valid if inside the chunk and (current tile) causally after the key
-      int cmax = min(kTile, p.C - t * kTile);  // columns [0, cmax) are inside the chunk
-      int cmin = 0;
-      if (!is_past) cmin = key_local - t * kTile;  // q_local >= key_local
-      uint32_t pk[kTile / 2];
+      const int cmax = min(kTile, p.C - t * kTile);  // columns [0, cmax) are inside the chunk
+      const int cmin = is_past ? 0 : key_local - t * kTile;  // q_local >= key_local
+      const bool full = key_valid && cmin <= 0 && cmax >= kTile;
+      // P^T = 2^(S^T*scale*log2e - LSE*log2e); LSE read 4 at a time (broadcast)
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const bool v = key_valid && c < cmax && c >= cmin;
-        const float e = fast_exp2(fmaf(pr[c], p.scale_log2, -L[c] * kLog2e));
-        pr[c] = v ? e : 0.f;
+      for (int c4 = 0; c4 < kTile / 4; ++c4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(L + 4 * c4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          pr[c] = fast_exp2(fmaf(pr[c], p.scale_log2, -lv[e] * kLog2e));
+        }
       }
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          pr[c] = (key_valid && c < cmax && c >= cmin) ? pr[c] : 0.f;
+      }
+      uint32_t pk[kTile / 2];
 #pragma unroll
       for (int c = 0; c < kTile / 2; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
 #pragma unroll
@@ -312,13 +322,19 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld_wait();
         uint32_t dk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = c * 32 + 2 * e;
-          float a = pr[c0] * (__uint_as_float(dp[2 * e]) - Dl[c0]);
-          float b = pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - Dl[c0 + 1]);
-          a = pr[c0] != 0.f ? a : 0.f;
-          b = pr[c0 + 1] != 0.f ? b : 0.f;
-          dk[e] = pack_bf16(a, b);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(Dl + c * 32 + 4 * e4);
+          const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+          float ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = c * 32 + 4 * e4 + e;
+            ds[e] = pr[c0] * (__uint_as_float(dp[4 * e4 + e]) - dv[e]);
+            // masked columns may hold stale delta values: force an exact zero
+            if (!full) ds[e] = pr[c0] != 0.f ? ds[e] : 0.f;
+          }
+          dk[2 * e4] = pack_bf16(ds[0], ds[1]);
+          dk[2 * e4 + 1] = pack_bf16(ds[2], ds[3]);
         }
         tmem_st16(tmem + lane_off + Cfg::kColDPT + c * 16, dk);
       }
@@ -574,10 +590,12 @@ __global__ void __launch_bounds__(192, 1)
       int lim;
       if (j < sch.n_past_tiles) lim = n_past_keys - j * kTile;
       else lim = min(p.C, q_local + 1) - (j - sch.n_past_tiles) * kTile;
+      if (!row_valid) lim = 0;
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const float e = fast_exp2(fmaf(pr[c], p.scale_log2, -lse2));
-        pr[c] = (c < lim && row_valid) ? e : 0.f;
+      for (int c = 0; c < kTile; ++c) pr[c] = fast_exp2(fmaf(pr[c], p.scale_log2, -lse2));
+      if (lim < kTile) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) pr[c] = c < lim ? pr[c] : 0.f;
       }
       if (!(ok = warp_wait(&bar_dp, j & 1, abort_flag))) break;
       tc_fence_after();

@@ -227,13 +227,18 @@ __global__ void __launch_bounds__(192, 1)
         const int key0 = (j - sch.n_past_tiles) * kTile;
         lim = min(p.C, q_local + 1) - key0;
       }
-      float mt = -INFINITY;
+      if (lim < kTile) {  // diagonal or ragged tile: keys at and past `lim` are masked
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const float x = c < lim ? s[c] * p.scale_log2 : -INFINITY;
-        s[c] = x;
-        mt = fmaxf(mt, x);
+        for (int c = 0; c < kTile; ++c) s[c] = c < lim ? s[c] : -INFINITY;
       }
+      // row max with 8 independent chains (raw logits; scale > 0 keeps the order)
+      float m8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
       const bool need = mt > m_used + kRescaleThreshold;
       const float m_new = need ? mt : m_used;
       const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
@@ -254,17 +259,21 @@ __global__ void __launch_bounds__(192, 1)
         }
         tmem_st_wait();
       }
-      l *= alpha;
       m_used = m_new;
-      const float mref = m_used == -INFINITY ? 0.f : m_used;
+      const float neg_mref = m_used == -INFINITY ? 0.f : -m_used;
+      // p = 2^(S*scale*log2e - m); masked logits are -inf and give 0
+      float l8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) l8[e] = 0.f;
       uint32_t pk[kTile / 2];
 #pragma unroll
       for (int c = 0; c < kTile / 2; ++c) {
-        const float p0 = fast_exp2(s[2 * c] - mref);
-        const float p1 = fast_exp2(s[2 * c + 1] - mref);
-        l += p0 + p1;
+        const float p0 = fast_exp2(fmaf(s[2 * c], p.scale_log2, neg_mref));
+        const float p1 = fast_exp2(fmaf(s[2 * c + 1], p.scale_log2, neg_mref));
+        l8[c & 7] += p0 + p1;
         pk[c] = pack_bf16(p0, p1);
       }
+      l = l * alpha + (((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7])));
 #pragma unroll
       for (int c = 0; c < kTile / 2 / 16; ++c)
         tmem_st16(tmem + lane_off + b * 128 + c * 16, pk + c * 16);
