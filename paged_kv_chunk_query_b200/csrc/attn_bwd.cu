@@ -69,9 +69,12 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) 
 // ------------------------------------------------------------------ dK / dV
 // One CTA per (KV tile of 128 keys, KV head g); loops over the group's query
 // tiles (G heads x 128-row tiles; for the chunk's own keys only the causally
-// reachable tiles).  Thread r of warps 0-3 owns key r (TMEM lane r).
-// TMEM: S^T [0,128) (then P^T bf16 in [0,64)), dP^T [128,256) (then dS^T in
-// [128,192)), dV [256,256+D), dK [256+D, 256+2D).
+// reachable tiles).  Warps 0-7 compute: warps w and w+4 share keys
+// 32(w%4)..+31 (TMEM lanes); warp w < 4 takes query columns 0-63 (and d
+// columns [0, D/2) in the epilogue), warp w >= 4 the other halves.  Warp 8
+// loads (TMA), warp 9 issues UMMA.
+// TMEM: S^T [0,128) (then P^T bf16: query half k in [64k, 64k+32)), dP^T
+// [128,256) (then dS^T likewise), dV [256,256+D), dK [256+D, 256+2D).
 template <int D>
 struct KvCfg {
   static constexpr int kHalves = D / 64;
@@ -84,7 +87,7 @@ struct KvCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bwd_dkdv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap qmap,
                     const __grid_constant__ CUtensorMap domap,
                     const __grid_constant__ CUtensorMap kvmap) {
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(192, 1)
   };
 
   __shared__ uint64_t bar_kv, bar_qf[Cfg::kNS], bar_qe[Cfg::kNS];
-  __shared__ uint64_t bar_st, bar_dpt, bar_p, bar_ds, bar_acc, bar_drain;
+  __shared__ uint64_t bar_st, bar_sl, bar_dpt, bar_pds, bar_acc, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh, q_issued_sh, q_used_sh, kv_issued_sh;
 
@@ -131,9 +134,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bar_qe[i], 1);
     }
     mbar_init(&bar_st, 1);
+    mbar_init(&bar_sl, 8);
     mbar_init(&bar_dpt, 1);
-    mbar_init(&bar_p, 4);
-    mbar_init(&bar_ds, 4);
+    mbar_init(&bar_pds, 8);
     mbar_init(&bar_acc, 1);
     mbar_init(&bar_drain, 1);
     fence_mbar_init();
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(192, 1)
   const int32_t* past_list = p.past_pages ? p.past_pages + static_cast<size_t>(g) * p.max_past
                                           : nullptr;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&domap);
@@ -187,20 +190,20 @@ __global__ void __launch_bounds__(192, 1)
       if (*abort_flag) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
       q_issued_sh = issued;
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
+      // Order per query tile i: S^T_{i+1} as soon as the compute warps hold S^T_i
+      // in registers; dV_i, dK_i once P^T_i, dS^T_i are in TMEM; then dP^T_{i+1}.
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       int used = 0;
-      bool ok = mbar_wait(&bar_kv, 0, abort_flag);
-      for (int i = 0; ok && i < n_iter; ++i) {
+      auto issue_s = [&](int i) -> bool {  // S^T_i = K Q_i^T
         const int s = i % Cfg::kNS;
-        if (!(ok = mbar_wait(&bar_qf[s], (i / Cfg::kNS) & 1, abort_flag))) break;
+        if (!mbar_wait(&bar_qf[s], (i / Cfg::kNS) & 1, abort_flag)) return false;
         ++used;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ(s)), do_addr = smem_u32(sDO(s));
-        // S^T_i = K Q_i^T
+        const uint32_t q_addr = smem_u32(sQ(s));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
@@ -208,20 +211,10 @@ __global__ void __launch_bounds__(192, 1)
                   sw128_desc(q_addr + off, 16, 1024), idesc_s, kk > 0);
         }
         umma_commit(&bar_st);
-        if (i > 0) {
-          // dK += dS^T_{i-1} Q_{i-1}
-          if (!(ok = mbar_wait(&bar_ds, (i - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          const int sp = (i - 1) % Cfg::kNS;
-          const uint32_t qp = smem_u32(sQ(sp));
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPT + kk * 8,
-                    sw128_desc(qp + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
-                    (i - 1 > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bar_qe[sp]);
-        }
-        // dP^T_i = V dO_i^T
+        return true;
+      };
+      auto issue_dp = [&](int i) {  // dP^T_i = V dO_i^T (its stage is already resident)
+        const uint32_t do_addr = smem_u32(sDO(i % Cfg::kNS));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
@@ -229,30 +222,36 @@ __global__ void __launch_bounds__(192, 1)
                   sw128_desc(do_addr + off, 16, 1024), idesc_s, kk > 0);
         }
         umma_commit(&bar_dpt);
-        // dV += P^T_i dO_i
-        if (!(ok = mbar_wait(&bar_p, i & 1, abort_flag))) break;
+      };
+      bool ok = mbar_wait(&bar_kv, 0, abort_flag);
+      if (ok && n_iter > 0) {
+        ok = issue_s(0);
+        if (ok) issue_dp(0);
+      }
+      for (int i = 0; ok && i < n_iter; ++i) {
+        const int s = i % Cfg::kNS;
+        if (i + 1 < n_iter) {
+          if (!(ok = mbar_wait(&bar_sl, i & 1, abort_flag))) break;
+          if (!(ok = issue_s(i + 1))) break;
+        }
+        if (!(ok = mbar_wait(&bar_pds, i & 1, abort_flag))) break;
         tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ(s)), do_addr = smem_u32(sDO(s));
+        // dV += P^T_i dO_i ; dK += dS^T_i Q_i  (A operands packed in the dP^T columns)
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColST + kk * 8,
+          umma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColDPT + (kk / 4) * 64 + (kk % 4) * 8,
                   sw128_desc(do_addr + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
                   (i > 0 || kk > 0) ? 1u : 0u);
-      }
-      if (ok && n_iter > 0) {
-        const int i = n_iter;
-        if ((ok = mbar_wait(&bar_ds, (i - 1) & 1, abort_flag))) {
-          tc_fence_after();
-          const int sp = (i - 1) % Cfg::kNS;
-          const uint32_t qp = smem_u32(sQ(sp));
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPT + kk * 8,
-                    sw128_desc(qp + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
-                    (i - 1 > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bar_qe[sp]);
-          umma_commit(&bar_acc);
-        }
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPT + (kk / 4) * 64 + 32 + (kk % 4) * 8,
+                  sw128_desc(q_addr + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bar_qe[s]);
+        if (i + 1 < n_iter) issue_dp(i + 1);
       }
+      if (ok && n_iter > 0) umma_commit(&bar_acc);
       if (!ok) {
         *abort_flag = 1;
         atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
@@ -262,8 +261,10 @@ __global__ void __launch_bounds__(192, 1)
       q_used_sh = used;
     }
   } else {
-    const int r = threadIdx.x;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int lg = warp & 3, half = warp >> 2;  // lane group, query/d column half
+    const int r = lg * 32 + lane;               // key row (TMEM lane)
+    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+    const uint32_t cs = half * 64;              // this half's columns in S^T / dP^T
     bool key_valid;
     if (is_past) key_valid = j * kTile + r < sch.n_past_pages * p.P;
     else key_valid = u * kTile + r < p.C;
@@ -275,19 +276,23 @@ __global__ void __launch_bounds__(192, 1)
       if (!(ok = warp_wait(&bar_st, i & 1, abort_flag))) break;
       if (!(ok = warp_wait(&bar_qf[s], (i / Cfg::kNS) & 1, abort_flag))) break;
       tc_fence_after();
-      float pr[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c)
-        tmem_ld32(tmem + lane_off + Cfg::kColST + c * 32, reinterpret_cast<uint32_t*>(pr + c * 32));
+      float pr[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColST + cs, reinterpret_cast<uint32_t*>(pr));
+      tmem_ld32(tmem + lane_off + Cfg::kColST + cs + 32, reinterpret_cast<uint32_t*>(pr + 32));
       tmem_ld_wait();
-      const float* L = sL(s);
-      // query column c is valid if inside the chunk and (current tile) causally after the key
-      const int cmax = min(kTile, p.C - t * kTile);  // columns [0, cmax) are inside the chunk
-      const int cmin = is_past ? 0 : key_local - t * kTile;  // q_local >= key_local
-      const bool full = key_valid && cmin <= 0 && cmax >= kTile;
+      // S^T_i is in registers: the next S^T may overwrite its columns
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sl);
+      const float* L = sL(s) + cs;
+      // query column c (of this half) is valid if inside the chunk and, for the
+      // chunk's own keys, causally at or after the key
+      const int cmax = min(kTile, p.C - t * kTile) - static_cast<int>(cs);
+      const int cmin = (is_past ? 0 : key_local - t * kTile) - static_cast<int>(cs);
+      const bool full = key_valid && cmin <= 0 && cmax >= 64;
       // P^T = 2^(S^T*scale*log2e - LSE*log2e); LSE read 4 at a time (broadcast)
 #pragma unroll
-      for (int c4 = 0; c4 < kTile / 4; ++c4) {
+      for (int c4 = 0; c4 < 16; ++c4) {
         const float4 l4 = *reinterpret_cast<const float4*>(L + 4 * c4);
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
@@ -298,50 +303,43 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          pr[c] = (key_valid && c < cmax && c >= cmin) ? pr[c] : 0.f;
+        for (int c = 0; c < 64; ++c) pr[c] = (key_valid && c < cmax && c >= cmin) ? pr[c] : 0.f;
       }
-      uint32_t pk[kTile / 2];
-#pragma unroll
-      for (int c = 0; c < kTile / 2; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-#pragma unroll
-      for (int c = 0; c < kTile / 2 / 16; ++c)
-        tmem_st16(tmem + lane_off + Cfg::kColST + c * 16, pk + c * 16);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_p);
-
       if (!(ok = warp_wait(&bar_dpt, i & 1, abort_flag))) break;
       tc_fence_after();
-      const float* Dl = sDl(s);
+      uint32_t dp[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColDPT + cs, dp);
+      tmem_ld32(tmem + lane_off + Cfg::kColDPT + cs + 32, dp + 32);
+      tmem_ld_wait();
+      const float* Dl = sDl(s) + cs;
+      uint32_t dsk[32];
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t dp[32];
-        tmem_ld32(tmem + lane_off + Cfg::kColDPT + c * 32, dp);
-        tmem_ld_wait();
-        uint32_t dk[16];
+      for (int e4 = 0; e4 < 16; ++e4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(Dl + 4 * e4);
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float ds[4];
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(Dl + c * 32 + 4 * e4);
-          const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-          float ds[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c0 = c * 32 + 4 * e4 + e;
-            ds[e] = pr[c0] * (__uint_as_float(dp[4 * e4 + e]) - dv[e]);
-            // masked columns may hold stale delta values: force an exact zero
-            if (!full) ds[e] = pr[c0] != 0.f ? ds[e] : 0.f;
-          }
-          dk[2 * e4] = pack_bf16(ds[0], ds[1]);
-          dk[2 * e4 + 1] = pack_bf16(ds[2], ds[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = 4 * e4 + e;
+          ds[e] = pr[c0] * (__uint_as_float(dp[c0]) - dv[e]);
+          // masked columns may hold stale delta values: force an exact zero
+          if (!full) ds[e] = pr[c0] != 0.f ? ds[e] : 0.f;
         }
-        tmem_st16(tmem + lane_off + Cfg::kColDPT + c * 16, dk);
+        dsk[2 * e4] = pack_bf16(ds[0], ds[1]);
+        dsk[2 * e4 + 1] = pack_bf16(ds[2], ds[3]);
       }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+      // P^T and dS^T (bf16) into this half's dP^T columns, already read
+      tmem_st16(tmem + lane_off + Cfg::kColDPT + cs, pk);
+      tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 16, pk + 16);
+      tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 32, dsk);
+      tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 48, dsk + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_ds);
+      if (lane == 0) mbar_arrive(&bar_pds);
     }
     if (ok && n_iter > 0) ok = warp_wait(&bar_acc, 0, abort_flag);
     if (!ok) {
@@ -355,13 +353,14 @@ __global__ void __launch_bounds__(192, 1)
                          p.num_pool_pages, p.status);
       const bool write = key_valid && page >= 0 && page < p.num_pool_pages;
       const size_t blk = (static_cast<size_t>(write ? page : 0) * p.Hkv + g) * 2;
-      float* gk = p.grad + (blk * p.P + r % p.P) * D;
-      float* gv = p.grad + ((blk + 1) * p.P + r % p.P) * D;
+      const int d0 = half * (D / 2);
+      float* gk = p.grad + (blk * p.P + r % p.P) * D + d0;
+      float* gv = p.grad + ((blk + 1) * p.P + r % p.P) * D + d0;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tmem + lane_off + Cfg::kColDK + c * 32, a);
-        tmem_ld32(tmem + lane_off + Cfg::kColDV + c * 32, b);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t a[32], bb[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColDK + d0 + c * 32, a);
+        tmem_ld32(tmem + lane_off + Cfg::kColDV + d0 + c * 32, bb);
         tmem_ld_wait();
         if (write) {
 #pragma unroll
@@ -372,8 +371,8 @@ __global__ void __launch_bounds__(192, 1)
                                   __uint_as_float(a[4 * e + 2]) * p.scale,
                                   __uint_as_float(a[4 * e + 3]) * p.scale));
             atomicAdd(reinterpret_cast<float4*>(gv + c * 32 + 4 * e),
-                      make_float4(__uint_as_float(b[4 * e]), __uint_as_float(b[4 * e + 1]),
-                                  __uint_as_float(b[4 * e + 2]), __uint_as_float(b[4 * e + 3])));
+                      make_float4(__uint_as_float(bb[4 * e]), __uint_as_float(bb[4 * e + 1]),
+                                  __uint_as_float(bb[4 * e + 2]), __uint_as_float(bb[4 * e + 3])));
           }
         }
       }
@@ -382,7 +381,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     // Loads that were issued but never consumed must land before the CTA exits.
     if (kv_issued_sh && (abort_sh || n_iter == 0)) mbar_wait_drain(&bar_kv, 0);
     if (abort_sh)
@@ -397,20 +396,27 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ------------------------------------------------------------------ dQ
-// One CTA per (128-row query tile, head).  TMEM: S0 [0,128), S1 [128,256),
-// dP [256,384) (then dS bf16 in [256,320)), dQ [384, 384+D).
+// One CTA per (128-row query tile, head).  Two slots walk the KV tiles in
+// turn (slot 0 the even tiles, slot 1 the odd ones), so one slot's softmax
+// overlaps the other slot's UMMAs.  Warps 0-3 serve slot 0 and warps 4-7
+// slot 1 (thread = query row = TMEM lane, all 128 key columns); warp 8 loads
+// (TMA), warp 9 issues UMMA in the order
+//   S(0) S(1) dP(0) | dQ(j) dP(j+1) S(j+2) for j = 0, 1, ...
+// TMEM: S of slot s [128s, 128s+128) (its dS, bf16, overwrites [128s, +64)
+// once S is in registers); dP [256,384) shared by the slots in turn; dQ
+// [384, 384+D).
 template <int D>
 struct QCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kNK = 2, kNV = 2;
+  static constexpr int kNK = 3, kNV = 2;
   static constexpr int kSmem = kTileBytes * (2 + kNK + kNV) + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColDP = 256, kColDQ = 384;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap domap,
                   const __grid_constant__ CUtensorMap kvmap) {
@@ -425,7 +431,7 @@ __global__ void __launch_bounds__(192, 1)
 
   __shared__ uint64_t bar_q, bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV],
       bar_ve[Cfg::kNV];
-  __shared__ uint64_t bar_s[2], bar_dp, bar_ds, bar_fin, bar_drain;
+  __shared__ uint64_t bar_s[2], bar_dp[2], bar_ds[2], bar_fin, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh, k_issued_sh, v_issued_sh, k_used_sh, v_used_sh;
 
@@ -447,10 +453,11 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bar_vf[i], 1);
       mbar_init(&bar_ve[i], 1);
     }
-    mbar_init(&bar_s[0], 1);
-    mbar_init(&bar_s[1], 1);
-    mbar_init(&bar_dp, 1);
-    mbar_init(&bar_ds, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_dp[i], 1);
+      mbar_init(&bar_ds[i], 4);
+    }
     mbar_init(&bar_fin, 1);
     mbar_init(&bar_drain, 1);
     fence_mbar_init();
@@ -465,7 +472,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&domap);
@@ -505,14 +512,14 @@ __global__ void __launch_bounds__(192, 1)
       k_issued_sh = k_issued;
       v_issued_sh = v_issued;
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       int k_used = 0, v_used = 0;
-      auto issue_s = [&](int j) -> bool {
+      auto issue_s = [&](int j) -> bool {  // S(j) into slot j&1
         const int ks = j % Cfg::kNK;
         if (!mbar_wait(&bar_kf[ks], (j / Cfg::kNK) & 1, abort_flag)) return false;
         ++k_used;
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit(&bar_s[j & 1]);
         return true;
       };
-      auto issue_dp = [&](int j) -> bool {
+      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T into the shared dP buffer
         const int vs = j % Cfg::kNV;
         if (!mbar_wait(&bar_vf[vs], (j / Cfg::kNV) & 1, abort_flag)) return false;
         ++v_used;
@@ -540,24 +547,25 @@ __global__ void __launch_bounds__(192, 1)
                   sw128_desc(vb + off, 16, 1024), idesc_s, kk > 0);
         }
         umma_commit(&bar_ve[vs]);
-        umma_commit(&bar_dp);
+        umma_commit(&bar_dp[j & 1]);
         return true;
       };
       bool ok = mbar_wait(&bar_q, 0, abort_flag);
-      ok = ok && issue_s(0) && issue_dp(0);
+      ok = ok && issue_s(0) && (T < 2 || issue_s(1)) && issue_dp(0);
       for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(&bar_ds, j & 1, abort_flag))) break;
+        // dQ += dS(j) K_j, dS(j) packed in its slot's S columns
+        if (!(ok = mbar_wait(&bar_ds[j & 1], (j >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const int ks = j % Cfg::kNK;
         const uint32_t kb = k_addr + ks * Cfg::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * 8,
+          umma_ts(tmem + Cfg::kColDQ, tmem + (j & 1) * 128 + kk * 8,
                   sw128_desc(kb + kk * 16 * 128, kTile * 128, 1024), idesc_dq,
                   (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bar_ke[ks]);
         if (j + 1 < T && !(ok = issue_dp(j + 1))) break;
+        if (j + 2 < T && !(ok = issue_s(j + 2))) break;
       }
       if (ok) umma_commit(&bar_fin);
       if (!ok) {
@@ -570,22 +578,24 @@ __global__ void __launch_bounds__(192, 1)
       v_used_sh = v_used;
     }
   } else {
-    const int r = threadIdx.x;
+    const int slot = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;  // query row (TMEM lane)
     const int q_local = qt * kTile + r;
     const bool row_valid = q_local < p.C;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t col_s = slot * 128;
     const float lse2 = row_valid ? p.lse[static_cast<size_t>(h) * p.C + q_local] * kLog2e : 0.f;
     const float dl = row_valid ? p.delta[static_cast<size_t>(h) * p.C + q_local] : 0.f;
     const int n_past_keys = sch.n_past_pages * p.P;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int b = j & 1;
-      if (!(ok = warp_wait(&bar_s[b], (j >> 1) & 1, abort_flag))) break;
+    for (int j = slot; j < T; j += 2) {
+      const int use = j >> 1;  // this slot's use count
+      if (!(ok = warp_wait(&bar_s[slot], use & 1, abort_flag))) break;
       tc_fence_after();
       float pr[kTile];
 #pragma unroll
       for (int c = 0; c < kTile / 32; ++c)
-        tmem_ld32(tmem + lane_off + b * 128 + c * 32, reinterpret_cast<uint32_t*>(pr + c * 32));
+        tmem_ld32(tmem + lane_off + col_s + c * 32, reinterpret_cast<uint32_t*>(pr + c * 32));
       tmem_ld_wait();
       int lim;
       if (j < sch.n_past_tiles) lim = n_past_keys - j * kTile;
@@ -597,7 +607,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c = 0; c < kTile; ++c) pr[c] = c < lim ? pr[c] : 0.f;
       }
-      if (!(ok = warp_wait(&bar_dp, j & 1, abort_flag))) break;
+      if (!(ok = warp_wait(&bar_dp[slot], use & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < kTile / 32; ++c) {
@@ -611,12 +621,12 @@ __global__ void __launch_bounds__(192, 1)
           ds[e] = pack_bf16(pr[c0] * (__uint_as_float(dp[2 * e]) - dl),
                             pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - dl));
         }
-        tmem_st16(tmem + lane_off + Cfg::kColDP + c * 16, ds);
+        tmem_st16(tmem + lane_off + col_s + c * 16, ds);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_ds);
+      if (lane == 0) mbar_arrive(&bar_ds[slot]);
     }
     if (ok) ok = warp_wait(&bar_fin, 0, abort_flag);
     if (!ok) {
@@ -624,11 +634,12 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
     } else {
       tc_fence_after();
-      __nv_bfloat16* row = p.dq + (static_cast<size_t>(q_local) * p.Hq + h) * D;
+      const int d0 = slot * (D / 2);  // each slot writes half of the row
+      __nv_bfloat16* row = p.dq + (static_cast<size_t>(q_local) * p.Hq + h) * D + d0;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t a[32];
-        tmem_ld32(tmem + lane_off + Cfg::kColDQ + c * 32, a);
+        tmem_ld32(tmem + lane_off + Cfg::kColDQ + d0 + c * 32, a);
         tmem_ld_wait();
         if (row_valid) {
           uint32_t pk[16];
@@ -647,7 +658,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (abort_sh && warp == 4 && lane == 0) {
+  if (abort_sh && warp == 8 && lane == 0) {
     for (int i = k_used_sh; i < k_issued_sh; ++i)
       mbar_wait_drain(&bar_kf[i % Cfg::kNK], (i / Cfg::kNK) & 1);
     for (int i = v_used_sh; i < v_issued_sh; ++i)
@@ -729,12 +740,12 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
       return OOMB_ERR_CUDA;
     if (step < 0 || step == OOMB_BWD_DKDV) {
       dim3 grid(p.max_past_tiles + s.n_qtiles, s.Hkv);
-      bwd_dkdv_kernel<D><<<grid, 192, KvCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
+      bwd_dkdv_kernel<D><<<grid, 320, KvCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
       if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
     }
     if (step < 0 || step == OOMB_BWD_DQ) {
       dim3 grid(s.n_qtiles, s.Hq);
-      bwd_dq_kernel<D><<<grid, 192, QCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
+      bwd_dq_kernel<D><<<grid, 320, QCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
       if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
     }
   }
