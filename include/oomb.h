@@ -183,6 +183,28 @@ oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk
                            int32_t* d_out_physical, int32_t* d_out_count, float* d_out_scores,
                            void* d_workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of oomb_page_topk (this one has no counterpart in
+ * the paper; it exists for callers that cannot allocate device memory, e.g.
+ * code running under a host framework that owns every device allocation, or a
+ * latency-critical loop that must not call cudaMalloc, which can synchronise
+ * the device).  Same arguments and results as oomb_page_topk minus the
+ * workspace: the scratch is a static device array of
+ * OOMB_TOPK_STATIC_SCRATCH_BYTES inside the library, held on every GPU that
+ * loads it until the process exits.  Returns OOMB_ERR_UNSUPPORTED when
+ * oomb_page_topk_workspace_size() of the call exceeds that size (e.g. with
+ * Hkv = 4 and d = 128, n_past up to 28,672 pages fits).  It allocates nothing.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All calls
+ * share the one array: calls that overlap on the GPU (different streams) race
+ * on it and must be ordered by the caller.  No scratch word needs clearing:
+ * each call writes what it reads. */
+#define OOMB_TOPK_STATIC_SCRATCH_BYTES (1u << 20)
+oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* d_q, int32_t chunk_len,
+                                  int32_t num_q_heads, const int32_t* d_page_table,
+                                  int32_t n_past, int32_t top_k, int32_t n_recent,
+                                  int32_t* d_out_logical, int32_t* d_out_physical,
+                                  int32_t* d_out_count, float* d_out_scores, void* stream);
+
 /* ---------------------------------------------------------------- offload
  * A block is the K and V of one page and one KV head: block id = page *
  * num_kv_heads + head, contiguous in both pools ([pt] §2D, [it] §2C: KV and

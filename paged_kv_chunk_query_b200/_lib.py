@@ -33,7 +33,7 @@ EXPORTS = (
     "oomb_chunk_attn_fwd", "oomb_chunk_attn_bwd", "oomb_chunk_attn_bwd_step",
     "oomb_page_topk_workspace_size", "oomb_page_topk", "oomb_page_prefetch",
     "oomb_grad_writeback", "oomb_wait", "oomb_get_device_status", "oomb_status_string",
-    "oomb_version",
+    "oomb_version", "oomb_page_topk_static",
 )
 
 
@@ -85,6 +85,7 @@ def load() -> ctypes.CDLL:
         "oomb_chunk_attn_bwd_step": [vp, ctypes.POINTER(AttnArgs), i32, vp],
         "oomb_page_topk": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp,
                            ctypes.c_size_t, vp],
+        "oomb_page_topk_static": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp],
         "oomb_page_prefetch": [vp, vp, vp, vp, i32, vp, vp],
         "oomb_grad_writeback": [vp, vp, vp, vp, i32, vp],
         "oomb_wait": [vp, ctypes.c_int64],
@@ -276,6 +277,24 @@ def page_topk(pool, q, page_table, n_past, top_k, n_recent, out_logical, out_phy
         _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
         _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "oomb_page_topk")
+
+
+TOPK_STATIC_SCRATCH_BYTES = 1 << 20
+
+
+def page_topk_static(pool, q, page_table, n_past, top_k, n_recent, out_logical, out_physical,
+                     out_count, out_scores=None, stream=None):
+    """oomb_page_topk_static: Top-K with the library's static scratch (no
+    workspace argument; allocates nothing)."""
+    C, Hq, _ = q.shape
+    _check(load().oomb_page_topk_static(
+        pool, _dev_tensor(q, torch.bfloat16, "q"), C, Hq,
+        _dev_tensor(page_table, torch.int32, "page_table") if n_past else None, n_past, top_k,
+        n_recent, _dev_tensor(out_logical, torch.int32, "out_logical"),
+        _dev_tensor(out_physical, torch.int32, "out_physical") if out_physical is not None
+        else None, _dev_tensor(out_count, torch.int32, "out_count"),
+        _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
+        _stream(stream)), "oomb_page_topk_static")
 
 
 def _host_i32(blocks):

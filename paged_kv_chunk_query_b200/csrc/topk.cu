@@ -22,6 +22,8 @@
 //   compacts the kept ids in ascending order.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "internal.h"
 
 namespace {
@@ -305,6 +307,96 @@ extern "C" oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, in
   float* partial = static_cast<float*>(d_workspace);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(
       static_cast<uint8_t*>(d_workspace) + align256(static_cast<size_t>(kSplits) * Hkv * D * 4));
+  const int G = num_q_heads / Hkv;
+  const float inv_rows = 1.0f / (static_cast<float>(chunk_len) * static_cast<float>(G));
+  const auto* q = static_cast<const __nv_bfloat16*>(d_q);
+  dim3 g1(kSplits, Hkv), g2((n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv);
+  if (D == 128) {
+    qmean_partial_kernel<128><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
+    if (n_past > 0)
+      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
+                                                          n_past, Hkv, d.num_pages, inv_rows,
+                                                          keys, d_out_scores, pool->d_status);
+  } else {
+    qmean_partial_kernel<64><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
+    if (n_past > 0)
+      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
+                                                         n_past, Hkv, d.num_pages, inv_rows, keys,
+                                                         d_out_scores, pool->d_status);
+  }
+  topk_select_kernel<<<Hkv, kSelectThreads, 0, s>>>(keys, d_page_table, n_past, top_k, n_recent,
+                                                     d.num_pages, d_out_logical, d_out_physical,
+                                                     d_out_count);
+  return oomb::check_launch();
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+// Some callers of this library cannot allocate device memory: a host
+// framework that owns every device allocation and forbids side allocations,
+// or a latency-critical loop in which a cudaMalloc (which may synchronise the
+// device) is not acceptable.  oomb_page_topk_static serves them: it is
+// oomb_page_topk with its scratch (query-mean partials and 64-bit page keys)
+// taken from the file-scope device array below instead of a caller workspace.
+// Every GPU that loads the library holds this array until the process exits.
+// All calls share it and it keeps the last call's contents; the kernels write
+// every scratch word before reading it, so nothing needs clearing, but calls
+// that overlap on the GPU (on different streams) race on it.
+namespace {
+
+static __device__ __align__(256) uint8_t g_topk_static_scratch[OOMB_TOPK_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once
+// per device; the host-side name is only a stand-in, not a device address).
+oomb_status static_scratch(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return OOMB_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_addr[device]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_topk_static_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return OOMB_ERR_CUDA;
+    }
+    g_static_addr[device] = p;
+  }
+  *out = g_static_addr[device];
+  return OOMB_OK;
+}
+
+}  // namespace
+
+extern "C" oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* d_q,
+                                             int32_t chunk_len, int32_t num_q_heads,
+                                             const int32_t* d_page_table, int32_t n_past,
+                                             int32_t top_k, int32_t n_recent,
+                                             int32_t* d_out_logical, int32_t* d_out_physical,
+                                             int32_t* d_out_count, float* d_out_scores,
+                                             void* stream) {
+  if (!pool || pool->desc.location == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
+  const oomb_pool_desc& d = pool->desc;
+  const int Hkv = d.num_kv_heads, D = d.head_dim;
+  if (!d_q || !d_out_logical || !d_out_count) return OOMB_ERR_INVALID_ARG;
+  if (chunk_len <= 0 || num_q_heads <= 0 || num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
+  if (n_past < 0 || n_past > 65536 || top_k < 0 || n_recent < 0 || top_k + n_recent > 4096 ||
+      top_k + n_recent == 0)
+    return OOMB_ERR_INVALID_ARG;
+  if (n_past > 0 && !d_page_table) return OOMB_ERR_INVALID_ARG;
+  if (!oomb::aligned16(d_q)) return OOMB_ERR_INVALID_ARG;
+  // the scratch array has a fixed size: larger problems must use oomb_page_topk
+  if (oomb_page_topk_workspace_size(chunk_len, num_q_heads, Hkv, D, n_past) >
+      OOMB_TOPK_STATIC_SCRATCH_BYTES)
+    return OOMB_ERR_UNSUPPORTED;
+  oomb::DeviceGuard guard(d.device);
+  void* scratch = nullptr;
+  const oomb_status st = static_scratch(d.device, &scratch);
+  if (st != OOMB_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* partial = static_cast<float*>(scratch);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(
+      static_cast<uint8_t*>(scratch) + align256(static_cast<size_t>(kSplits) * Hkv * D * 4));
   const int G = num_q_heads / Hkv;
   const float inv_rows = 1.0f / (static_cast<float>(chunk_len) * static_cast<float>(G));
   const auto* q = static_cast<const __nv_bfloat16*>(d_q);
