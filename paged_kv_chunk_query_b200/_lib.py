@@ -190,18 +190,15 @@ class _CudaArray:
 
 
 def pool_views(pool: int):
-    """Torch views (kv, grad, summary) of a device pool's buffers, borrowed: they
-    are valid until pool_destroy.  Host pools give CPU tensors."""
+    """Torch views (kv, grad, summary) of a pool's buffers, borrowed: valid until
+    pool_destroy.  Device pools give CUDA tensors; pinned-host pools give CPU
+    tensors for kv and grad and a CUDA tensor for the summaries (which the
+    library keeps on the device); host pools give CPU tensors."""
     d = pool_get_desc(pool)
     kv, grad, summ = pool_buffers(pool)
     shape = (d.num_pages, d.num_kv_heads, 2, d.page_size, d.head_dim)
     sshape = (d.num_pages, d.num_kv_heads, d.head_dim)
-    if d.location == LOC_DEVICE:
-        dev = torch.device("cuda", d.device)
-        t_kv = torch.as_tensor(_CudaArray(kv, shape, "<i2"), device=dev).view(torch.bfloat16)
-        t_g = torch.as_tensor(_CudaArray(grad, shape, "<f4"), device=dev) if grad else None
-        t_s = torch.as_tensor(_CudaArray(summ, sshape, "<f4"), device=dev)
-        return t_kv, t_g, t_s
+    dev = torch.device("cuda", d.device)
 
     def host(ptr, shp, ctype, dt):
         n = 1
@@ -210,10 +207,30 @@ def pool_views(pool: int):
         buf = (ctype * n).from_address(ptr)
         return torch.frombuffer(buf, dtype=dt).view(shp)
 
+    if d.location == LOC_DEVICE:
+        t_kv = torch.as_tensor(_CudaArray(kv, shape, "<i2"), device=dev).view(torch.bfloat16)
+        t_g = torch.as_tensor(_CudaArray(grad, shape, "<f4"), device=dev) if grad else None
+        t_s = torch.as_tensor(_CudaArray(summ, sshape, "<f4"), device=dev)
+        return t_kv, t_g, t_s
     t_kv = host(kv, shape, ctypes.c_int16, torch.int16).view(torch.bfloat16)
     t_g = host(grad, shape, ctypes.c_float, torch.float32) if grad else None
-    t_s = host(summ, sshape, ctypes.c_float, torch.float32)
+    if d.location == LOC_PINNED_HOST:
+        t_s = torch.as_tensor(_CudaArray(summ, sshape, "<f4"), device=dev)
+    else:
+        t_s = host(summ, sshape, ctypes.c_float, torch.float32)
     return t_kv, t_g, t_s
+
+
+def _event_handle(event, stream):
+    """Raw cudaEvent_t of a torch.cuda.Event.  torch creates the CUDA event on
+    its first record, so an event never recorded is recorded once here to
+    exist (the library records it again after its own work)."""
+    if event is None:
+        return None
+    if not event.cuda_event:
+        event.record(stream if isinstance(stream, torch.cuda.Stream)
+                     else torch.cuda.current_stream())
+    return event.cuda_event
 
 
 # ------------------------------------------------------------------- compute
@@ -305,7 +322,7 @@ def _host_i32(blocks):
 def page_prefetch(host_pool, device_pool, src_blocks, dst_blocks, stream=None, done_event=None):
     s, sp = _host_i32(src_blocks)
     d, dp = _host_i32(dst_blocks)
-    ev = done_event.cuda_event if done_event is not None else None
+    ev = _event_handle(done_event, stream)
     _check(load().oomb_page_prefetch(host_pool, device_pool, sp, dp, s.numel(), _stream(stream),
                                      ev), "oomb_page_prefetch")
 
@@ -318,7 +335,7 @@ def grad_writeback(device_pool, host_pool, src_blocks, dst_blocks, stream=None):
 
 
 def wait(event, timeout_us: int):
-    _check(load().oomb_wait(event.cuda_event, timeout_us), "oomb_wait")
+    _check(load().oomb_wait(event.cuda_event or None, timeout_us), "oomb_wait")
 
 
 def get_device_status(pool) -> int:

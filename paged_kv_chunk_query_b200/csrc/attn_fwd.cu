@@ -5,22 +5,17 @@
 // query rows of one head and walks the KV tiles of its group: the listed past
 // pages (all visible) and then the chunk's own pages (causal).
 //
-// Warp roles (320 threads):
-//   warps 0-7  softmax: warps w and w+4 share query rows 32(w%4)..+31 (TMEM
-//              lanes); warp w < 4 takes the tile's key columns 0-63 and O
-//              columns [0, D/2), warp w >= 4 the other halves.  Each thread
-//              reads its 64 logits from TMEM; the two halves of a row swap
-//              their maxima through shared memory (a per-pair mbarrier, two
-//              slots) so both take identical rescale decisions; P (bf16) goes
-//              back into the half's own TMEM columns; O is rescaled when the
-//              max grows; finally O is normalised and written with the LSE.
-//   warp 8     TMA producer: Q once, then K and V tiles page by page through
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Reads S from
+//              TMEM, keeps the running max / sum, writes P (bf16) back into the
+//              same TMEM columns, rescales O when the max grows, and finally
+//              normalises O and writes O and the LSE.
+//   warp 4     TMA producer: Q once, then K and V tiles page by page through
 //              a 4-D tensor map over the pool (page id = outermost coordinate).
-//   warp 9     UMMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
+//   warp 5     UMMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
 //              buffers, O += P_j V_j with P read from TMEM (A operand) and V
 //              from shared memory (MN-major B operand).
-// TMEM: S0 [0,128), S1 [128,256), O [256, 256+D).  P of key half k sits in
-// packed bf16 columns [64k, 64k+32) of its S buffer.
+// TMEM: S0 [0,128), S1 [128,256), O [256, 256+D).
 //
 // Online softmax in base 2: s2 = S * scale * log2(e).  The running maximum is
 // only moved when a tile's maximum exceeds it by more than 8 (a factor 256),
@@ -62,7 +57,7 @@ struct FwdCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(192, 1)
     attn_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap qmap,
                     const __grid_constant__ CUtensorMap kvmap) {
   using Cfg = FwdCfg<D>;
@@ -76,8 +71,6 @@ __global__ void __launch_bounds__(320, 1)
   __shared__ uint64_t bar_q, bar_drain, bar_o, bar_fin;
   __shared__ uint64_t bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV], bar_ve[Cfg::kNV];
   __shared__ uint64_t bar_s[2], bar_p[2];
-  __shared__ uint64_t bar_x[4];           // row-pair exchange, one per lane group
-  __shared__ float xch[2][2][kTile];      // [slot][half][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ int k_issued_sh, v_issued_sh, k_used_sh, v_used_sh;
@@ -105,9 +98,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_p[i], 8);
+      mbar_init(&bar_p[i], 4);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&bar_x[i], 2);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -120,7 +112,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
 
-  if (warp == 8) {
+  if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&qmap);
@@ -159,7 +151,7 @@ __global__ void __launch_bounds__(320, 1)
       k_issued_sh = k_issued;
       v_issued_sh = v_issued;
     }
-  } else if (warp == 9) {
+  } else if (warp == 5) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
@@ -193,7 +185,7 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t vb = v_addr + vs * Cfg::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tmem + Cfg::kColO, tmem + b * 128 + (kk / 4) * 64 + (kk % 4) * 8,
+            umma_ts(tmem + Cfg::kColO, tmem + b * 128 + kk * 8,
                     sw128_desc(vb + kk * 16 * 128, kTile * 128, 1024), idesc_pv,
                     (jp > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&bar_ve[vs]);
@@ -213,30 +205,20 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int lg = warp & 3, half = warp >> 2;  // lane group, key/O column half
-    const int r = lg * 32 + lane;               // query row (TMEM lane)
+    const int r = threadIdx.x;  // 0..127
     const int q_local = qt * kTile + r;
-    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
-    const uint32_t col_s = half * 64;           // this half's S columns in a buffer
-    const uint32_t col_o = Cfg::kColO + half * (D / 2);
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int n_past_keys = sch.n_past_pages * p.P;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    // swap one float per row with the partner warp; slot alternates by use
-    auto exchange = [&](float mine, int use) -> float {
-      xch[use & 1][half][r] = mine;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_x[lg]);
-      if (!warp_wait(&bar_x[lg], use & 1, abort_flag)) return NAN;
-      return xch[use & 1][half ^ 1][r];
-    };
     for (int j = 0; j < T; ++j) {
       const int b = j & 1;
       if (!(ok = warp_wait(&bar_s[b], (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      float s[64];
-      tmem_ld32(tmem + lane_off + b * 128 + col_s, reinterpret_cast<uint32_t*>(s));
-      tmem_ld32(tmem + lane_off + b * 128 + col_s + 32, reinterpret_cast<uint32_t*>(s + 32));
+      float s[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c)
+        tmem_ld32(tmem + lane_off + b * 128 + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
       tmem_ld_wait();
       int lim;
       if (j < sch.n_past_tiles) {
@@ -245,26 +227,18 @@ __global__ void __launch_bounds__(320, 1)
         const int key0 = (j - sch.n_past_tiles) * kTile;
         lim = min(p.C, q_local + 1) - key0;
       }
-      lim -= half * 64;  // in this half's columns
-      if (lim < 64) {    // diagonal or ragged tile: keys at and past `lim` are masked
+      if (lim < kTile) {  // diagonal or ragged tile: keys at and past `lim` are masked
 #pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+        for (int c = 0; c < kTile; ++c) s[c] = c < lim ? s[c] : -INFINITY;
       }
-      // row max: 8 independent chains, then the partner half's maximum
+      // row max with 8 independent chains (raw logits; scale > 0 keeps the order)
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-      for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-      const float mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      const float mo = exchange(mh, j);
-      if (mo != mo && *abort_flag) {  // exchange gave up
-        ok = false;
-        break;
-      }
-      // both halves combine the same two values in the same order
-      const float mt = (half == 0 ? fmaxf(mh, mo) : fmaxf(mo, mh)) * p.scale_log2;
+      for (int c = 8; c < kTile; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
       const bool need = mt > m_used + kRescaleThreshold;
       const float m_new = need ? mt : m_used;
       const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
@@ -275,13 +249,13 @@ __global__ void __launch_bounds__(320, 1)
         if (!(ok = warp_wait(&bar_o, (j - 1) & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + col_o + c * 32, o);
+          tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tmem + lane_off + col_o + c * 32, o);
+          tmem_st32(tmem + lane_off + Cfg::kColO + c * 32, o);
         }
         tmem_st_wait();
       }
@@ -291,41 +265,36 @@ __global__ void __launch_bounds__(320, 1)
       float l8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) l8[e] = 0.f;
-      uint32_t pk[32];
+      uint32_t pk[kTile / 2];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < kTile / 2; ++c) {
         const float p0 = fast_exp2(fmaf(s[2 * c], p.scale_log2, neg_mref));
         const float p1 = fast_exp2(fmaf(s[2 * c + 1], p.scale_log2, neg_mref));
         l8[c & 7] += p0 + p1;
         pk[c] = pack_bf16(p0, p1);
       }
       l = l * alpha + (((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7])));
-      tmem_st16(tmem + lane_off + b * 128 + col_s, pk);
-      tmem_st16(tmem + lane_off + b * 128 + col_s + 16, pk + 16);
+#pragma unroll
+      for (int c = 0; c < kTile / 2 / 16; ++c)
+        tmem_st16(tmem + lane_off + b * 128 + c * 16, pk + c * 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_p[b]);
     }
     if (ok) ok = warp_wait(&bar_fin, 0, abort_flag);
-    float l_row = 0.f;
-    if (ok) {
-      const float lo = exchange(l, T);
-      ok = !(lo != lo && *abort_flag);
-      l_row = half == 0 ? l + lo : lo + l;  // fixed order in both halves
-    }
     if (!ok) {
       *abort_flag = 1;
       if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
     } else {
       tc_fence_after();
-      const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool valid = q_local < p.C;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D + half * (D / 2);
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + col_o + c * 32, o);
+        tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
         tmem_ld_wait();
         if (valid) {
           uint32_t pk[16];
@@ -338,15 +307,14 @@ __global__ void __launch_bounds__(320, 1)
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (valid && half == 0)
-        p.lse[static_cast<size_t>(h) * p.C + q_local] = kLn2 * (m_used + log2f(l_row));
+      if (valid) p.lse[static_cast<size_t>(h) * p.C + q_local] = kLn2 * (m_used + log2f(l));
     }
   }
 
   tc_fence_before();
   __syncthreads();
   // After an abort, wait (bounded) for TMA loads still landing in shared memory.
-  if (abort_sh && warp == 8 && lane == 0) {
+  if (abort_sh && warp == 4 && lane == 0) {
     for (int i = k_used_sh; i < k_issued_sh; ++i)
       mbar_wait_drain(&bar_kf[i % Cfg::kNK], (i / Cfg::kNK) & 1);
     for (int i = v_used_sh; i < v_issued_sh; ++i)
@@ -405,7 +373,7 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.num_pool_pages = pool->desc.num_pages;
   p.scale_log2 = a->softmax_scale * kLog2e;
   dim3 grid(s.n_qtiles, s.Hq);
-  attn_fwd_kernel<D><<<grid, 320, Cfg::kSmem, stream>>>(p, qmap, kvmap);
+  attn_fwd_kernel<D><<<grid, 192, Cfg::kSmem, stream>>>(p, qmap, kvmap);
   return check_launch();
 }
 
