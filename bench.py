@@ -339,6 +339,43 @@ def e2e_dense(w, steps, device):
         pk.pool_destroy(pool)
 
 
+def offload_run(w, steps, device, dist_on):
+    """1M-token Top-K run with every page's KV and gradients in pinned host
+    memory (selected pages prefetched into an HBM staging pool on a copy
+    stream, gradient deltas written back asynchronously).  One step = all
+    chunks, timed with CUDA events on the compute stream, max over ranks."""
+    from paged_kv_chunk_query_b200 import synth
+    from paged_kv_chunk_query_b200.offload import OffloadRun
+    ins = [synth.device_chunk_inputs(w, c, device) for c in range(w.num_chunks)]
+    run = OffloadRun(w, device)
+    try:
+        run.run(lambda c: ins[c])  # warm-up pass (also fills the host pools)
+        torch.cuda.synchronize()
+        run.h2d_bytes = run.d2h_bytes = 0
+        _barrier(dist_on)
+        comp = torch.cuda.current_stream()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        for _ in range(steps):
+            run.run(lambda c: ins[c])
+        b.record(comp)
+        torch.cuda.synchronize()
+        ms = _max_over_ranks(a.elapsed_time(b) / steps, dist_on, device)
+        import paged_kv_chunk_query_b200 as pk
+        status = pk.get_device_status(run.stage)
+        h2d, d2h = run.h2d_bytes / steps, run.d2h_bytes / steps
+    finally:
+        run.close()
+        del ins
+        torch.cuda.empty_cache()
+    return {"workload": w.name, "context": w.context, "ms_per_step": ms,
+            "ms_per_chunk": ms / w.num_chunks, "tokens_per_s": w.context / (ms / 1e3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "h2d_gbs": h2d / (ms / 1e3) / 1e9, "d2h_gbs": d2h / (ms / 1e3) / 1e9,
+            "device_status": status}
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(w, rows, seed_chunk=None):
     """Bounded sample of the same workload for the CPU oracle: the first `rows`
@@ -408,6 +445,8 @@ def main():
     ap.add_argument("--no-sparse", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-offload", action="store_true")
+    ap.add_argument("--offload-workload", default="qwen1m_topk_offload")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0: auto)")
     a = ap.parse_args()
 
@@ -515,6 +554,18 @@ def main():
         del sp
         torch.cuda.empty_cache()
 
+    offload_obj = None
+    if not a.no_offload:
+        offload_obj = offload_run(synth.WORKLOADS[a.offload_workload], max(1, min(a.steps, 2)),
+                                  device, dist_on)
+        if sparse_obj and offload_obj:
+            # per-chunk time against the device-resident Top-K run of the same shape
+            per_chunk_dev = sparse_obj["ms_per_step"] / synth.WORKLOADS[ws_name].num_chunks
+            offload_obj["ms_per_chunk_device_resident"] = per_chunk_dev
+            offload_obj["overhead_vs_device_resident"] = (
+                offload_obj["ms_per_chunk"] / per_chunk_dev - 1.0)
+        offload_obj["tokens_per_s"] *= world
+
     e2e = None
     if not a.no_e2e:
         ms_e, h2d, d2h = e2e_dense(w, max(1, min(a.steps, 2)), device)
@@ -547,6 +598,7 @@ def main():
         "kernels": kernels,
         "roofline": roof,
         "sparse": sparse_obj,
+        "offload": offload_obj,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": w.num_chunks * 5 * a.steps

@@ -54,6 +54,7 @@ struct FwdCfg {
   static constexpr int kSmem = kTileBytes * (1 + kNK + kNV) + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
+  static constexpr uint32_t kColQ = 384;  // Q as a bf16 A operand (D/2 columns)
 };
 
 template <int D>
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sK = sQ + Cfg::kTileBytes;
   uint8_t* sV = sK + Cfg::kNK * Cfg::kTileBytes;
 
-  __shared__ uint64_t bar_q, bar_drain, bar_o, bar_fin;
+  __shared__ uint64_t bar_q, bar_qt, bar_drain, bar_o, bar_fin;
   __shared__ uint64_t bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV], bar_ve[Cfg::kNV];
   __shared__ uint64_t bar_s[2], bar_p[2];
   __shared__ uint32_t tmem_base_sh;
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(192, 1)
     abort_sh = 0;
     k_issued_sh = v_issued_sh = k_used_sh = v_used_sh = 0;
     mbar_init(&bar_q, 1);
+    mbar_init(&bar_qt, 4);
     mbar_init(&bar_drain, 1);
     mbar_init(&bar_o, 1);
     mbar_init(&bar_fin, 1);
@@ -156,9 +158,9 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       int k_used = 0, v_used = 0;
-      bool ok = mbar_wait(&bar_q, 0, abort_flag);
+      bool ok = mbar_wait(&bar_qt, 0, abort_flag);  // Q copied into TMEM
       for (int j = 0; ok && j <= T; ++j) {
         if (j < T) {
           const int ks = j % Cfg::kNK;
@@ -170,8 +172,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
-            umma_ss(sd, sw128_desc(q_addr + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
-                    idesc_s, kk > 0);
+            umma_ts(sd, tmem + Cfg::kColQ + kk * 8, sw128_desc(kb + off, 16, 1024), idesc_s,
+                    kk > 0);
           }
           umma_commit(&bar_ke[ks]);
           umma_commit(&bar_s[j & 1]);
@@ -210,8 +212,30 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int n_past_keys = sch.n_past_pages * p.P;
     float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
+    // Q row r into TMEM (packed bf16 pairs, A operand of S = Q K^T): the S
+    // UMMAs then read only K from shared memory
+    bool ok = warp_wait(&bar_q, 0, abort_flag);
+    if (ok) {
+#pragma unroll
+      for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sQ + hf * kTile * 128 +
+                                                          sw128_offset(r, ch * 8));
+          qv[4 * ch] = v.x;
+          qv[4 * ch + 1] = v.y;
+          qv[4 * ch + 2] = v.z;
+          qv[4 * ch + 3] = v.w;
+        }
+        tmem_st32(tmem + lane_off + Cfg::kColQ + hf * 32, qv);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_qt);
+    }
+    for (int j = 0; ok && j < T; ++j) {
       const int b = j & 1;
       if (!(ok = warp_wait(&bar_s[b], (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
