@@ -192,7 +192,7 @@ oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk
  * OOMB_TOPK_STATIC_SCRATCH_BYTES inside the library, held on every GPU that
  * loads it until the process exits.  Returns OOMB_ERR_UNSUPPORTED when
  * oomb_page_topk_workspace_size() of the call exceeds that size (e.g. with
- * Hkv = 4 and d = 128, n_past up to 28,672 pages fits).  It allocates nothing.
+ * Hkv = 4 and d = 128, n_past up to 24,576 pages fits).  It allocates nothing.
  * The first call on a device looks up the array's device address (with that
  * device current); make that first call before any stream capture.  All calls
  * share the one array: calls that overlap on the GPU (different streams) race
@@ -225,15 +225,22 @@ oomb_status oomb_page_prefetch(const oomb_pool* src_pool, oomb_pool* dst_pool,
 
 /* oomb_grad_writeback: adds the device pool's gradient blocks h_src_blocks
  * into the pinned host pool's gradient blocks h_dst_blocks (same order), then
- * zero-fills the device blocks.  The blocks are copied device -> host into a
- * pinned staging area owned by the device pool, and a host function enqueued
- * on `stream` adds them with up to 16 CPU threads; later work on `stream` is
- * ordered after the add.  Calls for one device pool must be ordered (same
- * stream), since they share the staging area.  Destination blocks should be
- * distinct within one call. */
+ * zero-fills the device blocks.  On `stream` the blocks are copied device ->
+ * host into one of two pinned staging slots owned by the device pool (one
+ * cudaMemcpyAsync per run of consecutive source blocks) and the device blocks
+ * are zero-filled; a library worker thread then adds the slot into the host
+ * pool with up to 16 CPU threads, in submission order, without holding up the
+ * stream.  The call itself blocks only while both slots are still being
+ * added (OOMB_ERR_TIMEOUT after 120 s).  Destination blocks must be distinct
+ * within one call.  The host gradients include a call's blocks once
+ * oomb_grad_writeback_sync() has returned OOMB_OK. */
 oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* host_pool,
                                 const int32_t* h_src_blocks, const int32_t* h_dst_blocks,
                                 int32_t n_blocks, void* stream);
+/* Waits until every gradient addition queued by oomb_grad_writeback for this
+ * device pool has been applied to the host pool (OOMB_ERR_TIMEOUT after
+ * timeout_us microseconds). */
+oomb_status oomb_grad_writeback_sync(oomb_pool* device_pool, int64_t timeout_us);
 
 /* ---------------------------------------------------------------- status
  * Waits for a cudaEvent_t (given as void*) by polling, for at most timeout_us

@@ -33,7 +33,7 @@ EXPORTS = (
     "oomb_chunk_attn_fwd", "oomb_chunk_attn_bwd", "oomb_chunk_attn_bwd_step",
     "oomb_page_topk_workspace_size", "oomb_page_topk", "oomb_page_prefetch",
     "oomb_grad_writeback", "oomb_wait", "oomb_get_device_status", "oomb_status_string",
-    "oomb_version", "oomb_page_topk_static",
+    "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
 )
 
 
@@ -88,6 +88,7 @@ def load() -> ctypes.CDLL:
         "oomb_page_topk_static": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp],
         "oomb_page_prefetch": [vp, vp, vp, vp, i32, vp, vp],
         "oomb_grad_writeback": [vp, vp, vp, vp, i32, vp],
+        "oomb_grad_writeback_sync": [vp, ctypes.c_int64],
         "oomb_wait": [vp, ctypes.c_int64],
         "oomb_get_device_status": [vp, ctypes.POINTER(ctypes.c_uint32)],
     }
@@ -332,6 +333,10 @@ def grad_writeback(device_pool, host_pool, src_blocks, dst_blocks, stream=None):
     d, dp = _host_i32(dst_blocks)
     _check(load().oomb_grad_writeback(device_pool, host_pool, sp, dp, s.numel(),
                                       _stream(stream)), "oomb_grad_writeback")
+
+
+def grad_writeback_sync(device_pool, timeout_us: int = 120_000_000):
+    _check(load().oomb_grad_writeback_sync(device_pool, timeout_us), "oomb_grad_writeback_sync")
 
 
 def wait(event, timeout_us: int):

@@ -14,6 +14,8 @@
 #define OOMB_DEV_WAIT_LIMIT 2u
 #define OOMB_DEV_BAD_COUNT 4u
 
+struct oomb_wb_engine;  // gradient write-back worker (offload.cu)
+
 struct oomb_pool {
   oomb_pool_desc desc{};
   void* kv = nullptr;          // bf16 [pages][Hkv][2][P][d]
@@ -23,9 +25,8 @@ struct oomb_pool {
   std::vector<int32_t> free_stack;  // top = back()
   std::vector<uint8_t> used;
   std::mutex mu;
-  // pinned staging for gradient write-back (device pools), grown on demand
-  float* wb_stage = nullptr;
-  size_t wb_stage_bytes = 0;
+  // gradient write-back engine (device pools), created on first use
+  oomb_wb_engine* wb = nullptr;
 
   size_t block_elems() const {  // K+V of one (page, head)
     return static_cast<size_t>(2) * desc.page_size * desc.head_dim;
@@ -70,6 +71,8 @@ struct DeviceGuard {
 struct AttnShape {
   int C, Hq, Hkv, G, D, P, n_qtiles, n_cur_pages;
 };
+void destroy_wb_engine(oomb_pool* pool);  // drains and joins the worker
+
 oomb_status validate_attn(const oomb_pool* pool, const oomb_attn_args* a, bool backward,
                           AttnShape* s);
 

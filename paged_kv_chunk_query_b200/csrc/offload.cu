@@ -9,10 +9,15 @@
 // A block is the K and V of one (page, KV head): 2 * P * d values, contiguous
 // in both pools.  Copies are issued as one cudaMemcpyAsync per run of blocks
 // that are consecutive in both pools.  Gradient write-back copies the device
-// blocks' fp32 gradients to a pinned staging area, then a host function
-// enqueued on the same stream adds them into the host pool with several CPU
-// threads, and the device blocks are zero-filled for their next use.
+// blocks' fp32 gradients to a pinned staging slot (one copy per run of
+// consecutive source blocks), zero-fills the device blocks for their next
+// use, and hands the slot to a library worker thread that adds it into the
+// host pool with several CPU threads once the copy has landed.
 #include <algorithm>
+#include <chrono>
+#include <condition_variable>
+#include <deque>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -44,35 +49,111 @@ void for_each_run(const int32_t* src, const int32_t* dst, int n, F f) {
   }
 }
 
-struct AddJob {
-  float* host_grad;     // host pool gradient base
-  const float* stage;   // pinned staging area, blocks in list order
-  std::vector<int32_t> dst;
-  size_t block_floats;
-  int threads;
-};
-
-void CUDART_CB add_into_host(void* arg) {
-  AddJob* job = static_cast<AddJob*>(arg);
-  const size_t n = job->dst.size();
-  const int T = std::max(1, std::min<int>(job->threads, static_cast<int>(n)));
-  auto work = [job, n, T](int t) {
-    for (size_t b = t; b < n; b += T) {
-      float* out = job->host_grad + static_cast<size_t>(job->dst[b]) * job->block_floats;
-      const float* in = job->stage + b * job->block_floats;
-      for (size_t e = 0; e < job->block_floats; ++e) out[e] += in[e];
-    }
-  };
-  std::vector<std::thread> pool;
-  for (int t = 1; t < T; ++t) pool.emplace_back(work, t);
-  work(0);
-  for (auto& th : pool) th.join();
-  delete job;
-}
-
 int host_threads() {
   const unsigned hc = std::thread::hardware_concurrency();
   return static_cast<int>(std::max(1u, std::min(hc, 16u)));
+}
+
+}  // namespace
+
+// Gradient write-back engine of a device pool: two pinned staging slots used
+// in turn, and one worker thread that, job by job in submission order, waits
+// for a slot's device->host copy to finish and adds the slot into the host
+// pool with several CPU threads.  The worker never calls back into a stream,
+// so the copy stream is not held up by the additions.
+struct oomb_wb_engine {
+  struct Job {
+    int slot;
+    float* host_grad;
+    std::vector<int32_t> dst;
+    size_t block_floats;
+  };
+  std::mutex mu;
+  std::condition_variable cv;
+  std::deque<Job> jobs;
+  bool stop = false;
+  int pending = 0;              // jobs submitted and not yet added
+  float* slot_ptr[2] = {nullptr, nullptr};
+  size_t slot_bytes[2] = {0, 0};
+  bool slot_busy[2] = {false, false};
+  cudaEvent_t slot_ev[2] = {nullptr, nullptr};
+  int next_slot = 0;
+  int device = 0;
+  std::thread worker;
+
+  void run() {
+    cudaSetDevice(device);
+    while (true) {
+      Job job;
+      {
+        std::unique_lock<std::mutex> lk(mu);
+        cv.wait(lk, [&] { return stop || !jobs.empty(); });
+        if (jobs.empty()) return;
+        job = std::move(jobs.front());
+        jobs.pop_front();
+      }
+      cudaEventSynchronize(slot_ev[job.slot]);
+      const float* stage = slot_ptr[job.slot];
+      const size_t n = job.dst.size();
+      const int T = std::max(1, std::min<int>(host_threads(), static_cast<int>(n)));
+      auto work = [&](int t) {
+        for (size_t b = t; b < n; b += T) {
+          float* out = job.host_grad + static_cast<size_t>(job.dst[b]) * job.block_floats;
+          const float* in = stage + b * job.block_floats;
+          for (size_t e = 0; e < job.block_floats; ++e) out[e] += in[e];
+        }
+      };
+      std::vector<std::thread> pool;
+      for (int t = 1; t < T; ++t) pool.emplace_back(work, t);
+      work(0);
+      for (auto& th : pool) th.join();
+      {
+        std::lock_guard<std::mutex> lk(mu);
+        slot_busy[job.slot] = false;
+        --pending;
+      }
+      cv.notify_all();
+    }
+  }
+};
+
+namespace oomb {
+
+void destroy_wb_engine(oomb_pool* pool) {
+  oomb_wb_engine* e = pool->wb;
+  if (!e) return;
+  {
+    std::lock_guard<std::mutex> lk(e->mu);
+    e->stop = true;
+  }
+  e->cv.notify_all();
+  if (e->worker.joinable()) e->worker.join();
+  for (int i = 0; i < 2; ++i) {
+    if (e->slot_ptr[i]) cudaFreeHost(e->slot_ptr[i]);
+    if (e->slot_ev[i]) cudaEventDestroy(e->slot_ev[i]);
+  }
+  delete e;
+  pool->wb = nullptr;
+}
+
+}  // namespace oomb
+
+namespace {
+
+oomb_wb_engine* wb_engine(oomb_pool* pool) {
+  if (!pool->wb) {
+    oomb_wb_engine* e = new oomb_wb_engine();
+    e->device = pool->desc.device;
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&e->slot_ev[i], cudaEventDisableTiming) != cudaSuccess) {
+        for (int k = 0; k < i; ++k) cudaEventDestroy(e->slot_ev[k]);
+        delete e;
+        return nullptr;
+      }
+    e->worker = std::thread([e] { e->run(); });
+    pool->wb = e;
+  }
+  return pool->wb;
 }
 
 }  // namespace
@@ -129,23 +210,30 @@ extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* ho
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bfloats = device_pool->block_elems();
   const size_t need = static_cast<size_t>(n_blocks) * bfloats * 4;
+  oomb_wb_engine* e = wb_engine(device_pool);
+  if (!e) return OOMB_ERR_CUDA;
+  int slot;
   {
-    std::lock_guard<std::mutex> lk(device_pool->mu);
-    if (device_pool->wb_stage_bytes < need) {
-      // the staging area may still be read by an earlier add on this stream
-      if (cudaStreamSynchronize(s) != cudaSuccess) return OOMB_ERR_CUDA;
-      if (device_pool->wb_stage) cudaFreeHost(device_pool->wb_stage);
-      device_pool->wb_stage = nullptr;
-      device_pool->wb_stage_bytes = 0;
-      if (cudaHostAlloc(reinterpret_cast<void**>(&device_pool->wb_stage), need,
+    // take the next staging slot once the worker has finished adding from it
+    std::unique_lock<std::mutex> lk(e->mu);
+    slot = e->next_slot;
+    if (!e->cv.wait_for(lk, std::chrono::seconds(120), [&] { return !e->slot_busy[slot]; }))
+      return OOMB_ERR_TIMEOUT;
+    e->next_slot ^= 1;
+    if (e->slot_bytes[slot] < need) {
+      if (e->slot_ptr[slot]) cudaFreeHost(e->slot_ptr[slot]);
+      e->slot_ptr[slot] = nullptr;
+      e->slot_bytes[slot] = 0;
+      if (cudaHostAlloc(reinterpret_cast<void**>(&e->slot_ptr[slot]), need,
                         cudaHostAllocPortable) != cudaSuccess)
         return OOMB_ERR_CUDA;
-      device_pool->wb_stage_bytes = need;
+      e->slot_bytes[slot] = need;
     }
+    e->slot_busy[slot] = true;
   }
-  float* stage = device_pool->wb_stage;
+  float* stage = e->slot_ptr[slot];
   bool ok = true;
-  // device -> pinned staging, in list order (runs of consecutive source blocks)
+  // device -> pinned slot in list order, one copy per run of consecutive source blocks
   int done = 0;
   for (int i = 0; i < n_blocks && ok;) {
     int j = i + 1;
@@ -156,14 +244,7 @@ extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* ho
     done += j - i;
     i = j;
   }
-  if (!ok) return OOMB_ERR_CUDA;
-  AddJob* job = new AddJob{host_pool->grad, stage,
-                           std::vector<int32_t>(h_dst_blocks, h_dst_blocks + n_blocks), bfloats,
-                           host_threads()};
-  if (cudaLaunchHostFunc(s, add_into_host, job) != cudaSuccess) {
-    delete job;
-    return OOMB_ERR_CUDA;
-  }
+  ok = ok && cudaEventRecord(e->slot_ev[slot], s) == cudaSuccess;
   // the device blocks start from zero for their next contributions
   for (int i = 0; i < n_blocks && ok;) {
     int j = i + 1;
@@ -172,5 +253,27 @@ extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* ho
                          (j - i) * bfloats * 4, s) == cudaSuccess;
     i = j;
   }
+  {
+    std::lock_guard<std::mutex> lk(e->mu);
+    if (!ok) {
+      e->slot_busy[slot] = false;
+    } else {
+      e->jobs.push_back(oomb_wb_engine::Job{
+          slot, host_pool->grad, std::vector<int32_t>(h_dst_blocks, h_dst_blocks + n_blocks),
+          bfloats});
+      ++e->pending;
+    }
+  }
+  e->cv.notify_all();
   return ok ? OOMB_OK : OOMB_ERR_CUDA;
+}
+
+extern "C" oomb_status oomb_grad_writeback_sync(oomb_pool* device_pool, int64_t timeout_us) {
+  if (!device_pool) return OOMB_ERR_INVALID_ARG;
+  oomb_wb_engine* e = device_pool->wb;
+  if (!e) return OOMB_OK;
+  std::unique_lock<std::mutex> lk(e->mu);
+  const bool done = e->cv.wait_for(lk, std::chrono::microseconds(timeout_us),
+                                   [&] { return e->pending == 0; });
+  return done ? OOMB_OK : OOMB_ERR_TIMEOUT;
 }

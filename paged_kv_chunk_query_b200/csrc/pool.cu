@@ -42,12 +42,10 @@ void release_buffers(oomb_pool* p) {
     free_one(p->summary);
   }
   if (p->d_status) cudaFree(p->d_status);
-  if (p->wb_stage) cudaFreeHost(p->wb_stage);
   p->kv = nullptr;
   p->grad = nullptr;
   p->summary = nullptr;
   p->d_status = nullptr;
-  p->wb_stage = nullptr;
 }
 
 }  // namespace
@@ -135,6 +133,7 @@ oomb_status oomb_pool_destroy(oomb_pool* pool) {
   {
     oomb::DeviceGuard g(pool->desc.device);
     if (pool->desc.location != OOMB_LOC_HOST) cudaDeviceSynchronize();
+    oomb::destroy_wb_engine(pool);  // finishes queued gradient additions first
     release_buffers(pool);
   }
   delete pool;

@@ -10,8 +10,8 @@
 // ties going to the lower logical id; pages [n_past - R, n_past) are always
 // kept; the output lists ascending logical ids.
 //
-// Kernel 1 (qmean_partial): grid (64 slices, Hkv); each CTA streams a slice of
-//   the chunk's rows with 16-byte loads, 4 in flight per thread, and writes one
+// Kernel 1 (qmean_partial): grid (128 slices, Hkv); each CTA streams a slice of
+//   the chunk's rows with 16-byte loads, 8 in flight per thread, and writes one
 //   fp32 partial sum per d.
 // Kernel 2 (page_score): grid (pages / 64, Hkv); each CTA reduces the partials
 //   in a fixed order into q_bar, then each warp scores 8 pages (float4 loads of
@@ -28,8 +28,8 @@
 
 namespace {
 
-constexpr int kSplits = 64;          // query-mean slices per group
-constexpr int kMeanThreads = 512;
+constexpr int kSplits = 128;         // query-mean slices per group (~3.5 CTAs per SM at Hkv 4)
+constexpr int kMeanThreads = 256;
 constexpr int kScoreThreads = 256;   // 8 warps x 8 pages per CTA
 constexpr int kPagesPerScoreCta = 64;
 constexpr int kSelectThreads = 1024;
@@ -37,13 +37,15 @@ constexpr int kSelectThreads = 1024;
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // ---------------------------------------------------------------- query mean
-// grid (kSplits, Hkv): CTA (s, g) sums rows (token, head in g) of token slice s.
+// grid (kSplits, Hkv): CTA (s, g) sums rows (token, head in g) of token slice
+// s.  Each thread keeps 8 independent 16-byte loads in flight (about 32 KiB
+// per CTA), enough with 3-4 CTAs per SM to stream Q at HBM speed.
 template <int D>
 __global__ void __launch_bounds__(kMeanThreads) qmean_partial_kernel(
     const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, int C, int Hq, int G) {
   constexpr int VPR = D / 8;               // 16-byte vectors per row
   constexpr int RG = kMeanThreads / VPR;   // rows per pass
-  constexpr int U = 4;                     // loads in flight per thread
+  constexpr int U = 8;                     // loads in flight per thread
   __shared__ float red[RG][D];
   const int split = blockIdx.x, g = blockIdx.y, t = threadIdx.x;
   const int vec = t % VPR, rg = t / VPR;
@@ -68,9 +70,9 @@ __global__ void __launch_bounds__(kMeanThreads) qmean_partial_kernel(
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
+      const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(b[e]);
+      for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(bv[e]);
     }
   }
 #pragma unroll

@@ -72,7 +72,7 @@ class OffloadRun:
         self.selections = []
 
     def close(self):
-        torch.cuda.synchronize(self.dev)
+        self.sync()
         L.pool_destroy(self.stage)
         if self.own_host:
             L.pool_destroy(self.host)
@@ -111,11 +111,15 @@ class OffloadRun:
         src, dst = [], []
         past = self.past_host[b]
         past.zero_()
+        # slot-major order: staging blocks (slot i, head g) are consecutive, so the
+        # gradient write-back of these blocks is one large device->host copy
+        for i in range(max(len(x) for x in sel)):
+            for g in range(Hkv):
+                if i < len(sel[g]):
+                    src.append(self.table[sel[g][i]] * Hkv + g)
+                    dst.append(self.stage_pages[b * self.half + i] * Hkv + g)
+                    past[g, i] = self.stage_pages[b * self.half + i]
         for g in range(Hkv):
-            for i, lp in enumerate(sel[g]):
-                src.append(self.table[lp] * Hkv + g)
-                dst.append(self.stage_pages[b * self.half + i] * Hkv + g)
-                past[g, i] = self.stage_pages[b * self.half + i]
             self.cnt_host[b][g] = len(sel[g])
         ev = torch.cuda.Event()
         with torch.cuda.stream(self.copy):
@@ -198,3 +202,8 @@ class OffloadRun:
             self.copy.wait_event(prev[0])
             self._writeback(N - 1, prev[1])
         comp.wait_stream(self.copy)
+
+    def sync(self):
+        """Waits for the device and for every queued host gradient addition."""
+        torch.cuda.synchronize(self.dev)
+        L.grad_writeback_sync(self.stage)

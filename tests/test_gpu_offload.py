@@ -80,6 +80,7 @@ def test_grad_writeback_adds_and_zeroes():
         with torch.cuda.stream(stream):
             pk.grad_writeback(a, h, src, dst, stream=stream)
         stream.synchronize()
+        pk.grad_writeback_sync(a)
         bh = before_h.view(-1, 2 * P * d)
         ba = before_a.view(-1, 2 * P * d)
         want = bh.clone()
@@ -108,7 +109,7 @@ def test_offloaded_topk_run_matches_device_resident_run():
     run = OffloadRun(w, dev)
     try:
         run.run(lambda c: ins[c], lambda c: outs[c])
-        torch.cuda.synchronize()
+        run.sync()
         assert pk.get_device_status(run.stage) == 0
         sels = run.selections
         _, gh, _ = pk.pool_views(run.host)
