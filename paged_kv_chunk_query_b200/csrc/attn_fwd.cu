@@ -5,17 +5,20 @@
 // query rows of one head and walks the KV tiles of its group: the listed past
 // pages (all visible) and then the chunk's own pages (causal).
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Reads S from
-//              TMEM, keeps the running max / sum, writes P (bf16) back into the
-//              same TMEM columns, rescales O when the max grows, and finally
-//              normalises O and writes O and the LSE.
-//   warp 4     TMA producer: Q once, then K and V tiles page by page through
-//              a 4-D tensor map over the pool (page id = outermost coordinate).
-//   warp 5     UMMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
-//              buffers, O += P_j V_j with P read from TMEM (A operand) and V
-//              from shared memory (MN-major B operand).
-// TMEM: S0 [0,128), S1 [128,256), O [256, 256+D).
+// Warp roles (224 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  First copies
+//              its Q row from shared memory into TMEM (A operand of QK^T);
+//              then per tile reads S from TMEM, keeps the running max / sum,
+//              writes P (bf16) back into the same TMEM columns, rescales O
+//              when the max grows, and finally normalises O and writes O and
+//              the LSE.
+//   warp 4     TMA producer of Q and the K tiles, warp 6 of the V tiles, page
+//              by page through a 4-D tensor map over the pool (page id =
+//              outermost coordinate).
+//   warp 5     UMMA issuer (one thread): S_j = Q K_j^T (Q from TMEM) into one of
+//              two TMEM S buffers, O += P_j V_j with P read from TMEM (A
+//              operand) and V from shared memory (MN-major B operand).
+// TMEM: S0 [0,128), S1 [128,256), O [256, 256+D), Q [384, 384+D/2).
 //
 // Online softmax in base 2: s2 = S * scale * log2(e).  The running maximum is
 // only moved when a tile's maximum exceeds it by more than 8 (a factor 256),
@@ -50,7 +53,7 @@ struct FwdCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTile * D * 2;  // Q, K or V tile
   static constexpr int kNK = 3;
-  static constexpr int kNV = 2;
+  static constexpr int kNV = 3;
   static constexpr int kSmem = kTileBytes * (1 + kNK + kNV) + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
@@ -58,7 +61,7 @@ struct FwdCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     attn_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap qmap,
                     const __grid_constant__ CUtensorMap kvmap) {
   using Cfg = FwdCfg<D>;
@@ -114,44 +117,44 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------ producers
+    // warp 4 loads Q and the K tiles, warp 6 the V tiles, so a K load never
+    // queues behind a V slot that frees only after a late PV.
     if (lane == 0) {
-      prefetch_tensormap(&qmap);
+      const bool is_k = warp == 4;
+      if (is_k) {
+        prefetch_tensormap(&qmap);
+        mbar_arrive_expect_tx(&bar_q, Cfg::kTileBytes);
+        for (int hf = 0; hf < Cfg::kHalves; ++hf)
+          tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
+      }
       prefetch_tensormap(&kvmap);
       const int32_t* past_list = p.past_pages + static_cast<size_t>(g) * p.max_past;
       const int per = kTile / p.P;
-      mbar_arrive_expect_tx(&bar_q, Cfg::kTileBytes);
-      for (int hf = 0; hf < Cfg::kHalves; ++hf)
-        tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
-      int k_issued = 0, v_issued = 0;
+      const int nst = is_k ? Cfg::kNK : Cfg::kNV;
+      uint64_t* full = is_k ? bar_kf : bar_vf;
+      uint64_t* empty = is_k ? bar_ke : bar_ve;
+      uint8_t* base = is_k ? sK : sV;
+      int issued = 0;
       for (int j = 0; j < T; ++j) {
         int pg[8];
         for (int s = 0; s < per; ++s)
           pg[s] = tile_page(j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
-                            p.num_pool_pages, p.status);
-        const int ks = j % Cfg::kNK;
-        if (!mbar_wait(&bar_ke[ks], ((j / Cfg::kNK) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bar_kf[ks], Cfg::kTileBytes);
-        uint8_t* kdst = sK + ks * Cfg::kTileBytes;
+                            p.num_pool_pages, is_k ? p.status : nullptr);
+        const int st = j % nst;
+        if (!mbar_wait(&empty[st], ((j / nst) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[st], Cfg::kTileBytes);
+        uint8_t* dst = base + st * Cfg::kTileBytes;
         for (int s = 0; s < per; ++s)
           for (int hf = 0; hf < Cfg::kHalves; ++hf)
-            tma_load_4d(kdst + hf * kTile * 128 + s * p.P * 128, &kvmap, &bar_kf[ks], hf * 64, 0,
-                        2 * g, pg[s]);
-        ++k_issued;
-        const int vs = j % Cfg::kNV;
-        if (!mbar_wait(&bar_ve[vs], ((j / Cfg::kNV) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bar_vf[vs], Cfg::kTileBytes);
-        uint8_t* vdst = sV + vs * Cfg::kTileBytes;
-        for (int s = 0; s < per; ++s)
-          for (int hf = 0; hf < Cfg::kHalves; ++hf)
-            tma_load_4d(vdst + hf * kTile * 128 + s * p.P * 128, &kvmap, &bar_vf[vs], hf * 64, 0,
-                        2 * g + 1, pg[s]);
-        ++v_issued;
+            tma_load_4d(dst + hf * kTile * 128 + s * p.P * 128, &kvmap, &full[st], hf * 64, 0,
+                        2 * g + (is_k ? 0 : 1), pg[s]);
+        ++issued;
       }
       if (*abort_flag) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
-      k_issued_sh = k_issued;
-      v_issued_sh = v_issued;
+      if (is_k) k_issued_sh = issued;
+      else v_issued_sh = issued;
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ UMMA issuer
@@ -397,7 +400,7 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.num_pool_pages = pool->desc.num_pages;
   p.scale_log2 = a->softmax_scale * kLog2e;
   dim3 grid(s.n_qtiles, s.Hq);
-  attn_fwd_kernel<D><<<grid, 192, Cfg::kSmem, stream>>>(p, qmap, kvmap);
+  attn_fwd_kernel<D><<<grid, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
   return check_launch();
 }
 

@@ -59,7 +59,7 @@ __device__ __forceinline__ int tile_page(int j, int slot, const KvSchedule& s,
     }
   }
   if (listed && (id < 0 || id >= oob)) {
-    atomicOr(status, OOMB_DEV_BAD_PAGE);
+    if (status) atomicOr(status, OOMB_DEV_BAD_PAGE);
     id = oob;
   }
   return id;
