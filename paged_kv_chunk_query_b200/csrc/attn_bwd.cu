@@ -396,15 +396,17 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ------------------------------------------------------------------ dQ
-// One CTA per (128-row query tile, head).  Two slots walk the KV tiles in
-// turn (slot 0 the even tiles, slot 1 the odd ones), so one slot's softmax
-// overlaps the other slot's UMMAs.  Warps 0-3 serve slot 0 and warps 4-7
-// slot 1 (thread = query row = TMEM lane, all 128 key columns); warp 8 loads
-// (TMA), warp 9 issues UMMA in the order
-//   S(0) S(1) dP(0) | dQ(j) dP(j+1) S(j+2) for j = 0, 1, ...
-// TMEM: S of slot s [128s, 128s+128) (its dS, bf16, overwrites [128s, +64)
-// once S is in registers); dP [256,384) shared by the slots in turn; dQ
-// [384, 384+D).
+// One CTA per (128-row query tile, head).  Q and dO are copied into TMEM once
+// and serve as the A operands of S = Q K_j^T and dP = dO V_j^T, so those
+// UMMAs read only K_j or V_j from shared memory.  S_{j+1} is computed while
+// the compute warps work on tile j; dS_j (bf16) goes into the dP columns the
+// warps have already read and feeds dQ += dS_j K_j.
+// Warps 0-7 compute (warps w and w+4 share rows 32(w%4)..+31; w < 4 takes key
+// columns 0-63 and copies Q into TMEM, w >= 4 the other half and dO), warp 8
+// loads Q, dO and the K tiles, warp 10 the V tiles, warp 9 issues UMMA:
+//   S(0) dP(0) | S(j+1) dQ(j) dP(j+1) for j = 0, 1, ...
+// TMEM: S [0,128), dP [128,256) (dS of key half k: [128+64k, +32)), dQ
+// [256, 256+D), Q [384, 384+D/2), dO [448, 448+D/2).
 template <int D>
 struct QCfg {
   static constexpr int kHalves = D / 64;
@@ -412,11 +414,11 @@ struct QCfg {
   static constexpr int kNK = 3, kNV = 2;
   static constexpr int kSmem = kTileBytes * (2 + kNK + kNV) + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColDP = 256, kColDQ = 384;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColQ = 384, kColDO = 448;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap domap,
                   const __grid_constant__ CUtensorMap kvmap) {
@@ -429,9 +431,9 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sK = sDO + Cfg::kTileBytes;
   uint8_t* sV = sK + Cfg::kNK * Cfg::kTileBytes;
 
-  __shared__ uint64_t bar_q, bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV],
+  __shared__ uint64_t bar_q, bar_qt, bar_kf[Cfg::kNK], bar_ke[Cfg::kNK], bar_vf[Cfg::kNV],
       bar_ve[Cfg::kNV];
-  __shared__ uint64_t bar_s[2], bar_dp[2], bar_ds[2], bar_fin, bar_drain;
+  __shared__ uint64_t bar_s, bar_sl, bar_dp, bar_ds, bar_fin, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh, k_issued_sh, v_issued_sh, k_used_sh, v_used_sh;
 
@@ -445,6 +447,7 @@ __global__ void __launch_bounds__(320, 1)
     abort_sh = 0;
     k_issued_sh = v_issued_sh = k_used_sh = v_used_sh = 0;
     mbar_init(&bar_q, 1);
+    mbar_init(&bar_qt, 8);
     for (int i = 0; i < Cfg::kNK; ++i) {
       mbar_init(&bar_kf[i], 1);
       mbar_init(&bar_ke[i], 1);
@@ -453,11 +456,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bar_vf[i], 1);
       mbar_init(&bar_ve[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_dp[i], 1);
-      mbar_init(&bar_ds[i], 4);
-    }
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_sl, 8);
+    mbar_init(&bar_dp, 1);
+    mbar_init(&bar_ds, 8);
     mbar_init(&bar_fin, 1);
     mbar_init(&bar_drain, 1);
     fence_mbar_init();
@@ -472,54 +474,52 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
 
-  if (warp == 8) {
+  if (warp == 8 || warp == 10) {
     if (lane == 0) {
-      prefetch_tensormap(&qmap);
-      prefetch_tensormap(&domap);
+      const bool is_k = warp == 8;
+      if (is_k) {
+        prefetch_tensormap(&qmap);
+        prefetch_tensormap(&domap);
+        mbar_arrive_expect_tx(&bar_q, 2 * Cfg::kTileBytes);
+        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+          tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
+          tma_load_3d(sDO + hf * kTile * 128, &domap, &bar_q, hf * 64, h, qt * kTile);
+        }
+      }
       prefetch_tensormap(&kvmap);
       const int32_t* past_list =
           p.past_pages ? p.past_pages + static_cast<size_t>(g) * p.max_past : nullptr;
       const int per = kTile / p.P;
-      mbar_arrive_expect_tx(&bar_q, 2 * Cfg::kTileBytes);
-      for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-        tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
-        tma_load_3d(sDO + hf * kTile * 128, &domap, &bar_q, hf * 64, h, qt * kTile);
-      }
-      int k_issued = 0, v_issued = 0;
+      const int nst = is_k ? Cfg::kNK : Cfg::kNV;
+      uint64_t* full = is_k ? bar_kf : bar_vf;
+      uint64_t* empty = is_k ? bar_ke : bar_ve;
+      uint8_t* base = is_k ? sK : sV;
+      int issued = 0;
       for (int j = 0; j < T; ++j) {
         int pg[8];
         for (int s = 0; s < per; ++s)
           pg[s] = tile_page(j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
-                            p.num_pool_pages, p.status);
-        const int ks = j % Cfg::kNK;
-        if (!mbar_wait(&bar_ke[ks], ((j / Cfg::kNK) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bar_kf[ks], Cfg::kTileBytes);
+                            p.num_pool_pages, is_k ? p.status : nullptr);
+        const int st = j % nst;
+        if (!mbar_wait(&empty[st], ((j / nst) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[st], Cfg::kTileBytes);
         for (int s = 0; s < per; ++s)
           for (int hf = 0; hf < Cfg::kHalves; ++hf)
-            tma_load_4d(sK + ks * Cfg::kTileBytes + hf * kTile * 128 + s * p.P * 128, &kvmap,
-                        &bar_kf[ks], hf * 64, 0, 2 * g, pg[s]);
-        ++k_issued;
-        const int vs = j % Cfg::kNV;
-        if (!mbar_wait(&bar_ve[vs], ((j / Cfg::kNV) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bar_vf[vs], Cfg::kTileBytes);
-        for (int s = 0; s < per; ++s)
-          for (int hf = 0; hf < Cfg::kHalves; ++hf)
-            tma_load_4d(sV + vs * Cfg::kTileBytes + hf * kTile * 128 + s * p.P * 128, &kvmap,
-                        &bar_vf[vs], hf * 64, 0, 2 * g + 1, pg[s]);
-        ++v_issued;
+            tma_load_4d(base + st * Cfg::kTileBytes + hf * kTile * 128 + s * p.P * 128, &kvmap,
+                        &full[st], hf * 64, 0, 2 * g + (is_k ? 0 : 1), pg[s]);
+        ++issued;
       }
       if (*abort_flag) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
-      k_issued_sh = k_issued;
-      v_issued_sh = v_issued;
+      if (is_k) k_issued_sh = issued;
+      else v_issued_sh = issued;
     }
   } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       int k_used = 0, v_used = 0;
-      auto issue_s = [&](int j) -> bool {  // S(j) into slot j&1
+      auto issue_s = [&](int j) -> bool {  // S(j) = Q K_j^T, Q from TMEM
         const int ks = j % Cfg::kNK;
         if (!mbar_wait(&bar_kf[ks], (j / Cfg::kNK) & 1, abort_flag)) return false;
         ++k_used;
@@ -528,13 +528,13 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
-          umma_ss(tmem + (j & 1) * 128, sw128_desc(q_addr + off, 16, 1024),
-                  sw128_desc(kb + off, 16, 1024), idesc_s, kk > 0);
+          umma_ts(tmem + Cfg::kColS, tmem + Cfg::kColQ + kk * 8, sw128_desc(kb + off, 16, 1024),
+                  idesc_s, kk > 0);
         }
-        umma_commit(&bar_s[j & 1]);
+        umma_commit(&bar_s);
         return true;
       };
-      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T into the shared dP buffer
+      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T, dO from TMEM
         const int vs = j % Cfg::kNV;
         if (!mbar_wait(&bar_vf[vs], (j / Cfg::kNV) & 1, abort_flag)) return false;
         ++v_used;
@@ -543,29 +543,31 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
-          umma_ss(tmem + Cfg::kColDP, sw128_desc(do_addr + off, 16, 1024),
+          umma_ts(tmem + Cfg::kColDP, tmem + Cfg::kColDO + kk * 8,
                   sw128_desc(vb + off, 16, 1024), idesc_s, kk > 0);
         }
         umma_commit(&bar_ve[vs]);
-        umma_commit(&bar_dp[j & 1]);
+        umma_commit(&bar_dp);
         return true;
       };
-      bool ok = mbar_wait(&bar_q, 0, abort_flag);
-      ok = ok && issue_s(0) && (T < 2 || issue_s(1)) && issue_dp(0);
+      bool ok = mbar_wait(&bar_qt, 0, abort_flag);  // Q and dO are in TMEM
+      ok = ok && issue_s(0) && issue_dp(0);
       for (int j = 0; ok && j < T; ++j) {
-        // dQ += dS(j) K_j, dS(j) packed in its slot's S columns
-        if (!(ok = mbar_wait(&bar_ds[j & 1], (j >> 1) & 1, abort_flag))) break;
+        if (j + 1 < T) {
+          if (!(ok = mbar_wait(&bar_sl, j & 1, abort_flag))) break;  // S(j) in registers
+          if (!(ok = issue_s(j + 1))) break;
+        }
+        if (!(ok = mbar_wait(&bar_ds, j & 1, abort_flag))) break;
         tc_fence_after();
         const int ks = j % Cfg::kNK;
         const uint32_t kb = k_addr + ks * Cfg::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tmem + Cfg::kColDQ, tmem + (j & 1) * 128 + kk * 8,
+          umma_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + (kk / 4) * 64 + (kk % 4) * 8,
                   sw128_desc(kb + kk * 16 * 128, kTile * 128, 1024), idesc_dq,
                   (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bar_ke[ks]);
         if (j + 1 < T && !(ok = issue_dp(j + 1))) break;
-        if (j + 2 < T && !(ok = issue_s(j + 2))) break;
       }
       if (ok) umma_commit(&bar_fin);
       if (!ok) {
@@ -577,56 +579,78 @@ __global__ void __launch_bounds__(320, 1)
       k_used_sh = k_used;
       v_used_sh = v_used;
     }
-  } else {
-    const int slot = warp >> 2;
-    const int r = (warp & 3) * 32 + lane;  // query row (TMEM lane)
+  } else if (warp < 8) {
+    const int lg = warp & 3, half = warp >> 2;  // lane group, key/d column half
+    const int r = lg * 32 + lane;               // query row (TMEM lane)
     const int q_local = qt * kTile + r;
     const bool row_valid = q_local < p.C;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t col_s = slot * 128;
+    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+    const uint32_t cs = half * 64;
     const float lse2 = row_valid ? p.lse[static_cast<size_t>(h) * p.C + q_local] * kLog2e : 0.f;
     const float dl = row_valid ? p.delta[static_cast<size_t>(h) * p.C + q_local] : 0.f;
     const int n_past_keys = sch.n_past_pages * p.P;
-    bool ok = true;
-    for (int j = slot; j < T; j += 2) {
-      const int use = j >> 1;  // this slot's use count
-      if (!(ok = warp_wait(&bar_s[slot], use & 1, abort_flag))) break;
-      tc_fence_after();
-      float pr[kTile];
+    // half 0 copies its Q row, half 1 its dO row, into TMEM (packed bf16 pairs)
+    bool ok = warp_wait(&bar_q, 0, abort_flag);
+    if (ok) {
+      const uint8_t* src = half == 0 ? sQ : sDO;
+      const uint32_t col = half == 0 ? Cfg::kColQ : Cfg::kColDO;
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c)
-        tmem_ld32(tmem + lane_off + col_s + c * 32, reinterpret_cast<uint32_t*>(pr + c * 32));
-      tmem_ld_wait();
-      int lim;
-      if (j < sch.n_past_tiles) lim = n_past_keys - j * kTile;
-      else lim = min(p.C, q_local + 1) - (j - sch.n_past_tiles) * kTile;
-      if (!row_valid) lim = 0;
+      for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+        uint32_t v[32];
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) pr[c] = fast_exp2(fmaf(pr[c], p.scale_log2, -lse2));
-      if (lim < kTile) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) pr[c] = c < lim ? pr[c] : 0.f;
-      }
-      if (!(ok = warp_wait(&bar_dp[slot], use & 1, abort_flag))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t dp[32];
-        tmem_ld32(tmem + lane_off + Cfg::kColDP + c * 32, dp);
-        tmem_ld_wait();
-        uint32_t ds[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = c * 32 + 2 * e;
-          ds[e] = pack_bf16(pr[c0] * (__uint_as_float(dp[2 * e]) - dl),
-                            pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - dl));
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 x = *reinterpret_cast<const uint4*>(src + hf * kTile * 128 +
+                                                          sw128_offset(r, ch * 8));
+          v[4 * ch] = x.x;
+          v[4 * ch + 1] = x.y;
+          v[4 * ch + 2] = x.z;
+          v[4 * ch + 3] = x.w;
         }
-        tmem_st16(tmem + lane_off + col_s + c * 16, ds);
+        tmem_st32(tmem + lane_off + col + hf * 32, v);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_ds[slot]);
+      if (lane == 0) mbar_arrive(&bar_qt);
+    }
+    for (int j = 0; ok && j < T; ++j) {
+      if (!(ok = warp_wait(&bar_s, j & 1, abort_flag))) break;
+      tc_fence_after();
+      float pr[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColS + cs, reinterpret_cast<uint32_t*>(pr));
+      tmem_ld32(tmem + lane_off + Cfg::kColS + cs + 32, reinterpret_cast<uint32_t*>(pr + 32));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sl);  // the next S may overwrite these columns
+      int lim;
+      if (j < sch.n_past_tiles) lim = n_past_keys - j * kTile;
+      else lim = min(p.C, q_local + 1) - (j - sch.n_past_tiles) * kTile;
+      if (!row_valid) lim = 0;
+      lim -= static_cast<int>(cs);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) pr[c] = fast_exp2(fmaf(pr[c], p.scale_log2, -lse2));
+      if (lim < 64) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pr[c] = c < lim ? pr[c] : 0.f;
+      }
+      if (!(ok = warp_wait(&bar_dp, j & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t dp[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColDP + cs, dp);
+      tmem_ld32(tmem + lane_off + Cfg::kColDP + cs + 32, dp + 32);
+      tmem_ld_wait();
+      uint32_t ds[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        ds[e] = pack_bf16(pr[2 * e] * (__uint_as_float(dp[2 * e]) - dl),
+                          pr[2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - dl));
+      tmem_st16(tmem + lane_off + Cfg::kColDP + cs, ds);
+      tmem_st16(tmem + lane_off + Cfg::kColDP + cs + 16, ds + 16);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_ds);
     }
     if (ok) ok = warp_wait(&bar_fin, 0, abort_flag);
     if (!ok) {
@@ -634,7 +658,7 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
     } else {
       tc_fence_after();
-      const int d0 = slot * (D / 2);  // each slot writes half of the row
+      const int d0 = half * (D / 2);
       __nv_bfloat16* row = p.dq + (static_cast<size_t>(q_local) * p.Hq + h) * D + d0;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
@@ -745,7 +769,7 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
     }
     if (step < 0 || step == OOMB_BWD_DQ) {
       dim3 grid(s.n_qtiles, s.Hq);
-      bwd_dq_kernel<D><<<grid, 320, QCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
+      bwd_dq_kernel<D><<<grid, 352, QCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
       if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
     }
   }
