@@ -215,6 +215,12 @@ def _barrier(dist_on):
         torch.distributed.barrier()
 
 
+def whole_job_rate(units_per_rank, ms_max, world):
+    """Whole-job throughput of `world` replicas: every rank processes
+    `units_per_rank`, the job takes the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def _max_over_ranks(x, dist_on, device):
     if not dist_on:
         return x
@@ -504,8 +510,8 @@ def main():
     clk = clocks.stop()
     dense_status = pk.get_device_status(dense.pool)
     step_flops = dense.step_flops
-    value = step_flops * world / (ms / 1e3) / 1e12
-    tokens = w.context * world / (ms / 1e3)
+    value = whole_job_rate(step_flops, ms, world) / 1e12
+    tokens = whole_job_rate(w.context, ms, world)
     kernel_flops = {k: sum(v) for k, v in dense.flops.items()}
     dense.close()
     del dense
