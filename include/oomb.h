@@ -252,6 +252,12 @@ oomb_status oomb_wait(void* event, int64_t timeout_us);
  *   bit 0 invalid page id, bit 1 wait limit reached, bit 2 bad count. */
 oomb_status oomb_get_device_status(oomb_pool* pool, uint32_t* out_word);
 const char* oomb_status_string(oomb_status status);
+/* Self-test of the kernels' bounded waits (no counterpart in the paper): one
+ * thread waits on an mbarrier that nothing arrives at; after the wait limit
+ * (about a second) it gives up and sets bit 1 of the pool's device status
+ * word, exactly as a kernel whose arrival was lost would.  Device or
+ * pinned-host pools only. */
+oomb_status oomb_selftest_wait_limit(oomb_pool* pool, void* stream);
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t oomb_version(void);
 

@@ -34,6 +34,7 @@ EXPORTS = (
     "oomb_page_topk_workspace_size", "oomb_page_topk", "oomb_page_prefetch",
     "oomb_grad_writeback", "oomb_wait", "oomb_get_device_status", "oomb_status_string",
     "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
+    "oomb_selftest_wait_limit",
 )
 
 
@@ -91,6 +92,7 @@ def load() -> ctypes.CDLL:
         "oomb_grad_writeback_sync": [vp, ctypes.c_int64],
         "oomb_wait": [vp, ctypes.c_int64],
         "oomb_get_device_status": [vp, ctypes.POINTER(ctypes.c_uint32)],
+        "oomb_selftest_wait_limit": [vp, vp],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):  # completeness is checked by the export test
@@ -349,6 +351,10 @@ def get_device_status(pool) -> int:
     if st not in (OK, ERR_DEVICE_CHECK):
         raise OombError(st, "oomb_get_device_status")
     return w.value
+
+
+def selftest_wait_limit(pool, stream=None):
+    _check(load().oomb_selftest_wait_limit(pool, _stream(stream)), "oomb_selftest_wait_limit")
 
 
 def status_string(status: int) -> str:
