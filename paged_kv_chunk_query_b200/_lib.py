@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -318,7 +319,10 @@ def page_topk_static(pool, q, page_table, n_past, top_k, n_recent, out_logical, 
 
 
 def _host_i32(blocks):
-    t = torch.as_tensor(blocks, dtype=torch.int32).contiguous()
+    if isinstance(blocks, np.ndarray):
+        t = torch.from_numpy(np.ascontiguousarray(blocks, dtype=np.int32))
+    else:
+        t = torch.as_tensor(blocks, dtype=torch.int32).contiguous()
     return t, t.data_ptr()
 
 

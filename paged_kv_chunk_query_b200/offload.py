@@ -10,20 +10,22 @@ CUDA streams; every copy and every computation runs inside liboomb.so.
 Pools: a pinned-host pool holds every page's K/V and fp32 gradients (its page
 representatives stay on the device); a small device staging pool holds, per
 chunk, the pages Top-K kept for each KV-head group and the chunk's own pages.
-The staging pool has two halves used by alternate chunks, so chunk c+1's
-prefetch fills one half while chunk c computes on the other.
+The staging pool has three parts used by chunks in turn, so chunk c+1's
+prefetch fills one part while chunk c computes on another and chunk c-1's
+gradients drain from the third.
 
-Per chunk c (compute stream C, copy stream S; half = c % 2):
-  C: wait for prefetch(c); append K_c, V_c into the half's current pages
+Per chunk c (compute stream C, copy stream S; part = c % 3):
+  C: wait for prefetch(c); append K_c, V_c into the part's current pages
      (page summaries, zeroed gradient blocks)
   S: store those pages and summaries into the host pool
   S: Top-K for chunk c+1 against the host pool's summaries; selection -> host
-  C: forward + backward of chunk c on the staging half
+  C: forward + backward of chunk c on the staging part
   host: wait for the selection of c+1, build the block lists
-  S: write back chunk c-1's gradient deltas (D2H + host add, zeroes them),
-     then prefetch chunk c+1's selected blocks into the other half
-The prefetch of chunk c+1 and the write-back of chunk c-1 thus overlap the
-forward and backward of chunk c.
+  S: prefetch chunk c+1's selected blocks into part (c+1) % 3, then write
+     back chunk c-1's gradient deltas (D2H, zero-fill; the host add runs on
+     the library's worker thread)
+Part (c+1) % 3 was last used by chunk c-2, whose write-back (issued in
+iteration c-1, earlier on S) has drained and zeroed its gradient blocks.
 """
 from __future__ import annotations
 
@@ -39,14 +41,17 @@ class OffloadRun:
         P, Hkv, d = w.page_size, w.num_kv_heads, w.head_dim
         self.sel_max = w.top_k + w.n_recent
         self.ppc = w.pages_per_chunk
-        self.half = self.sel_max + self.ppc           # staging pages per half
+        self.parts = 3
+        self.half = self.sel_max + self.ppc           # staging pages per part
         self.host = host_pool or L.pool_create(w.num_pages, P, Hkv, d, L.LOC_PINNED_HOST, True,
                                                w.alloc_seed, device.index or 0)
         self.own_host = host_pool is None
-        self.stage = L.pool_create(2 * self.half, P, Hkv, d, L.LOC_DEVICE, True, 0,
+        self.stage = L.pool_create(self.parts * self.half, P, Hkv, d, L.LOC_DEVICE, True, 0,
                                    device.index or 0)
-        self.stage_pages = [L.pool_alloc_page(self.stage) for _ in range(2 * self.half)]
-        self.table = [L.pool_alloc_page(self.host) for _ in range(w.num_chunks * self.ppc)]
+        self.stage_pages = np.array([L.pool_alloc_page(self.stage)
+                                     for _ in range(self.parts * self.half)], dtype=np.int64)
+        self.table = np.array([L.pool_alloc_page(self.host) for _ in range(w.num_chunks * self.ppc)],
+                              dtype=np.int64)
         self.table_dev = torch.tensor(self.table, dtype=torch.int32, device=device)
         self.copy = torch.cuda.Stream(device=device)
         C, Hq = w.chunk_len, w.num_q_heads
@@ -56,17 +61,18 @@ class OffloadRun:
         ws = L.page_topk_workspace_size(C, Hq, Hkv, d, max(1, (w.num_chunks - 1) * self.ppc))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        n = self.parts
         self.cur_dev = [torch.tensor(self.stage_pages[b * self.half + self.sel_max:
                                                       (b + 1) * self.half],
-                                     dtype=torch.int32, device=device) for b in range(2)]
+                                     dtype=torch.int32, device=device) for b in range(n)]
         self.past_dev = [torch.zeros((Hkv, self.sel_max), dtype=torch.int32, device=device)
-                         for _ in range(2)]
-        # pinned upload buffers per half: rewritten two chunks after their last copy,
+                         for _ in range(n)]
+        # pinned upload buffers per part: rewritten three chunks after their last copy,
         # by which time the host has synchronised on later copy-stream events
         self.past_host = [torch.zeros((Hkv, self.sel_max), dtype=torch.int32).pin_memory()
-                          for _ in range(2)]
-        self.cnt_host = [torch.zeros(Hkv, dtype=torch.int32).pin_memory() for _ in range(2)]
-        self.cnt_dev = [torch.zeros(Hkv, dtype=torch.int32, device=device) for _ in range(2)]
+                          for _ in range(n)]
+        self.cnt_host = [torch.zeros(Hkv, dtype=torch.int32).pin_memory() for _ in range(n)]
+        self.cnt_dev = [torch.zeros(Hkv, dtype=torch.int32, device=device) for _ in range(n)]
         self.h2d_bytes = 0
         self.d2h_bytes = 0
         self.selections = []
@@ -78,9 +84,11 @@ class OffloadRun:
             L.pool_destroy(self.host)
 
     # ---------------------------------------------------------------- helpers
-    def _blocks_of_pages(self, pages, heads):
+    def _blocks_of_pages(self, pages):
+        """Block ids (page * Hkv + head) of whole pages, page-major."""
         Hkv = self.w.num_kv_heads
-        return [p * Hkv + h for p in pages for h in heads]
+        return (np.asarray(pages, dtype=np.int64)[:, None] * Hkv
+                + np.arange(Hkv, dtype=np.int64)[None, :]).reshape(-1)
 
     def _select(self, c, q):
         """Top-K for chunk c on the copy stream; returns an event recorded after
@@ -105,25 +113,28 @@ class OffloadRun:
         return [ids[g, :cnt[g]].tolist() for g in range(Hkv)]
 
     def _prefetch(self, c, sel):
-        """Selected blocks of chunk c into staging half c % 2 (copy stream)."""
-        b = c % 2
+        """Selected blocks of chunk c into staging part c % 3 (copy stream)."""
+        b = c % self.parts
         Hkv = self.w.num_kv_heads
-        src, dst = [], []
-        past = self.past_host[b]
-        past.zero_()
+        counts = np.array([len(x) for x in sel], dtype=np.int64)
+        slots = self.stage_pages[b * self.half: b * self.half + self.sel_max]
+        past = self.past_host[b].numpy()
+        past[:] = 0
         # slot-major order: staging blocks (slot i, head g) are consecutive, so the
         # gradient write-back of these blocks is one large device->host copy
-        for i in range(max(len(x) for x in sel)):
-            for g in range(Hkv):
-                if i < len(sel[g]):
-                    src.append(self.table[sel[g][i]] * Hkv + g)
-                    dst.append(self.stage_pages[b * self.half + i] * Hkv + g)
-                    past[g, i] = self.stage_pages[b * self.half + i]
-        for g in range(Hkv):
-            self.cnt_host[b][g] = len(sel[g])
+        src, dst = [], []
+        for i in range(int(counts.max()) if len(counts) else 0):
+            gs = np.nonzero(counts > i)[0]
+            lp = np.array([sel[g][i] for g in gs], dtype=np.int64)
+            src.append(self.table[lp] * Hkv + gs)
+            dst.append(slots[i] * Hkv + gs)
+            past[gs, i] = slots[i]
+        src = np.concatenate(src) if src else np.zeros(0, dtype=np.int64)
+        dst = np.concatenate(dst) if dst else np.zeros(0, dtype=np.int64)
+        self.cnt_host[b].numpy()[:] = counts
         ev = torch.cuda.Event()
         with torch.cuda.stream(self.copy):
-            self.past_dev[b].copy_(past, non_blocking=True)
+            self.past_dev[b].copy_(self.past_host[b], non_blocking=True)
             self.cnt_dev[b].copy_(self.cnt_host[b], non_blocking=True)
             L.page_prefetch(self.host, self.stage, src, dst, stream=self.copy, done_event=ev)
         self.h2d_bytes += len(src) * 2 * self.w.page_size * self.w.head_dim * 2
@@ -143,13 +154,13 @@ class OffloadRun:
         w = self.w
         N, Hkv = w.num_chunks, w.num_kv_heads
         comp = torch.cuda.current_stream(self.dev)
-        heads = list(range(Hkv))
         scratch = None
         pending = None          # (prefetch event, (host blocks, staging blocks)) of chunk c
         prev = None             # (computed event, gradient blocks) of chunk c-1
         self.selections = [[[] for _ in range(Hkv)]]
+        empty = np.zeros(0, dtype=np.int64)
         for c in range(N):
-            b = c % 2
+            b = c % self.parts
             x = chunks(c)
             cur_pages = self.stage_pages[b * self.half + self.sel_max:(b + 1) * self.half]
             if outputs is not None:
@@ -162,14 +173,13 @@ class OffloadRun:
                 o, lse, dq = scratch
             if pending is not None:
                 comp.wait_event(pending[0])
-            pf_blocks = pending[1] if pending is not None else ([], [])
-            # append chunk c into the half's current pages; store them on the host
+            pf_blocks = pending[1] if pending is not None else (empty, empty)
+            # append chunk c into the part's current pages; store them on the host
             L.kv_append(self.stage, self.cur_dev[b], x["k"], x["v"], comp)
             appended = torch.cuda.Event()
             appended.record(comp)
-            host_pages = self.table[c * self.ppc:(c + 1) * self.ppc]
-            store_src = self._blocks_of_pages(cur_pages, heads)
-            store_dst = self._blocks_of_pages(host_pages, heads)
+            store_src = self._blocks_of_pages(cur_pages)
+            store_dst = self._blocks_of_pages(self.table[c * self.ppc:(c + 1) * self.ppc])
             self.copy.wait_event(appended)
             L.page_prefetch(self.stage, self.host, store_src, store_dst, stream=self.copy)
             self.d2h_bytes += len(store_src) * 2 * w.page_size * w.head_dim * 2
@@ -185,19 +195,18 @@ class OffloadRun:
             computed = torch.cuda.Event()
             computed.record(comp)
             # gradient blocks of chunk c: its selected past blocks and its own pages
-            grads = (list(pf_blocks[1]) + store_src, list(pf_blocks[0]) + store_dst)
-            sel_next = None
+            grads = (np.concatenate([pf_blocks[1], store_src]),
+                     np.concatenate([pf_blocks[0], store_dst]))
             if ev_sel is not None:
                 sel_next = self._read_selection(ev_sel)
                 self.selections.append(sel_next)
+                # part (c+1) % 3 last served chunk c-2, drained by its write-back
+                # (issued in iteration c-1, earlier on the copy stream)
+                pending = self._prefetch(c + 1, sel_next)
             if backward and prev is not None:
                 self.copy.wait_event(prev[0])
                 self._writeback(c - 1, prev[1])
             prev = (computed, grads)
-            if sel_next is not None:
-                # staging half (c+1)%2 was last read by chunk c-1, whose write-back
-                # (above, same stream) waited for it
-                pending = self._prefetch(c + 1, sel_next)
         if backward and prev is not None:
             self.copy.wait_event(prev[0])
             self._writeback(N - 1, prev[1])
