@@ -411,7 +411,6 @@ def offload_run(w, steps, device, dist_on):
     try:
         run.run(lambda c: ins[c])  # warm-up pass (also fills the host pools)
         run.sync()
-        run.h2d_bytes = run.d2h_bytes = 0
         _barrier(dist_on)
         comp = torch.cuda.current_stream()
         a = torch.cuda.Event(enable_timing=True)
@@ -421,24 +420,145 @@ def offload_run(w, steps, device, dist_on):
         for _ in range(steps):
             run.run(lambda c: ins[c])
         b.record(comp)
-        run.sync()  # includes the host-side gradient additions of the last chunks
+        run.sync()  # every gradient addition is stream-ordered on the device
         wall = (time.perf_counter() - t0) * 1e3 / steps
         ev_ms = a.elapsed_time(b) / steps
-        # the step ends when the host gradients are complete: take the later clock
-        ms = _max_over_ranks(max(ev_ms, wall), dist_on, device)
+        ms = _max_over_ranks(ev_ms, dist_on, device)
         import paged_kv_chunk_query_b200 as pk
-        status = pk.get_device_status(run.stage)
-        h2d, d2h = run.h2d_bytes / steps, run.d2h_bytes / steps
+        status = pk.get_device_status(run.stage) | pk.get_device_status(run.host)
+        h2d, d2h = run.link_bytes()
     finally:
         run.close()
         del ins
         torch.cuda.empty_cache()
     return {"workload": w.name, "context": w.context, "ms_per_step": ms,
-            "ms_per_step_device_events": ev_ms, "ms_per_step_wall_incl_host_adds": wall,
+            "ms_per_step_wall": wall,
             "ms_per_chunk": ms / w.num_chunks, "tokens_per_s": w.context / (ms / 1e3),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "h2d_gbs": h2d / (ms / 1e3) / 1e9, "d2h_gbs": d2h / (ms / 1e3) / 1e9,
+            "link_bytes_note": "host link: prefetched KV + host gradients read for the "
+                               "additions (h2d); stored KV + gradients written back (d2h)",
             "device_status": status}
+
+
+# ------------------------------------------------------------------ HBM / host-link kernels
+def _event_ms(fn, reps=5, warmup=2):
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def hbm_kernels(w, device, peaks):
+    """The memory-bound kernels measured in batched launches (per-chunk
+    launches are microseconds long): the append of a whole 256K context in
+    one launch, every chunk's Top-K in one batched launch, a gather and a
+    gradient scatter-add of every (page, head) block of a shuffled 4096-page
+    pool, and the same moves over the host link against a measured pinned
+    memcpy peak.  Inputs are larger than L2 (512 MiB pools, 1.75 GiB of Q)."""
+    import paged_kv_chunk_query_b200 as pk
+    P, Hkv, d, Hq, C, N = (w.page_size, w.num_kv_heads, w.head_dim, w.num_q_heads, w.chunk_len,
+                           w.num_chunks)
+    T, npg = w.context, w.num_pages
+    dev_i = device.index or 0
+    hbm = peaks["hbm_gbs"]
+    out = {}
+
+    def entry(nbytes, ms, peak, what):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac": gbs / peak, "what": what}
+
+    a = pk.pool_create(npg, P, Hkv, d, pk.LOC_DEVICE, True, w.alloc_seed or 1, dev_i)
+    b = pk.pool_create(npg, P, Hkv, d, pk.LOC_DEVICE, True, 0, dev_i)
+    h = None
+    try:
+        table = torch.tensor([pk.pool_alloc_page(a) for _ in range(npg)], dtype=torch.int32,
+                             device=device)
+        gen = torch.Generator(device=device).manual_seed(w.seed)
+        k = torch.randn((T, Hkv, d), generator=gen, device=device).to(torch.bfloat16)
+        v = torch.randn((T, Hkv, d), generator=gen, device=device).to(torch.bfloat16)
+        ms = _event_ms(lambda: pk.kv_append(a, table, k, v))
+        nb = 2 * T * Hkv * d * 2 * 2 + 2 * T * Hkv * d * 4 + npg * Hkv * d * 4
+        out["kv_append_whole_context"] = entry(
+            nb, ms, hbm, f"{T} tokens into {npg} shuffled pages in one launch: K,V read + "
+            "written, fp32 page means written, fp32 gradient blocks zeroed")
+        del k, v
+        # every chunk's Top-K in one batched launch
+        q_all = torch.randn((N * C, Hq, d), generator=gen, device=device).to(torch.bfloat16)
+        n_past = torch.tensor([c * w.pages_per_chunk for c in range(N)], dtype=torch.int32,
+                              device=device)
+        row_start = torch.tensor([c * C for c in range(N + 1)], dtype=torch.int32, device=device)
+        K, R = 64, 2
+        max_past = (N - 1) * w.pages_per_chunk
+        out_l = torch.empty((N, Hkv, K + R), dtype=torch.int32, device=device)
+        out_c = torch.empty((N, Hkv), dtype=torch.int32, device=device)
+        ws = torch.empty(pk.page_topk_batched_workspace_size(N, Hkv, d, max_past),
+                         dtype=torch.uint8, device=device)
+        ms = _event_ms(lambda: pk.page_topk_batched(a, q_all, row_start, C, n_past, max_past,
+                                                    table, K, R, out_l, None, out_c, ws))
+        n_scored = int(n_past.sum())
+        nb = N * C * Hq * d * 2 + n_scored * (Hkv * d * 4 + 4) + N * Hkv * (K + R) * 4
+        out["topk_batched_all_chunks"] = entry(
+            nb, ms, hbm, f"{N} chunks x {Hkv} groups in one batched call (query means of "
+            f"{N * C} rows, {n_scored} page scores per group, K={K}, R={R})")
+        del q_all
+        # gather / scatter-add of every block of the shuffled pool
+        nblk = npg * Hkv
+        perm = torch.randperm(nblk, device=device, generator=gen).to(torch.int32)
+        ident = torch.arange(nblk, dtype=torch.int32, device=device)
+        ms = _event_ms(lambda: pk.block_copy(a, b, perm, ident))
+        nb = nblk * (2 * P * d * 2 * 2 + d * 4 * 2)
+        out["block_gather_all_pages"] = entry(nb, ms, hbm, f"{nblk} shuffled (page, head) "
+                                              "blocks (K, V, page mean) device -> device")
+        ms = _event_ms(lambda: pk.grad_block_add(a, b, perm, ident, zero_src=False))
+        nb = nblk * 2 * P * d * 4 * 3
+        out["grad_scatter_add_all_pages"] = entry(nb, ms, hbm, f"{nblk} shuffled fp32 gradient "
+                                                  "blocks added into another pool (read src, "
+                                                  "read + write dst)")
+        # host link: memcpy peak, then the same moves to / from pinned pages
+        big = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+        dbig = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        ms_h2d = _event_ms(lambda: dbig.copy_(big, non_blocking=True), reps=3)
+        ms_d2h = _event_ms(lambda: big.copy_(dbig, non_blocking=True), reps=3)
+        peak_h2d = (256 << 20) / (ms_h2d / 1e3) / 1e9
+        peak_d2h = (256 << 20) / (ms_d2h / 1e3) / 1e9
+        del big, dbig
+        h = pk.pool_create(npg, P, Hkv, d, pk.LOC_PINNED_HOST, True, 0, dev_i)
+        blk_kv = 2 * P * d * 2
+        ms = _event_ms(lambda: pk.block_copy(a, h, perm, ident), reps=3)
+        link = {"memcpy_h2d_gbs": peak_h2d, "memcpy_d2h_gbs": peak_d2h}
+        link["store_all_blocks_d2h"] = entry(nblk * blk_kv, ms, peak_d2h,
+                                             f"{nblk} shuffled KV blocks device -> pinned host")
+        ms = _event_ms(lambda: pk.block_copy(h, b, ident, perm), reps=3)
+        link["gather_all_blocks_h2d"] = entry(nblk * blk_kv, ms, peak_h2d,
+                                              f"{nblk} KV blocks pinned host -> shuffled device")
+        sel = perm[:(K + R) * Hkv].contiguous()
+        ms = _event_ms(lambda: pk.block_copy(h, b, sel, ident[:sel.numel()].contiguous()))
+        link["gather_one_chunk_selection_h2d"] = entry(
+            sel.numel() * blk_kv, ms, peak_h2d, f"{sel.numel()} KV blocks (one chunk's "
+            "selection) pinned host -> device")
+        ms = _event_ms(lambda: pk.grad_block_add(a, h, perm, ident, zero_src=False), reps=3)
+        link["grad_add_all_blocks_to_host"] = entry(
+            nblk * 2 * P * d * 4, ms, min(peak_h2d, peak_d2h), f"{nblk} fp32 gradient blocks "
+            "added into pinned host pages (each byte crosses the link both ways)")
+        out["host_link"] = link
+        torch.cuda.synchronize()
+        out["device_status"] = (pk.get_device_status(a) | pk.get_device_status(b) |
+                                pk.get_device_status(h))
+    finally:
+        for pool in (a, b, h):
+            if pool:
+                pk.pool_destroy(pool)
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -511,6 +631,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-offload", action="store_true")
+    ap.add_argument("--no-hbm", action="store_true", help="skip the batched HBM/host-link kernels")
     ap.add_argument("--serial-bwd", action="store_true",
                     help="run each chunk's dQ launch after its dK/dV launch on one stream")
     ap.add_argument("--offload-workload", default="qwen1m_topk_offload")
@@ -642,6 +763,10 @@ def main():
                 offload_obj["ms_per_chunk"] / per_chunk_dev - 1.0)
         offload_obj["tokens_per_s"] *= world
 
+    hbm_obj = None
+    if not a.no_hbm:
+        hbm_obj = hbm_kernels(w, device, peaks)
+
     e2e = None
     if not a.no_e2e:
         ms_e, h2d, d2h = e2e_dense(w, max(1, min(a.steps, 2)), device)
@@ -677,6 +802,7 @@ def main():
         "roofline": roof,
         "sparse": sparse_obj,
         "offload": offload_obj,
+        "hbm_kernels": hbm_obj,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": w.num_chunks * 5 * a.steps

@@ -205,6 +205,34 @@ oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* d_q, int32_
                                   int32_t* d_out_logical, int32_t* d_out_physical,
                                   int32_t* d_out_count, float* d_out_scores, void* stream);
 
+/* Batched Top-K: n_problems independent selections in one set of launches
+ * (three kernels for the whole batch).  Problem b takes the query rows
+ * [d_row_start[b], d_row_start[b+1]) of d_q ([num_rows][num_q_heads][d]
+ * bf16) and the candidates among logical pages [0, d_n_past[b]) of the one
+ * page table d_page_table (length >= max_past); each problem is exactly one
+ * oomb_page_topk call on those rows.  Uses: the selections of many chunks at
+ * once, and one selection per query page of a chunk ([pt] §2C speaks of the
+ * pages relevant to each query page).
+ *   d_row_start [n_problems + 1], d_n_past [n_problems]: device int32; values
+ *     outside [0, num_rows] / [0, max_past] are clamped and set bit 2 of the
+ *     device status word.
+ *   max_rows: the largest row count of a problem (host-known bound, picks the
+ *     slice count of the query mean; 1 <= max_rows <= num_rows).
+ *   Outputs [n_problems][Hkv][top_k + n_recent] (ids), [n_problems][Hkv]
+ *     (counts), optional scores [n_problems][Hkv][max_past].
+ *   Workspace: oomb_page_topk_batched_workspace_size(n_problems, Hkv, d,
+ *     max_past) bytes, 16-byte aligned; n_problems <= 65535. */
+size_t oomb_page_topk_batched_workspace_size(int32_t n_problems, int32_t num_kv_heads,
+                                             int32_t head_dim, int32_t max_past);
+oomb_status oomb_page_topk_batched(const oomb_pool* pool, const void* d_q, int32_t num_rows,
+                                   int32_t num_q_heads, int32_t n_problems,
+                                   const int32_t* d_row_start, int32_t max_rows,
+                                   const int32_t* d_n_past, int32_t max_past,
+                                   const int32_t* d_page_table, int32_t top_k, int32_t n_recent,
+                                   int32_t* d_out_logical, int32_t* d_out_physical,
+                                   int32_t* d_out_count, float* d_out_scores, void* d_workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- offload
  * A block is the K and V of one page and one KV head: block id = page *
  * num_kv_heads + head, contiguous in both pools ([pt] §2D, [it] §2C: KV and
@@ -241,6 +269,56 @@ oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* host_pool,
  * device pool has been applied to the host pool (OOMB_ERR_TIMEOUT after
  * timeout_us microseconds). */
 oomb_status oomb_grad_writeback_sync(oomb_pool* device_pool, int64_t timeout_us);
+
+/* ---------------------------------------------------------------- block moves with device lists
+ * The same moves as above, but driven by block lists that live in DEVICE
+ * memory (int32, caller-owned) and executed by one kernel launch each, so
+ * that lists computed on the GPU (a Top-K selection) never travel to the host
+ * ([pt] §2D: for sparse attention the page ids are known ahead of the
+ * compute, which lets the transfer overlap it).  Pinned-host pools are read
+ * and written in place over the host link (mapped memory); between two
+ * device pools the moves are HBM gathers and scatter-adds.
+ * Common rules: entry i moves src block d_src_blocks[i] to dst block
+ * d_dst_blocks[i]; an entry with a negative id is padding and is skipped; an
+ * id beyond its pool is skipped and sets bit 0 of dst_pool's device status
+ * word; the pools must share page_size, num_kv_heads and head_dim and may not
+ * be OOMB_LOC_HOST; n_blocks == 0 is a no-op; all work is on `stream`.
+ *
+ * oomb_block_copy: dst.kv[dst_i] = src.kv[src_i] and
+ * dst.summary[dst_i] = src.summary[src_i] (the page representative travels
+ * with its block).  Destination ids must be distinct within a call. */
+oomb_status oomb_block_copy(const oomb_pool* src_pool, oomb_pool* dst_pool,
+                            const int32_t* d_src_blocks, const int32_t* d_dst_blocks,
+                            int32_t n_blocks, void* stream);
+/* oomb_grad_block_add: dst.grad[dst_i] += src.grad[src_i] in fp32, then, if
+ * zero_src != 0, src.grad[src_i] = 0.  src_pool must be a device pool; both
+ * pools need gradients.  A device dst_pool is added with vector atomics (a
+ * destination may repeat); a pinned-host dst_pool gets a plain
+ * read-modify-write over the host link, so its destinations must be distinct
+ * within a call.  With zero_src, source ids must be distinct too. */
+oomb_status oomb_grad_block_add(oomb_pool* src_pool, oomb_pool* dst_pool,
+                                const int32_t* d_src_blocks, const int32_t* d_dst_blocks,
+                                int32_t n_blocks, int32_t zero_src, void* stream);
+/* oomb_prefetch_lists: turns a Top-K selection into the lists that move the
+ * selected blocks of src_pool into staging slots of dst_pool.
+ *   d_sel_logical [Hkv][max_sel], d_sel_count [Hkv]: as written by
+ *     oomb_page_topk (logical page ids, ascending, count per group);
+ *   d_page_table [table_len]: logical -> physical page of src_pool;
+ *   d_slot_pages [max_sel]: staging pages of dst_pool; slot i holds the i-th
+ *     selected page of every group (one block per group).
+ * Writes, for entry e = i * Hkv + g (slot-major, max_sel * Hkv entries):
+ *   d_src_blocks[e] = table[sel[g][i]] * Hkv + g, d_dst_blocks[e] =
+ *   slot_pages[i] * Hkv + g when i < count[g], else -1 (padding);
+ *   d_past_pages[g][i] = slot_pages[i] (0 past the count): the past page list
+ *   of the staging pool for oomb_chunk_attn_fwd / _bwd, with d_sel_count as
+ *   its counts.
+ * Ids out of range set bit 0 (a count out of [0, max_sel] bit 2) of
+ * dst_pool's device status word and give padding entries. */
+oomb_status oomb_prefetch_lists(const oomb_pool* src_pool, oomb_pool* dst_pool,
+                                const int32_t* d_sel_logical, const int32_t* d_sel_count,
+                                int32_t max_sel, const int32_t* d_page_table, int32_t table_len,
+                                const int32_t* d_slot_pages, int32_t* d_src_blocks,
+                                int32_t* d_dst_blocks, int32_t* d_past_pages, void* stream);
 
 /* ---------------------------------------------------------------- status
  * Waits for a cudaEvent_t (given as void*) by polling, for at most timeout_us

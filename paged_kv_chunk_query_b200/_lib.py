@@ -35,7 +35,8 @@ EXPORTS = (
     "oomb_page_topk_workspace_size", "oomb_page_topk", "oomb_page_prefetch",
     "oomb_grad_writeback", "oomb_wait", "oomb_get_device_status", "oomb_status_string",
     "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
-    "oomb_selftest_wait_limit",
+    "oomb_selftest_wait_limit", "oomb_page_topk_batched_workspace_size", "oomb_page_topk_batched",
+    "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists",
 )
 
 
@@ -94,6 +95,11 @@ def load() -> ctypes.CDLL:
         "oomb_wait": [vp, ctypes.c_int64],
         "oomb_get_device_status": [vp, ctypes.POINTER(ctypes.c_uint32)],
         "oomb_selftest_wait_limit": [vp, vp],
+        "oomb_page_topk_batched": [vp, vp, i32, i32, i32, vp, i32, vp, i32, vp, i32, i32, vp, vp,
+                                   vp, vp, vp, ctypes.c_size_t, vp],
+        "oomb_block_copy": [vp, vp, vp, vp, i32, vp],
+        "oomb_grad_block_add": [vp, vp, vp, vp, i32, i32, vp],
+        "oomb_prefetch_lists": [vp, vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):  # completeness is checked by the export test
@@ -104,6 +110,9 @@ def load() -> ctypes.CDLL:
     if hasattr(lib, "oomb_page_topk_workspace_size"):
         lib.oomb_page_topk_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         lib.oomb_page_topk_workspace_size.restype = ctypes.c_size_t
+    if hasattr(lib, "oomb_page_topk_batched_workspace_size"):
+        lib.oomb_page_topk_batched_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.oomb_page_topk_batched_workspace_size.restype = ctypes.c_size_t
     lib.oomb_status_string.argtypes = [ctypes.c_int]
     lib.oomb_status_string.restype = ctypes.c_char_p
     lib.oomb_version.argtypes = []
@@ -300,6 +309,32 @@ def page_topk(pool, q, page_table, n_past, top_k, n_recent, out_logical, out_phy
         "oomb_page_topk")
 
 
+def page_topk_batched_workspace_size(n_problems, num_kv_heads, head_dim, max_past) -> int:
+    return load().oomb_page_topk_batched_workspace_size(n_problems, num_kv_heads, head_dim,
+                                                        max_past)
+
+
+def page_topk_batched(pool, q, row_start, max_rows, n_past, max_past, page_table, top_k,
+                      n_recent, out_logical, out_physical, out_count, workspace,
+                      out_scores=None, stream=None):
+    """oomb_page_topk_batched: one selection per problem b (query rows
+    row_start[b]:row_start[b+1] of q, candidates among the first n_past[b]
+    logical pages of page_table); outputs [B][Hkv][K+R] / [B][Hkv]."""
+    T, Hq, _ = q.shape
+    B = n_past.numel()
+    _check(load().oomb_page_topk_batched(
+        pool, _dev_tensor(q, torch.bfloat16, "q"), T, Hq, B,
+        _dev_tensor(row_start, torch.int32, "row_start"), max_rows,
+        _dev_tensor(n_past, torch.int32, "n_past"), max_past,
+        _dev_tensor(page_table, torch.int32, "page_table") if max_past else None, top_k, n_recent,
+        _dev_tensor(out_logical, torch.int32, "out_logical"),
+        _dev_tensor(out_physical, torch.int32, "out_physical") if out_physical is not None
+        else None, _dev_tensor(out_count, torch.int32, "out_count"),
+        _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
+        _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "oomb_page_topk_batched")
+
+
 TOPK_STATIC_SCRATCH_BYTES = 1 << 20
 
 
@@ -343,6 +378,45 @@ def grad_writeback(device_pool, host_pool, src_blocks, dst_blocks, stream=None):
 
 def grad_writeback_sync(device_pool, timeout_us: int = 120_000_000):
     _check(load().oomb_grad_writeback_sync(device_pool, timeout_us), "oomb_grad_writeback_sync")
+
+
+def block_copy(src_pool, dst_pool, src_blocks, dst_blocks, stream=None):
+    """oomb_block_copy with block lists in device memory (int32 CUDA tensors)."""
+    n = src_blocks.numel()
+    if dst_blocks.numel() != n:
+        raise ValueError("src_blocks and dst_blocks differ in length")
+    _check(load().oomb_block_copy(src_pool, dst_pool,
+                                  _dev_tensor(src_blocks, torch.int32, "src_blocks"),
+                                  _dev_tensor(dst_blocks, torch.int32, "dst_blocks"), n,
+                                  _stream(stream)), "oomb_block_copy")
+
+
+def grad_block_add(src_pool, dst_pool, src_blocks, dst_blocks, zero_src=True, stream=None):
+    """oomb_grad_block_add with block lists in device memory."""
+    n = src_blocks.numel()
+    if dst_blocks.numel() != n:
+        raise ValueError("src_blocks and dst_blocks differ in length")
+    _check(load().oomb_grad_block_add(src_pool, dst_pool,
+                                      _dev_tensor(src_blocks, torch.int32, "src_blocks"),
+                                      _dev_tensor(dst_blocks, torch.int32, "dst_blocks"), n,
+                                      int(bool(zero_src)), _stream(stream)),
+           "oomb_grad_block_add")
+
+
+def prefetch_lists(src_pool, dst_pool, sel_logical, sel_count, page_table, slot_pages,
+                   out_src_blocks, out_dst_blocks, out_past_pages, stream=None):
+    """oomb_prefetch_lists: selection [Hkv][max_sel] -> slot-major block lists
+    [max_sel * Hkv] and the staging past-page list [Hkv][max_sel]."""
+    max_sel = sel_logical.shape[1]
+    _check(load().oomb_prefetch_lists(
+        src_pool, dst_pool, _dev_tensor(sel_logical, torch.int32, "sel_logical"),
+        _dev_tensor(sel_count, torch.int32, "sel_count"), max_sel,
+        _dev_tensor(page_table, torch.int32, "page_table") if page_table.numel() else None,
+        page_table.numel(), _dev_tensor(slot_pages, torch.int32, "slot_pages"),
+        _dev_tensor(out_src_blocks, torch.int32, "out_src_blocks"),
+        _dev_tensor(out_dst_blocks, torch.int32, "out_dst_blocks"),
+        _dev_tensor(out_past_pages, torch.int32, "out_past_pages"), _stream(stream)),
+        "oomb_prefetch_lists")
 
 
 def wait(event, timeout_us: int):

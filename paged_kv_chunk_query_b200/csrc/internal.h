@@ -21,7 +21,11 @@ struct oomb_pool {
   void* kv = nullptr;          // bf16 [pages][Hkv][2][P][d]
   float* grad = nullptr;       // fp32, same shape (optional)
   float* summary = nullptr;    // fp32 [pages][Hkv][d]
-  uint32_t* d_status = nullptr;  // device status word (device pools)
+  uint32_t* d_status = nullptr;  // device status word (device and pinned pools)
+  // kernel-side addresses of kv / grad (pinned pools: the mapped device
+  // pointers of the host pages; device pools: kv / grad themselves)
+  void* kv_dev = nullptr;
+  float* grad_dev = nullptr;
   std::vector<int32_t> free_stack;  // top = back()
   std::vector<uint8_t> used;
   std::mutex mu;

@@ -82,12 +82,21 @@ oomb_status oomb_pool_create(const oomb_pool_desc* desc, oomb_pool** out_pool) {
     ok = ok && cudaMalloc(reinterpret_cast<void**>(&p->d_status), sizeof(uint32_t)) == cudaSuccess;
     ok = ok && cudaMemset(p->d_status, 0, sizeof(uint32_t)) == cudaSuccess;
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    p->kv_dev = p->kv;
+    p->grad_dev = p->grad;
   } else if (desc->location == OOMB_LOC_PINNED_HOST) {
     oomb::DeviceGuard g(desc->device);
-    ok = ok && cudaHostAlloc(&p->kv, kv_bytes, cudaHostAllocPortable) == cudaSuccess;
+    // mapped: the block-copy kernels read and write these pages directly over
+    // the host link
+    const unsigned flags = cudaHostAllocPortable | cudaHostAllocMapped;
+    ok = ok && cudaHostAlloc(&p->kv, kv_bytes, flags) == cudaSuccess;
     if (desc->with_grad)
-      ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&p->grad), grad_bytes,
-                               cudaHostAllocPortable) == cudaSuccess;
+      ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&p->grad), grad_bytes, flags) ==
+                     cudaSuccess;
+    ok = ok && cudaHostGetDevicePointer(&p->kv_dev, p->kv, 0) == cudaSuccess;
+    if (ok && p->grad)
+      ok = cudaHostGetDevicePointer(reinterpret_cast<void**>(&p->grad_dev), p->grad, 0) ==
+           cudaSuccess;
     // Page representatives stay in device memory: Top-K reads them on the GPU.
     ok = ok && cudaMalloc(reinterpret_cast<void**>(&p->summary), sum_bytes) == cudaSuccess;
     ok = ok && cudaMemset(p->summary, 0, sum_bytes) == cudaSuccess;

@@ -14,18 +14,22 @@ The staging pool has three parts used by chunks in turn, so chunk c+1's
 prefetch fills one part while chunk c computes on another and chunk c-1's
 gradients drain from the third.
 
-Per chunk c (compute stream C, copy stream S; part = c % 3):
+Nothing goes through the host between Top-K and the prefetch: the selection
+stays on the device, oomb_prefetch_lists turns it into block lists, and
+oomb_block_copy / oomb_grad_block_add move the blocks by reading and writing
+the pinned pages in place (one launch per list).  The host only enqueues.
+
+Per chunk c (compute stream C, copy stream S with higher priority; part =
+c % 3):
   C: wait for prefetch(c); append K_c, V_c into the part's current pages
      (page summaries, zeroed gradient blocks)
   S: store those pages and summaries into the host pool
-  S: Top-K for chunk c+1 against the host pool's summaries; selection -> host
+  S: Top-K for chunk c+1 against the host pool's summaries, its block lists,
+     and the prefetch of its blocks into part (c+1) % 3
   C: forward + backward of chunk c on the staging part
-  host: wait for the selection of c+1, build the block lists
-  S: prefetch chunk c+1's selected blocks into part (c+1) % 3, then write
-     back chunk c-1's gradient deltas (D2H, zero-fill; the host add runs on
-     the library's worker thread)
-Part (c+1) % 3 was last used by chunk c-2, whose write-back (issued in
-iteration c-1, earlier on S) has drained and zeroed its gradient blocks.
+  S: once chunk c-1 has computed, add its gradient blocks into the host pool
+     and zero them on the device
+Part (c+1) % 3 was last used by chunk c-2, whose write-back came earlier on S.
 """
 from __future__ import annotations
 
@@ -39,6 +43,7 @@ class OffloadRun:
     def __init__(self, w, device, host_pool=None):
         self.w, self.dev = w, device
         P, Hkv, d = w.page_size, w.num_kv_heads, w.head_dim
+        N = w.num_chunks
         self.sel_max = w.top_k + w.n_recent
         self.ppc = w.pages_per_chunk
         self.parts = 3
@@ -48,34 +53,40 @@ class OffloadRun:
         self.own_host = host_pool is None
         self.stage = L.pool_create(self.parts * self.half, P, Hkv, d, L.LOC_DEVICE, True, 0,
                                    device.index or 0)
-        self.stage_pages = np.array([L.pool_alloc_page(self.stage)
-                                     for _ in range(self.parts * self.half)], dtype=np.int64)
-        self.table = np.array([L.pool_alloc_page(self.host) for _ in range(w.num_chunks * self.ppc)],
+        stage_pages = np.array([L.pool_alloc_page(self.stage)
+                                for _ in range(self.parts * self.half)], dtype=np.int64)
+        self.table = np.array([L.pool_alloc_page(self.host) for _ in range(N * self.ppc)],
                               dtype=np.int64)
-        self.table_dev = torch.tensor(self.table, dtype=torch.int32, device=device)
-        self.copy = torch.cuda.Stream(device=device)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.table_dev = torch.tensor(self.table, **i32)
+        # a higher-priority copy stream: its short kernels take SMs as soon as
+        # an attention CTA retires
+        self.copy = torch.cuda.Stream(device=device, priority=-1)
         C, Hq = w.chunk_len, w.num_q_heads
-        self.sel_l = torch.zeros((Hkv, self.sel_max), dtype=torch.int32, device=device)
-        self.sel_n = torch.zeros(Hkv, dtype=torch.int32, device=device)
-        self.sel_host = torch.zeros((Hkv * self.sel_max + Hkv,), dtype=torch.int32).pin_memory()
-        ws = L.page_topk_workspace_size(C, Hq, Hkv, d, max(1, (w.num_chunks - 1) * self.ppc))
+        heads = np.arange(Hkv, dtype=np.int64)
+
+        def blocks(pages):  # page-major block ids of whole pages
+            return (np.asarray(pages, dtype=np.int64)[:, None] * Hkv + heads[None, :]).reshape(-1)
+
+        n = self.parts
+        slots = [stage_pages[b * self.half: b * self.half + self.sel_max] for b in range(n)]
+        cur = [stage_pages[b * self.half + self.sel_max:(b + 1) * self.half] for b in range(n)]
+        self.slots_dev = [torch.tensor(x, **i32) for x in slots]
+        self.cur_dev = [torch.tensor(x, **i32) for x in cur]
+        self.cur_blocks = [torch.tensor(blocks(x), **i32) for x in cur]
+        # host blocks of every chunk's own pages, [N][ppc * Hkv]
+        self.own_host_blocks = torch.tensor(blocks(self.table).reshape(N, -1), **i32)
+        self.sel_l = [torch.zeros((Hkv, self.sel_max), **i32) for _ in range(n)]
+        self.cnt_dev = [torch.zeros(Hkv, **i32) for _ in range(n)]
+        self.past_dev = [torch.zeros((Hkv, self.sel_max), **i32) for _ in range(n)]
+        self.pf_src = [torch.full((self.sel_max * Hkv,), -1, **i32) for _ in range(n)]
+        self.pf_dst = [torch.full((self.sel_max * Hkv,), -1, **i32) for _ in range(n)]
+        ws = L.page_topk_workspace_size(C, Hq, Hkv, d, max(1, (N - 1) * self.ppc))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
-        n = self.parts
-        self.cur_dev = [torch.tensor(self.stage_pages[b * self.half + self.sel_max:
-                                                      (b + 1) * self.half],
-                                     dtype=torch.int32, device=device) for b in range(n)]
-        self.past_dev = [torch.zeros((Hkv, self.sel_max), dtype=torch.int32, device=device)
-                         for _ in range(n)]
-        # pinned upload buffers per part: rewritten three chunks after their last copy,
-        # by which time the host has synchronised on later copy-stream events
-        self.past_host = [torch.zeros((Hkv, self.sel_max), dtype=torch.int32).pin_memory()
-                          for _ in range(n)]
-        self.cnt_host = [torch.zeros(Hkv, dtype=torch.int32).pin_memory() for _ in range(n)]
-        self.cnt_dev = [torch.zeros(Hkv, dtype=torch.int32, device=device) for _ in range(n)]
-        self.h2d_bytes = 0
-        self.d2h_bytes = 0
-        self.selections = []
+        # every chunk's selection, copied back for inspection (not on the schedule's path)
+        self.sel_hist = torch.zeros((N, Hkv, self.sel_max), dtype=torch.int32).pin_memory()
+        self.cnt_hist = torch.zeros((N, Hkv), dtype=torch.int32).pin_memory()
 
     def close(self):
         self.sync()
@@ -83,86 +94,21 @@ class OffloadRun:
         if self.own_host:
             L.pool_destroy(self.host)
 
-    # ---------------------------------------------------------------- helpers
-    def _blocks_of_pages(self, pages):
-        """Block ids (page * Hkv + head) of whole pages, page-major."""
-        Hkv = self.w.num_kv_heads
-        return (np.asarray(pages, dtype=np.int64)[:, None] * Hkv
-                + np.arange(Hkv, dtype=np.int64)[None, :]).reshape(-1)
-
-    def _select(self, c, q):
-        """Top-K for chunk c on the copy stream; returns an event recorded after
-        the selection was copied into pinned host memory."""
-        w = self.w
-        n_past = c * self.ppc
-        Hkv = w.num_kv_heads
-        ev = torch.cuda.Event()
-        with torch.cuda.stream(self.copy):
-            L.page_topk(self.host, q, self.table_dev[:n_past], n_past, w.top_k, w.n_recent,
-                        self.sel_l, None, self.sel_n, self.ws, stream=self.copy)
-            self.sel_host[:Hkv * self.sel_max].copy_(self.sel_l.view(-1), non_blocking=True)
-            self.sel_host[Hkv * self.sel_max:].copy_(self.sel_n, non_blocking=True)
-            ev.record(self.copy)
-        return ev
-
-    def _read_selection(self, ev):
-        ev.synchronize()
-        Hkv = self.w.num_kv_heads
-        ids = self.sel_host[:Hkv * self.sel_max].view(Hkv, self.sel_max).numpy()
-        cnt = self.sel_host[Hkv * self.sel_max:].numpy()
-        return [ids[g, :cnt[g]].tolist() for g in range(Hkv)]
-
-    def _prefetch(self, c, sel):
-        """Selected blocks of chunk c into staging part c % 3 (copy stream)."""
-        b = c % self.parts
-        Hkv = self.w.num_kv_heads
-        counts = np.array([len(x) for x in sel], dtype=np.int64)
-        slots = self.stage_pages[b * self.half: b * self.half + self.sel_max]
-        past = self.past_host[b].numpy()
-        past[:] = 0
-        # slot-major order: staging blocks (slot i, head g) are consecutive, so the
-        # gradient write-back of these blocks is one large device->host copy
-        src, dst = [], []
-        for i in range(int(counts.max()) if len(counts) else 0):
-            gs = np.nonzero(counts > i)[0]
-            lp = np.array([sel[g][i] for g in gs], dtype=np.int64)
-            src.append(self.table[lp] * Hkv + gs)
-            dst.append(slots[i] * Hkv + gs)
-            past[gs, i] = slots[i]
-        src = np.concatenate(src) if src else np.zeros(0, dtype=np.int64)
-        dst = np.concatenate(dst) if dst else np.zeros(0, dtype=np.int64)
-        self.cnt_host[b].numpy()[:] = counts
-        ev = torch.cuda.Event()
-        with torch.cuda.stream(self.copy):
-            self.past_dev[b].copy_(self.past_host[b], non_blocking=True)
-            self.cnt_dev[b].copy_(self.cnt_host[b], non_blocking=True)
-            L.page_prefetch(self.host, self.stage, src, dst, stream=self.copy, done_event=ev)
-        self.h2d_bytes += len(src) * 2 * self.w.page_size * self.w.head_dim * 2
-        return ev, (src, dst)
-
-    def _writeback(self, c, blocks):
-        """Gradient deltas of chunk c back into the host pool (copy stream)."""
-        src, dst = blocks
-        with torch.cuda.stream(self.copy):
-            L.grad_writeback(self.stage, self.host, src, dst, stream=self.copy)
-        self.d2h_bytes += len(src) * 2 * self.w.page_size * self.w.head_dim * 4
-
     # ---------------------------------------------------------------- run
     def run(self, chunks, outputs=None, backward=True):
         """chunks(c) -> dict of device tensors q, k, v, do; outputs(c) -> (o, lse,
         dq) device tensors to fill, or None to use scratch buffers."""
         w = self.w
-        N, Hkv = w.num_chunks, w.num_kv_heads
+        N = w.num_chunks
         comp = torch.cuda.current_stream(self.dev)
+        S = self.copy
         scratch = None
-        pending = None          # (prefetch event, (host blocks, staging blocks)) of chunk c
-        prev = None             # (computed event, gradient blocks) of chunk c-1
-        self.selections = [[[] for _ in range(Hkv)]]
-        empty = np.zeros(0, dtype=np.int64)
+        prefetched = None       # event: chunk c's blocks are in its staging part
+        prev_computed = None    # event: chunk c-1's backward has finished
+        self.copy.wait_stream(comp)
         for c in range(N):
             b = c % self.parts
             x = chunks(c)
-            cur_pages = self.stage_pages[b * self.half + self.sel_max:(b + 1) * self.half]
             if outputs is not None:
                 o, lse, dq = outputs(c)
             else:
@@ -171,20 +117,30 @@ class OffloadRun:
                                torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32,
                                            device=self.dev), torch.empty_like(x["q"]))
                 o, lse, dq = scratch
-            if pending is not None:
-                comp.wait_event(pending[0])
-            pf_blocks = pending[1] if pending is not None else (empty, empty)
-            # append chunk c into the part's current pages; store them on the host
+            if prefetched is not None:
+                comp.wait_event(prefetched)
             L.kv_append(self.stage, self.cur_dev[b], x["k"], x["v"], comp)
             appended = torch.cuda.Event()
             appended.record(comp)
-            store_src = self._blocks_of_pages(cur_pages)
-            store_dst = self._blocks_of_pages(self.table[c * self.ppc:(c + 1) * self.ppc])
-            self.copy.wait_event(appended)
-            L.page_prefetch(self.stage, self.host, store_src, store_dst, stream=self.copy)
-            self.d2h_bytes += len(store_src) * 2 * w.page_size * w.head_dim * 2
-            # Top-K of chunk c+1 (every earlier page's summary is now on the host side)
-            ev_sel = self._select(c + 1, chunks(c + 1)["q"]) if c + 1 < N else None
+            S.wait_event(appended)
+            # chunk c's pages (and their representatives) into the host pool
+            L.block_copy(self.stage, self.host, self.cur_blocks[b], self.own_host_blocks[c],
+                         stream=S)
+            if c + 1 < N:
+                b1 = (c + 1) % self.parts
+                n_past = (c + 1) * self.ppc
+                L.page_topk(self.host, chunks(c + 1)["q"], self.table_dev[:n_past], n_past,
+                            w.top_k, w.n_recent, self.sel_l[b1], None, self.cnt_dev[b1], self.ws,
+                            stream=S)
+                L.prefetch_lists(self.host, self.stage, self.sel_l[b1], self.cnt_dev[b1],
+                                 self.table_dev[:n_past], self.slots_dev[b1], self.pf_src[b1],
+                                 self.pf_dst[b1], self.past_dev[b1], stream=S)
+                L.block_copy(self.host, self.stage, self.pf_src[b1], self.pf_dst[b1], stream=S)
+                prefetched = torch.cuda.Event()
+                prefetched.record(S)
+                with torch.cuda.stream(S):
+                    self.sel_hist[c + 1].copy_(self.sel_l[b1], non_blocking=True)
+                    self.cnt_hist[c + 1].copy_(self.cnt_dev[b1], non_blocking=True)
             past = self.past_dev[b] if c else None
             cnt = self.cnt_dev[b] if c else None
             L.chunk_attn_fwd(self.stage, x["q"], o, lse, past, cnt, self.cur_dev[b],
@@ -192,27 +148,49 @@ class OffloadRun:
             if backward:
                 L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, self.delta, past, cnt,
                                  self.cur_dev[b], w.softmax_scale, comp)
-            computed = torch.cuda.Event()
-            computed.record(comp)
-            # gradient blocks of chunk c: its selected past blocks and its own pages
-            grads = (np.concatenate([pf_blocks[1], store_src]),
-                     np.concatenate([pf_blocks[0], store_dst]))
-            if ev_sel is not None:
-                sel_next = self._read_selection(ev_sel)
-                self.selections.append(sel_next)
-                # part (c+1) % 3 last served chunk c-2, drained by its write-back
-                # (issued in iteration c-1, earlier on the copy stream)
-                pending = self._prefetch(c + 1, sel_next)
-            if backward and prev is not None:
-                self.copy.wait_event(prev[0])
-                self._writeback(c - 1, prev[1])
-            prev = (computed, grads)
-        if backward and prev is not None:
-            self.copy.wait_event(prev[0])
-            self._writeback(N - 1, prev[1])
-        comp.wait_stream(self.copy)
+                computed = torch.cuda.Event()
+                computed.record(comp)
+                if prev_computed is not None:
+                    self._writeback(c - 1, prev_computed)
+                prev_computed = computed
+        if backward and prev_computed is not None:
+            self._writeback(N - 1, prev_computed)
+        comp.wait_stream(S)
+
+    def _writeback(self, c, computed):
+        """Chunk c's gradient blocks (its prefetched blocks and its own pages)
+        added into the host pool on the copy stream, zeroed on the device."""
+        b = c % self.parts
+        S = self.copy
+        S.wait_event(computed)
+        if c > 0:
+            L.grad_block_add(self.stage, self.host, self.pf_dst[b], self.pf_src[b], True, stream=S)
+        L.grad_block_add(self.stage, self.host, self.cur_blocks[b], self.own_host_blocks[c], True,
+                         stream=S)
 
     def sync(self):
-        """Waits for the device and for every queued host gradient addition."""
+        """Waits for the device (every copy and gradient addition is stream-ordered)."""
         torch.cuda.synchronize(self.dev)
-        L.grad_writeback_sync(self.stage)
+
+    # ---------------------------------------------------------------- inspection
+    @property
+    def selections(self):
+        """Per chunk, per group, the kept logical page ids (after sync())."""
+        out = [[[] for _ in range(self.w.num_kv_heads)]]
+        for c in range(1, self.w.num_chunks):
+            cnt = self.cnt_hist[c].tolist()
+            out.append([self.sel_hist[c, g, :cnt[g]].tolist() for g in range(len(cnt))])
+        return out
+
+    def link_bytes(self, backward=True):
+        """(host->device, device->host) bytes one run moves over the host link
+        (after sync()): prefetched KV blocks and the host gradients read for
+        the additions; stored KV blocks and the gradients written back."""
+        w = self.w
+        kv_block = 2 * w.page_size * w.head_dim * 2
+        g_block = 2 * w.page_size * w.head_dim * 4
+        sel = int(self.cnt_hist[1:].sum())
+        own = w.num_chunks * self.ppc * w.num_kv_heads
+        h2d = sel * kv_block + ((sel + own) * g_block if backward else 0)
+        d2h = own * kv_block + ((sel + own) * g_block if backward else 0)
+        return h2d, d2h
