@@ -10,16 +10,19 @@
 // ties going to the lower logical id; pages [n_past - R, n_past) are always
 // kept; the output lists ascending logical ids.
 //
-// Kernel 1 (qmean_partial): grid (128 slices, Hkv); each CTA streams a slice of
-//   the chunk's rows with 16-byte loads, 8 in flight per thread, and writes one
-//   fp32 partial sum per d.
-// Kernel 2 (page_score): grid (pages / 64, Hkv); each CTA reduces the partials
-//   in a fixed order into q_bar, then each warp scores 8 pages (float4 loads of
-//   the summaries, shuffle reduction).
-// Kernel 3 (select): one CTA per group; finds the K-th largest 64-bit key
-//   (ordered score, inverted id) by 8-bit radix passes from the top with a
-//   parallel bin scan, stopping once the boundary bin is kept whole, then
-//   compacts the kept ids in ascending order.
+// The kernels take a batch of independent problems (blockIdx.z / .y), each a
+// range of query rows and its own number of past pages; the per-chunk entry
+// points run a batch of one.
+// Kernel 1 (qmean_partial): grid (slices, Hkv, problems); each CTA streams a
+//   slice of its problem's rows with 16-byte loads, 8 in flight per thread,
+//   and writes one fp32 partial sum per d.
+// Kernel 2 (page_score): grid (pages / 64, Hkv, problems); each CTA reduces
+//   the partials in a fixed order into q_bar, then each warp scores 8 pages
+//   (float4 loads of the summaries, shuffle reduction).
+// Kernel 3 (select): one CTA per (group, problem); finds the K-th largest
+//   64-bit key (ordered score, inverted id) by 8-bit radix passes from the top
+//   with a parallel bin scan, stopping once the boundary bin is kept whole,
+//   then compacts the kept ids in ascending order.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -28,7 +31,7 @@
 
 namespace {
 
-constexpr int kSplits = 128;         // query-mean slices per group (~3.5 CTAs per SM at Hkv 4)
+constexpr int kSplits = 128;         // max query-mean slices per (problem, group)
 constexpr int kMeanThreads = 256;
 constexpr int kScoreThreads = 256;   // 8 warps x 8 pages per CTA
 constexpr int kPagesPerScoreCta = 64;
@@ -36,21 +39,69 @@ constexpr int kSelectThreads = 1024;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Slices per (problem, group): about 32 query rows (x G heads) per slice, at
+// most kSplits.  A 4096-row chunk gets 128.
+int choose_splits(int max_rows) {
+  const int s = (max_rows + 31) / 32;
+  return s < 1 ? 1 : (s > kSplits ? kSplits : s);
+}
+
+// A batch of independent selections.  Problem b takes query rows
+// [row_start[b], row_start[b+1]) and candidates among logical pages
+// [0, n_past[b]) of one page table.  With null arrays there is one problem:
+// rows [0, rows0) and n_past0 pages.  Values the device arrays hold out of
+// range are clamped and flagged (bad count).
+struct Problems {
+  const int32_t* row_start;
+  const int32_t* n_past;
+  int rows0, n_past0, max_past, num_rows, splits;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void problem_rows(const Problems& pb, int b, int& r0, int& r1) {
+  if (!pb.row_start) {
+    r0 = 0;
+    r1 = pb.rows0;
+    return;
+  }
+  r0 = pb.row_start[b];
+  r1 = pb.row_start[b + 1];
+  if (r0 < 0 || r1 < r0 || r1 > pb.num_rows) {
+    atomicOr(pb.status, OOMB_DEV_BAD_COUNT);
+    r0 = min(max(r0, 0), pb.num_rows);
+    r1 = min(max(r1, r0), pb.num_rows);
+  }
+}
+
+__device__ __forceinline__ int problem_npast(const Problems& pb, int b) {
+  if (!pb.n_past) return pb.n_past0;
+  const int n = pb.n_past[b];
+  if (n < 0 || n > pb.max_past) {
+    atomicOr(pb.status, OOMB_DEV_BAD_COUNT);
+    return n < 0 ? 0 : pb.max_past;
+  }
+  return n;
+}
+
 // ---------------------------------------------------------------- query mean
-// grid (kSplits, Hkv): CTA (s, g) sums rows (token, head in g) of token slice
-// s.  Each thread keeps 8 independent 16-byte loads in flight (about 32 KiB
-// per CTA), enough with 3-4 CTAs per SM to stream Q at HBM speed.
+// grid (splits, Hkv, problems): CTA (s, g, b) sums rows (token, head in g) of
+// slice s of problem b's tokens.  Each thread keeps 8 independent 16-byte
+// loads in flight (about 32 KiB per CTA), enough with 3-4 CTAs per SM to
+// stream Q at HBM speed.
 template <int D>
 __global__ void __launch_bounds__(kMeanThreads) qmean_partial_kernel(
-    const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, int C, int Hq, int G) {
+    const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, const Problems pb, int Hq,
+    int G) {
   constexpr int VPR = D / 8;               // 16-byte vectors per row
   constexpr int RG = kMeanThreads / VPR;   // rows per pass
   constexpr int U = 8;                     // loads in flight per thread
   __shared__ float red[RG][D];
-  const int split = blockIdx.x, g = blockIdx.y, t = threadIdx.x;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
   const int vec = t % VPR, rg = t / VPR;
-  const int per = (C + kSplits - 1) / kSplits;
-  const int tok0 = split * per, tok1 = min(C, tok0 + per);
+  int r0, r1;
+  problem_rows(pb, b, r0, r1);
+  const int per = (r1 - r0 + pb.splits - 1) / pb.splits;
+  const int tok0 = r0 + split * per, tok1 = min(r1, tok0 + per);
   const int rows = max(0, tok1 - tok0) * G;
   float acc[8];
 #pragma unroll
@@ -81,7 +132,7 @@ __global__ void __launch_bounds__(kMeanThreads) qmean_partial_kernel(
   if (t < D) {
     float s = 0.f;
     for (int r = 0; r < RG; ++r) s += red[r][t];  // fixed order: deterministic
-    partial[(static_cast<size_t>(split) * gridDim.y + g) * D + t] = s;
+    partial[((static_cast<size_t>(b) * pb.splits + split) * gridDim.y + g) * D + t] = s;
   }
 }
 
@@ -92,29 +143,31 @@ __device__ __forceinline__ uint32_t order_f32(float f) {
 }
 
 // ---------------------------------------------------------------- page scores
-// grid (ceil(n_past / 64), Hkv).  Every CTA reduces the kSplits partials of its
-// group in the same fixed order (so all CTAs use the identical q_bar), then
-// each warp scores 8 pages.  Key = (ordered score << 32) | (~logical id).
+// grid (ceil(max_past / 64), Hkv, problems).  Every CTA of a problem reduces
+// its slices' partials in the same fixed order (so all use the identical
+// q_bar), then each warp scores 8 pages.  Key = (ordered score << 32) |
+// (~logical id), stored at [problem][group][max_past].
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads) page_score_kernel(
     const float* __restrict__ partial, const float* __restrict__ summary,
-    const int32_t* __restrict__ page_table, int n_past, int Hkv, int num_pool_pages,
-    float inv_rows, unsigned long long* __restrict__ keys, float* __restrict__ out_scores,
-    uint32_t* status) {
+    const int32_t* __restrict__ page_table, const Problems pb, int Hkv, int G,
+    int num_pool_pages, unsigned long long* __restrict__ keys, float* __restrict__ out_scores) {
   constexpr int kParts = kScoreThreads / D;  // threads per d in the q_bar reduction
   __shared__ float part_sum[kParts][D];
   __shared__ float qbar[D];
-  const int g = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = blockIdx.y, b = blockIdx.z, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int n_past = problem_npast(pb, b);
+  if (static_cast<int>(blockIdx.x) * kPagesPerScoreCta >= n_past) return;  // whole CTA
   {
-    constexpr int PER = kSplits / kParts;  // partials per thread, all loads in flight
+    int r0, r1;
+    problem_rows(pb, b, r0, r1);
+    const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
+    const float inv_rows = rows > 0.f ? 1.0f / rows : 0.f;
     const int d = t % D, part = t / D;
-    float v[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      v[i] = __ldg(partial + (static_cast<size_t>(part * PER + i) * Hkv + g) * D + d);
+    const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D;
     float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) s += v[i];
+#pragma unroll 8
+    for (int i = part; i < pb.splits; i += kParts) s += __ldg(pp + (static_cast<size_t>(i) * Hkv + g) * D + d);
     part_sum[part][d] = s;
     __syncthreads();
     if (t < D) {
@@ -139,7 +192,7 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_kernel(
     if (p < n_past) {
       int phys = __ldg(page_table + p);
       if (phys < 0 || phys >= num_pool_pages) {
-        if (lane == 0) atomicOr(status, OOMB_DEV_BAD_PAGE);
+        if (lane == 0) atomicOr(pb.status, OOMB_DEV_BAD_PAGE);
         phys = 0;
       }
       const float* srow = summary + (static_cast<size_t>(phys) * Hkv + g) * D + lane * EPL;
@@ -164,33 +217,39 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_kernel(
       if (lane == i) mine = acc[i];
     const int p = p0 + lane;
     if (p < n_past) {
-      if (out_scores) out_scores[static_cast<size_t>(g) * n_past + p] = mine;
-      keys[static_cast<size_t>(g) * n_past + p] =
-          (static_cast<unsigned long long>(order_f32(mine)) << 32) |
-          static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
+      const size_t row = (static_cast<size_t>(b) * Hkv + g) * pb.max_past;
+      if (out_scores) out_scores[row + p] = mine;
+      keys[row + p] = (static_cast<unsigned long long>(order_f32(mine)) << 32) |
+                      static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
     }
   }
 }
 
 // ---------------------------------------------------------------- select
-// One CTA per group: the K-th largest candidate key by 8-bit radix passes from
-// the top, each with a parallel suffix scan over the 256 bins; stops early once
-// the boundary bin is taken whole.  Then compacts kept ids in ascending order.
+// One CTA per (group, problem): the K-th largest candidate key by 8-bit radix
+// passes from the top, each with a parallel suffix scan over the 256 bins;
+// stops early once the boundary bin is taken whole.  Then compacts kept ids in
+// ascending order.
 __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
     const unsigned long long* __restrict__ keys_all, const int32_t* __restrict__ page_table,
-    int n_past, int top_k, int n_recent, int num_pool_pages, int32_t* __restrict__ out_logical,
-    int32_t* __restrict__ out_physical, int32_t* __restrict__ out_count) {
+    const Problems pb, int top_k, int n_recent, int num_pool_pages,
+    int32_t* __restrict__ out_logical, int32_t* __restrict__ out_physical,
+    int32_t* __restrict__ out_count) {
   __shared__ unsigned int hist[256];
   __shared__ unsigned int warp_tot[8];
   __shared__ unsigned long long kth_sh;
   __shared__ int need_sh, done_sh;
   __shared__ int warp_sum[kSelectThreads / 32];
   __shared__ int running_sh;
-  const int g = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int n_past = problem_npast(pb, b);
   const int max_sel = top_k + n_recent;
   const int n_cand = max(0, n_past - n_recent);
   const int k_eff = min(top_k, n_cand);
-  const unsigned long long* keys = keys_all + static_cast<size_t>(g) * n_past;
+  const size_t row = static_cast<size_t>(b) * gridDim.x + g;
+  const unsigned long long* keys = keys_all + row * pb.max_past;
+  int32_t* out_l = out_logical + row * max_sel;
+  int32_t* out_p = out_physical ? out_physical + row * max_sel : nullptr;
 
   if (t == 0) {
     kth_sh = 0ull;  // with k_eff >= n_cand every candidate is kept
@@ -208,6 +267,10 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
         if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255ull], 1u);
       }
       __syncthreads();
+      // every thread reads the remaining count here, before the barrier that
+      // precedes its one update below (a read after the update could let a
+      // second bin match)
+      const int need = need_sh;
       // inclusive suffix sum over bins 255..0: thread t < 256 owns bin 255 - t
       unsigned int incl = 0;
       if (t < 256) {
@@ -226,7 +289,6 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
         const int bin = 255 - t;
         const unsigned int v = hist[bin];
         const unsigned int excl = incl - v;
-        const int need = need_sh;
         if (excl < static_cast<unsigned>(need) && static_cast<unsigned>(need) <= incl) {
           kth_sh = prefix | (static_cast<unsigned long long>(bin) << shift);
           need_sh = need - static_cast<int>(excl);
@@ -255,11 +317,10 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
     for (int w = 0; w < warp; ++w) before += warp_sum[w];
     before += __popc(ballot & ((1u << lane) - 1u));
     if (keep && before < max_sel) {
-      out_logical[static_cast<size_t>(g) * max_sel + before] = p;
-      if (out_physical) {
+      out_l[before] = p;
+      if (out_p) {
         const int phys = page_table[p];
-        out_physical[static_cast<size_t>(g) * max_sel + before] =
-            (phys >= 0 && phys < num_pool_pages) ? phys : 0;
+        out_p[before] = (phys >= 0 && phys < num_pool_pages) ? phys : 0;
       }
     }
     __syncthreads();
@@ -270,7 +331,68 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
     }
     __syncthreads();
   }
-  if (t == 0) out_count[g] = min(running_sh, max_sel);
+  if (t == 0) out_count[row] = min(running_sh, max_sel);
+}
+
+// Workspace: partials [problems][splits <= 128][Hkv][d] fp32, then keys
+// [problems][Hkv][max(max_past, 1)] u64.
+size_t workspace_bytes_for(int64_t problems, int Hkv, int D, int max_past) {
+  const size_t partial = static_cast<size_t>(problems) * kSplits * Hkv * D * 4;
+  const size_t keys = static_cast<size_t>(problems) * Hkv * (max_past > 0 ? max_past : 1) * 8;
+  return align256(partial) + align256(keys);
+}
+
+// Launches the three kernels for `n_problems` problems on `s`.
+oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
+                        const Problems& pb_in, int n_problems, const int32_t* d_page_table,
+                        int top_k, int n_recent, int32_t* d_out_logical, int32_t* d_out_physical,
+                        int32_t* d_out_count, float* d_out_scores, void* scratch,
+                        cudaStream_t s) {
+  const oomb_pool_desc& d = pool->desc;
+  const int Hkv = d.num_kv_heads, D = d.head_dim, G = num_q_heads / Hkv;
+  Problems pb = pb_in;
+  pb.status = pool->d_status;
+  float* partial = static_cast<float*>(scratch);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(
+      static_cast<uint8_t*>(scratch) +
+      align256(static_cast<size_t>(n_problems) * kSplits * Hkv * D * 4));
+  const auto* q = static_cast<const __nv_bfloat16*>(d_q);
+  dim3 g1(pb.splits, Hkv, n_problems);
+  dim3 g2((pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv, n_problems);
+  if (D == 128) {
+    qmean_partial_kernel<128><<<g1, kMeanThreads, 0, s>>>(q, partial, pb, num_q_heads, G);
+    if (pb.max_past > 0)
+      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
+                                                          pb, Hkv, G, d.num_pages, keys,
+                                                          d_out_scores);
+  } else {
+    qmean_partial_kernel<64><<<g1, kMeanThreads, 0, s>>>(q, partial, pb, num_q_heads, G);
+    if (pb.max_past > 0)
+      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
+                                                         pb, Hkv, G, d.num_pages, keys,
+                                                         d_out_scores);
+  }
+  topk_select_kernel<<<dim3(Hkv, n_problems), kSelectThreads, 0, s>>>(
+      keys, d_page_table, pb, top_k, n_recent, d.num_pages, d_out_logical, d_out_physical,
+      d_out_count);
+  return oomb::check_launch();
+}
+
+// Host-side checks shared by the entry points.
+oomb_status check_topk_args(const oomb_pool* pool, const void* d_q, int num_q_heads,
+                            const int32_t* d_page_table, int max_past, int top_k, int n_recent,
+                            const int32_t* d_out_logical, const int32_t* d_out_count) {
+  // device pools and pinned-host pools (whose summaries live on the device)
+  if (!pool || pool->desc.location == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
+  const int Hkv = pool->desc.num_kv_heads;
+  if (!d_q || !d_out_logical || !d_out_count) return OOMB_ERR_INVALID_ARG;
+  if (num_q_heads <= 0 || num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
+  if (max_past < 0 || max_past > 65536 || top_k < 0 || n_recent < 0 ||
+      top_k + n_recent > 4096 || top_k + n_recent == 0)
+    return OOMB_ERR_INVALID_ARG;
+  if (max_past > 0 && !d_page_table) return OOMB_ERR_INVALID_ARG;
+  if (!oomb::aligned16(d_q)) return OOMB_ERR_INVALID_ARG;
+  return OOMB_OK;
 }
 
 }  // namespace
@@ -280,9 +402,7 @@ extern "C" size_t oomb_page_topk_workspace_size(int32_t chunk_len, int32_t num_q
                                                 int32_t n_past) {
   (void)num_q_heads;
   if (chunk_len <= 0 || num_kv_heads <= 0 || head_dim <= 0 || n_past < 0) return 0;
-  const size_t partial = static_cast<size_t>(kSplits) * num_kv_heads * head_dim * 4;
-  const size_t keys = static_cast<size_t>(num_kv_heads) * (n_past > 0 ? n_past : 1) * 8;
-  return align256(partial) + align256(keys);
+  return workspace_bytes_for(1, num_kv_heads, head_dim, n_past);
 }
 
 extern "C" oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk_len,
@@ -291,45 +411,49 @@ extern "C" oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, in
                                       int32_t* d_out_logical, int32_t* d_out_physical,
                                       int32_t* d_out_count, float* d_out_scores,
                                       void* d_workspace, size_t workspace_bytes, void* stream) {
-  // device pools and pinned-host pools (whose summaries live on the device)
-  if (!pool || pool->desc.location == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
+  oomb_status st = check_topk_args(pool, d_q, num_q_heads, d_page_table, n_past, top_k, n_recent,
+                                   d_out_logical, d_out_count);
+  if (st != OOMB_OK) return st;
+  if (chunk_len <= 0 || !d_workspace || !oomb::aligned16(d_workspace)) return OOMB_ERR_INVALID_ARG;
   const oomb_pool_desc& d = pool->desc;
-  const int Hkv = d.num_kv_heads, D = d.head_dim;
-  if (!d_q || !d_out_logical || !d_out_count || !d_workspace) return OOMB_ERR_INVALID_ARG;
-  if (chunk_len <= 0 || num_q_heads <= 0 || num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
-  if (n_past < 0 || n_past > 65536 || top_k < 0 || n_recent < 0 || top_k + n_recent > 4096 ||
-      top_k + n_recent == 0)
-    return OOMB_ERR_INVALID_ARG;
-  if (n_past > 0 && !d_page_table) return OOMB_ERR_INVALID_ARG;
-  if (!oomb::aligned16(d_q) || !oomb::aligned16(d_workspace)) return OOMB_ERR_INVALID_ARG;
-  if (workspace_bytes < oomb_page_topk_workspace_size(chunk_len, num_q_heads, Hkv, D, n_past))
+  if (workspace_bytes < workspace_bytes_for(1, d.num_kv_heads, d.head_dim, n_past))
     return OOMB_ERR_INVALID_ARG;
   oomb::DeviceGuard guard(d.device);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* partial = static_cast<float*>(d_workspace);
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(
-      static_cast<uint8_t*>(d_workspace) + align256(static_cast<size_t>(kSplits) * Hkv * D * 4));
-  const int G = num_q_heads / Hkv;
-  const float inv_rows = 1.0f / (static_cast<float>(chunk_len) * static_cast<float>(G));
-  const auto* q = static_cast<const __nv_bfloat16*>(d_q);
-  dim3 g1(kSplits, Hkv), g2((n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv);
-  if (D == 128) {
-    qmean_partial_kernel<128><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
-    if (n_past > 0)
-      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
-                                                          n_past, Hkv, d.num_pages, inv_rows,
-                                                          keys, d_out_scores, pool->d_status);
-  } else {
-    qmean_partial_kernel<64><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
-    if (n_past > 0)
-      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
-                                                         n_past, Hkv, d.num_pages, inv_rows, keys,
-                                                         d_out_scores, pool->d_status);
-  }
-  topk_select_kernel<<<Hkv, kSelectThreads, 0, s>>>(keys, d_page_table, n_past, top_k, n_recent,
-                                                     d.num_pages, d_out_logical, d_out_physical,
-                                                     d_out_count);
-  return oomb::check_launch();
+  const Problems pb{nullptr, nullptr, chunk_len, n_past, n_past, chunk_len,
+                    choose_splits(chunk_len), nullptr};
+  return launch_topk(pool, d_q, num_q_heads, pb, 1, d_page_table, top_k, n_recent, d_out_logical,
+                     d_out_physical, d_out_count, d_out_scores, d_workspace,
+                     static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t oomb_page_topk_batched_workspace_size(int32_t n_problems, int32_t num_kv_heads,
+                                                        int32_t head_dim, int32_t max_past) {
+  if (n_problems <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_past < 0) return 0;
+  return workspace_bytes_for(n_problems, num_kv_heads, head_dim, max_past);
+}
+
+extern "C" oomb_status oomb_page_topk_batched(
+    const oomb_pool* pool, const void* d_q, int32_t num_rows, int32_t num_q_heads,
+    int32_t n_problems, const int32_t* d_row_start, int32_t max_rows, const int32_t* d_n_past,
+    int32_t max_past, const int32_t* d_page_table, int32_t top_k, int32_t n_recent,
+    int32_t* d_out_logical, int32_t* d_out_physical, int32_t* d_out_count, float* d_out_scores,
+    void* d_workspace, size_t workspace_bytes, void* stream) {
+  oomb_status st = check_topk_args(pool, d_q, num_q_heads, d_page_table, max_past, top_k,
+                                   n_recent, d_out_logical, d_out_count);
+  if (st != OOMB_OK) return st;
+  if (n_problems <= 0 || n_problems > 65535 || num_rows <= 0 || max_rows <= 0 ||
+      max_rows > num_rows || !d_row_start || !d_n_past || !d_workspace ||
+      !oomb::aligned16(d_workspace))
+    return OOMB_ERR_INVALID_ARG;
+  const oomb_pool_desc& d = pool->desc;
+  if (workspace_bytes < workspace_bytes_for(n_problems, d.num_kv_heads, d.head_dim, max_past))
+    return OOMB_ERR_INVALID_ARG;
+  oomb::DeviceGuard guard(d.device);
+  const Problems pb{d_row_start, d_n_past, 0, 0, max_past, num_rows, choose_splits(max_rows),
+                    nullptr};
+  return launch_topk(pool, d_q, num_q_heads, pb, n_problems, d_page_table, top_k, n_recent,
+                     d_out_logical, d_out_physical, d_out_count, d_out_scores, d_workspace,
+                     static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- no-allocation variant
@@ -377,47 +501,21 @@ extern "C" oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* 
                                              int32_t* d_out_logical, int32_t* d_out_physical,
                                              int32_t* d_out_count, float* d_out_scores,
                                              void* stream) {
-  if (!pool || pool->desc.location == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
+  oomb_status st = check_topk_args(pool, d_q, num_q_heads, d_page_table, n_past, top_k, n_recent,
+                                   d_out_logical, d_out_count);
+  if (st != OOMB_OK) return st;
+  if (chunk_len <= 0) return OOMB_ERR_INVALID_ARG;
   const oomb_pool_desc& d = pool->desc;
-  const int Hkv = d.num_kv_heads, D = d.head_dim;
-  if (!d_q || !d_out_logical || !d_out_count) return OOMB_ERR_INVALID_ARG;
-  if (chunk_len <= 0 || num_q_heads <= 0 || num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
-  if (n_past < 0 || n_past > 65536 || top_k < 0 || n_recent < 0 || top_k + n_recent > 4096 ||
-      top_k + n_recent == 0)
-    return OOMB_ERR_INVALID_ARG;
-  if (n_past > 0 && !d_page_table) return OOMB_ERR_INVALID_ARG;
-  if (!oomb::aligned16(d_q)) return OOMB_ERR_INVALID_ARG;
   // the scratch array has a fixed size: larger problems must use oomb_page_topk
-  if (oomb_page_topk_workspace_size(chunk_len, num_q_heads, Hkv, D, n_past) >
-      OOMB_TOPK_STATIC_SCRATCH_BYTES)
+  if (workspace_bytes_for(1, d.num_kv_heads, d.head_dim, n_past) > OOMB_TOPK_STATIC_SCRATCH_BYTES)
     return OOMB_ERR_UNSUPPORTED;
   oomb::DeviceGuard guard(d.device);
   void* scratch = nullptr;
-  const oomb_status st = static_scratch(d.device, &scratch);
+  st = static_scratch(d.device, &scratch);
   if (st != OOMB_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* partial = static_cast<float*>(scratch);
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(
-      static_cast<uint8_t*>(scratch) + align256(static_cast<size_t>(kSplits) * Hkv * D * 4));
-  const int G = num_q_heads / Hkv;
-  const float inv_rows = 1.0f / (static_cast<float>(chunk_len) * static_cast<float>(G));
-  const auto* q = static_cast<const __nv_bfloat16*>(d_q);
-  dim3 g1(kSplits, Hkv), g2((n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv);
-  if (D == 128) {
-    qmean_partial_kernel<128><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
-    if (n_past > 0)
-      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
-                                                          n_past, Hkv, d.num_pages, inv_rows,
-                                                          keys, d_out_scores, pool->d_status);
-  } else {
-    qmean_partial_kernel<64><<<g1, kMeanThreads, 0, s>>>(q, partial, chunk_len, num_q_heads, G);
-    if (n_past > 0)
-      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
-                                                         n_past, Hkv, d.num_pages, inv_rows, keys,
-                                                         d_out_scores, pool->d_status);
-  }
-  topk_select_kernel<<<Hkv, kSelectThreads, 0, s>>>(keys, d_page_table, n_past, top_k, n_recent,
-                                                     d.num_pages, d_out_logical, d_out_physical,
-                                                     d_out_count);
-  return oomb::check_launch();
+  const Problems pb{nullptr, nullptr, chunk_len, n_past, n_past, chunk_len,
+                    choose_splits(chunk_len), nullptr};
+  return launch_topk(pool, d_q, num_q_heads, pb, 1, d_page_table, top_k, n_recent, d_out_logical,
+                     d_out_physical, d_out_count, d_out_scores, scratch,
+                     static_cast<cudaStream_t>(stream));
 }
