@@ -10,7 +10,10 @@ pool, dQ).  The headline value is the dense run's algorithmic TFLOP/s; the
 same line carries the Top-K sparse run (Top-64 + 2 recent pages per chunk and
 KV-head group, Top-K selection included in the timed step), tokens/s for
 both, an end-to-end figure with host buffers, the roofline of the dominant
-kernel and the CPU oracle's throughput on a bounded sample.
+kernel, the 1M-token offloaded Top-K run (KV and gradients in pinned host
+memory), the memory-bound kernels in batched launches (append, Top-K, block
+gather and gradient scatter-add, over HBM and over the host link) and the CPU
+oracle's throughput on a bounded sample.
 
 Inputs are synthetic (seeded), drawn on the device before timing; the
 working set (Q, dO, KV pool, gradient pool) is far larger than L2.  Under
@@ -691,6 +694,15 @@ def main():
     value = whole_job_rate(step_flops, ms, world) / 1e12
     tokens = whole_job_rate(w.context, ms, world)
     kernel_flops = {k: sum(v) for k, v in dense.flops.items()}
+    kt_serial = None
+    if dense.concurrent_bwd:
+        # one more step, untimed as a whole, in the serial schedule: per-kernel
+        # event times without co-scheduled launches of the other stream
+        dense.concurrent_bwd = False
+        timers = {}
+        dense.step(timers)
+        torch.cuda.synchronize()
+        kt_serial = {n: sum(x.elapsed_time(y) for x, y in ev) for n, ev in timers.items()}
     dense.close()
     del dense
     torch.cuda.empty_cache()
@@ -799,6 +811,9 @@ def main():
                    "l2": "inputs larger than L2 (Q+dO 3.5 GiB, KV pool 512 MiB, grad pool 1 GiB)"},
         "tokens_per_s": tokens,
         "kernels": kernels,
+        "kernels_serial_step": None if kt_serial is None else {
+            k: {"ms_per_step": v, "tflops": (kernel_flops[k] / (v / 1e3) / 1e12)
+                if k in kernel_flops else None} for k, v in kt_serial.items()},
         "roofline": roof,
         "sparse": sparse_obj,
         "offload": offload_obj,
