@@ -615,8 +615,14 @@ def _traffic(kernel):
     e = d.get(kernel)
     if not e:
         return None
-    src = os.path.join(ROOT, e["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != e["sha256"]:
+    # the kernel's source and the headers it includes, hashed in order
+    h = hashlib.sha256()
+    for rel in e.get("sources", [e.get("source")]):
+        src = os.path.join(ROOT, rel) if rel else ""
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    if h.hexdigest() != e["sha256"]:
         return None
     return e
 
