@@ -86,3 +86,13 @@ def topk_for_chunk(q_chunk, k_past_tokens, page_size, top_k, n_recent):
     q_bar = group_query_means(q_chunk, k_bar.shape[1])
     s = page_scores(q_bar, k_bar)
     return select_pages(s, n_past, top_k, n_recent), s
+
+
+def local_pages(n_past, window, num_kv_heads):
+    """Recent-only page lists: layers that are sparse by construction attend
+    to the most recent pages ([it] §2D) — here the last ``window`` of the
+    ``n_past`` past pages, ascending, the same list for every group (plus,
+    as always, the chunk itself causally)."""
+    lo = max(0, n_past - window)
+    return [list(range(lo, n_past)) for _ in range(num_kv_heads)]
+

@@ -6,8 +6,9 @@ import numpy as np
 import pytest
 
 from oracle.pool import PoolModel, SplitMix64, initial_order
-from oracle.sparse import (group_query_means, kth_score, page_key_means, page_scores,
-                           select_pages, topk_for_chunk)
+from oracle.recurrent import run_sequence
+from oracle.sparse import (group_query_means, kth_score, local_pages, page_key_means,
+                           page_scores, select_pages, topk_for_chunk)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -112,3 +113,37 @@ def test_kth_score():
     s = np.array([0.5, 0.1, 0.9, 0.3, 0.7, 0.2])
     assert kth_score(s, 6, 2, 2) == 0.5      # candidates 0..3 sorted: .9 .5 .3 .1
     assert kth_score(s, 6, 4, 2) is None
+
+
+@pytest.mark.parametrize("n_past,W", [(0, 4), (3, 4), (4, 4), (10, 4), (10, 1), (200, 64)])
+def test_local_pages_are_the_last_window_pages(n_past, W):
+    got = local_pages(n_past, W, 3)
+    brute = [p for p in range(n_past) if n_past - p <= W]
+    assert got == [brute] * 3
+    assert len(got[0]) == min(W, n_past)
+    # the same rule as Top-K's forced recent pages with no Top-K candidates kept
+    s = np.zeros((3, max(n_past, 1)))
+    assert got == select_pages(s, n_past, 0, W)
+
+
+def test_local_window_covering_the_past_is_dense():
+    rng = np.random.default_rng(9)
+    L, C, P, Hq, Hkv, d = 64, 16, 4, 4, 2, 8
+    q, do = rng.standard_normal((L, Hq, d)), rng.standard_normal((L, Hq, d))
+    k, v = rng.standard_normal((L, Hkv, d)), rng.standard_normal((L, Hkv, d))
+    dense = run_sequence(q, k, v, do, C, P, 0.35)
+    sels = [local_pages(c * C // P, L // P, Hkv) for c in range(L // C)]
+    local = run_sequence(q, k, v, do, C, P, 0.35, selections=sels)
+    for key in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_allclose(local[key], dense[key], rtol=1e-12, atol=1e-12)
+    # a window of one page: rows see only the last past page and the chunk
+    sels1 = [local_pages(c * C // P, 1, Hkv) for c in range(L // C)]
+    one = run_sequence(q, k, v, do, C, P, 0.35, selections=sels1, with_backward=False)
+    from oracle.attention import chunk_forward
+    c = 2
+    a = c * C
+    kp = [k[a - P:a, g] for g in range(Hkv)]
+    vp = [v[a - P:a, g] for g in range(Hkv)]
+    o_c, _ = chunk_forward(q[a:a + C], kp, vp, k[a:a + C], v[a:a + C], 0.35)
+    np.testing.assert_allclose(one["o"][a:a + C], o_c, rtol=1e-12, atol=1e-12)
+
