@@ -153,6 +153,11 @@ class Run:
         self.dense_past = [None] + [pt[:c * ppc].repeat(Hkv, 1).contiguous() for c in range(1, N)]
         self.dense_cnt = [None] + [torch.full((Hkv,), c * ppc, dtype=torch.int32, device=device)
                                    for c in range(1, N)]
+        self.local = w.window > 0
+        if self.local:
+            self.loc_p = [torch.zeros((Hkv, w.window), dtype=torch.int32, device=device)
+                          for _ in range(N)]
+            self.loc_n = [torch.zeros((Hkv,), dtype=torch.int32, device=device) for _ in range(N)]
         if sparse:
             ms = w.top_k + w.n_recent
             self.sel_l = [torch.zeros((Hkv, ms), dtype=torch.int32, device=device) for _ in range(N)]
@@ -165,6 +170,8 @@ class Run:
         for c in range(N):
             if sparse and c:
                 n_keys = (min(w.top_k, max(0, c * ppc - w.n_recent)) + min(w.n_recent, c * ppc)) * P
+            elif self.local:
+                n_keys = min(w.window, c * ppc) * P
             else:
                 n_keys = c * C
             pairs = pairs_of_chunk(C, n_keys) * Hq
@@ -172,7 +179,10 @@ class Run:
             self.flops["dkdv"].append(8.0 * pairs * d)
             self.flops["dq"].append(2.0 * pairs * d)
         self.step_flops = sum(sum(v) for v in self.flops.values())
-        self.launches_per_step = N * 5 + ((N - 1) * 2 if sparse else 0)
+        # per chunk: append, forward, preprocess, dK/dV, dQ; Top-K adds query
+        # mean, page scores and select per chunk with a past; local lists one
+        self.launches_per_step = N * 5 + ((N - 1) * 3 if sparse else 0) + \
+            ((N - 1) if self.local else 0)
 
     def step(self, timers=None):
         """One pass over all chunks.  With concurrent_bwd, chunk c's dQ launch
@@ -205,6 +215,12 @@ class Run:
                                                      stream))
             if c == 0:
                 past, cnt = None, None
+            elif self.local:
+                n_past = c * ppc
+                timed("lists", lambda: pk.local_pages(self.pool, self.page_table_dev[:n_past],
+                                                      n_past, self.loc_p[c], self.loc_n[c],
+                                                      stream=stream))
+                past, cnt = self.loc_p[c], self.loc_n[c]
             elif self.sparse:
                 n_past = c * ppc
                 timed("topk", lambda: pk.page_topk(
@@ -641,6 +657,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-offload", action="store_true")
     ap.add_argument("--no-hbm", action="store_true", help="skip the batched HBM/host-link kernels")
+    ap.add_argument("--no-local", action="store_true", help="skip the recent-only page-list run")
+    ap.add_argument("--local-workload", default="qwen256k_local")
     ap.add_argument("--serial-bwd", action="store_true",
                     help="run each chunk's dQ launch after its dK/dV launch on one stream")
     ap.add_argument("--offload-workload", default="qwen1m_topk_offload")
@@ -697,6 +715,7 @@ def main():
     clk = clocks.stop()
     dense_status = pk.get_device_status(dense.pool)
     step_flops = dense.step_flops
+    launches_dense = dense.launches_per_step
     value = whole_job_rate(step_flops, ms, world) / 1e12
     tokens = whole_job_rate(w.context, ms, world)
     kernel_flops = {k: sum(v) for k, v in dense.flops.items()}
@@ -769,6 +788,21 @@ def main():
         del sp
         torch.cuda.empty_cache()
 
+    local_obj = None
+    if not a.no_local:
+        wl = synth.WORKLOADS[a.local_workload]
+        lr = Run(wl, False, device)
+        lr.concurrent_bwd = not a.serial_bwd
+        ms_l, kt_l = time_steps(lr, a.steps, a.warmup, dist_on, device)
+        local_obj = {"workload": wl.name, "window_pages": wl.window,
+                     "value": lr.step_flops * world / (ms_l / 1e3) / 1e12, "unit": "TFLOP/s",
+                     "ms_per_step": ms_l, "tokens_per_s": wl.context * world / (ms_l / 1e3),
+                     "kernels": {k: {"ms_per_step": v} for k, v in kt_l.items()},
+                     "device_status": pk.get_device_status(lr.pool)}
+        lr.close()
+        del lr
+        torch.cuda.empty_cache()
+
     offload_obj = None
     if not a.no_offload:
         offload_obj = offload_run(synth.WORKLOADS[a.offload_workload], max(1, min(a.steps, 2)),
@@ -822,11 +856,12 @@ def main():
                 if k in kernel_flops else None} for k, v in kt_serial.items()},
         "roofline": roof,
         "sparse": sparse_obj,
+        "local": local_obj,
         "offload": offload_obj,
         "hbm_kernels": hbm_obj,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "gpu_launches": w.num_chunks * 5 * a.steps
+        "gpu_launches": launches_dense * a.steps
         + ((w.num_chunks * 5 + (w.num_chunks - 1) * 2) * a.steps if sparse_obj else 0),
         "clocks": clk,
         "device_status": dense_status,

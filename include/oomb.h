@@ -233,6 +233,21 @@ oomb_status oomb_page_topk_batched(const oomb_pool* pool, const void* d_q, int32
                                    int32_t* d_out_count, float* d_out_scores, void* d_workspace,
                                    size_t workspace_bytes, void* stream);
 
+/* Recent-only page lists ([it] §2D: layers that are sparse by construction
+ * keep the most recent pages): for every KV-head group, the last `window` of
+ * the first n_past logical pages of d_page_table, ascending, as physical ids
+ * — the past-page arguments of oomb_chunk_attn_fwd / _bwd for attention over
+ * a sliding window of pages plus the chunk itself (causal).
+ *   d_page_table [>= n_past] device int32, logical -> physical page of `pool`
+ *   d_out_pages  [num_kv_heads][window] device int32 (row stride = window;
+ *                entries past the count are 0)
+ *   d_out_count  [num_kv_heads] device int32: min(window, n_past)
+ * window >= 1.  Ids outside the pool are written as 0 and set bit 0 of the
+ * device status word. */
+oomb_status oomb_local_pages(const oomb_pool* pool, const int32_t* d_page_table, int32_t n_past,
+                             int32_t window, int32_t* d_out_pages, int32_t* d_out_count,
+                             void* stream);
+
 /* ---------------------------------------------------------------- offload
  * A block is the K and V of one page and one KV head: block id = page *
  * num_kv_heads + head, contiguous in both pools ([pt] §2D, [it] §2C: KV and

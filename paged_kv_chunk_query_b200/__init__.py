@@ -10,7 +10,7 @@ compute runs in hand-written CUDA kernels inside ``liboomb.so`` (C ABI in
 from . import _lib
 from ._lib import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, LOC_DEVICE, LOC_HOST, LOC_PINNED_HOST,
                    OombError, block_copy, chunk_attn_bwd, chunk_attn_fwd, get_device_status,
-                   grad_block_add, grad_writeback, grad_writeback_sync, kv_append, page_prefetch,
+                   grad_block_add, grad_writeback, grad_writeback_sync, kv_append, local_pages, page_prefetch,
                    page_topk, page_topk_batched, page_topk_batched_workspace_size,
                    page_topk_workspace_size, pool_alloc_page, pool_buffers, pool_create,
                    pool_destroy, pool_free_page, pool_get_desc, pool_num_free, pool_views,
@@ -22,7 +22,7 @@ __all__ = [
     "pool_num_free", "pool_buffers", "pool_get_desc", "pool_views", "kv_append",
     "chunk_attn_fwd", "chunk_attn_bwd", "page_topk", "page_topk_workspace_size",
     "page_topk_batched", "page_topk_batched_workspace_size", "page_prefetch", "grad_writeback",
-    "grad_writeback_sync", "block_copy", "grad_block_add", "prefetch_lists", "wait",
+    "grad_writeback_sync", "local_pages", "block_copy", "grad_block_add", "prefetch_lists", "wait",
     "get_device_status", "status_string", "version",
     "LOC_DEVICE", "LOC_PINNED_HOST", "LOC_HOST", "BWD_PREPROCESS", "BWD_DKDV", "BWD_DQ",
     "WORKLOADS", "Workload",

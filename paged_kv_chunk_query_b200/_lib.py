@@ -36,7 +36,7 @@ EXPORTS = (
     "oomb_grad_writeback", "oomb_wait", "oomb_get_device_status", "oomb_status_string",
     "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
     "oomb_selftest_wait_limit", "oomb_page_topk_batched_workspace_size", "oomb_page_topk_batched",
-    "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists",
+    "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists", "oomb_local_pages",
 )
 
 
@@ -100,6 +100,7 @@ def load() -> ctypes.CDLL:
         "oomb_block_copy": [vp, vp, vp, vp, i32, vp],
         "oomb_grad_block_add": [vp, vp, vp, vp, i32, i32, vp],
         "oomb_prefetch_lists": [vp, vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp],
+        "oomb_local_pages": [vp, vp, i32, i32, vp, vp, vp],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):  # completeness is checked by the export test
@@ -333,6 +334,16 @@ def page_topk_batched(pool, q, row_start, max_rows, n_past, max_past, page_table
         _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
         _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "oomb_page_topk_batched")
+
+
+def local_pages(pool, page_table, n_past, out_pages, out_count, stream=None):
+    """oomb_local_pages: the last window = out_pages.shape[1] past pages of every
+    group (physical ids, ascending) and their counts."""
+    window = out_pages.shape[1]
+    _check(load().oomb_local_pages(
+        pool, _dev_tensor(page_table, torch.int32, "page_table") if n_past else None, n_past,
+        window, _dev_tensor(out_pages, torch.int32, "out_pages"),
+        _dev_tensor(out_count, torch.int32, "out_count"), _stream(stream)), "oomb_local_pages")
 
 
 TOPK_STATIC_SCRATCH_BYTES = 1 << 20

@@ -456,6 +456,49 @@ extern "C" oomb_status oomb_page_topk_batched(
                      static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------- recent-only lists
+// Layers that are sparse by construction attend to the most recent pages
+// ([it] §2D): group g's list is the last `window` of the n_past logical pages,
+// ascending, mapped to physical ids.  One thread per (group, slot).
+namespace {
+
+__global__ void local_pages_kernel(const int32_t* __restrict__ page_table, int n_past, int window,
+                                   int Hkv, int num_pool_pages, int32_t* __restrict__ out_pages,
+                                   int32_t* __restrict__ out_count, uint32_t* status) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= Hkv * window) return;
+  const int g = e / window, i = e % window;
+  const int n = min(window, n_past), lo = n_past - n;
+  int id = 0;
+  if (i < n) {
+    id = page_table[lo + i];
+    if (id < 0 || id >= num_pool_pages) {
+      atomicOr(status, OOMB_DEV_BAD_PAGE);
+      id = 0;
+    }
+  }
+  out_pages[static_cast<size_t>(g) * window + i] = id;
+  if (i == 0) out_count[g] = n;
+}
+
+}  // namespace
+
+extern "C" oomb_status oomb_local_pages(const oomb_pool* pool, const int32_t* d_page_table,
+                                        int32_t n_past, int32_t window, int32_t* d_out_pages,
+                                        int32_t* d_out_count, void* stream) {
+  if (!pool || pool->desc.location == OOMB_LOC_HOST || !d_out_pages || !d_out_count)
+    return OOMB_ERR_INVALID_ARG;
+  if (n_past < 0 || window <= 0 || (n_past > 0 && !d_page_table)) return OOMB_ERR_INVALID_ARG;
+  const int Hkv = pool->desc.num_kv_heads;
+  if (static_cast<int64_t>(window) * Hkv > (1 << 26)) return OOMB_ERR_UNSUPPORTED;
+  oomb::DeviceGuard guard(pool->desc.device);
+  const int n = window * Hkv;
+  local_pages_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      d_page_table, n_past, window, Hkv, pool->desc.num_pages, d_out_pages, d_out_count,
+      pool->d_status);
+  return oomb::check_launch();
+}
+
 // ---------------------------------------------------------------- no-allocation variant
 // Some callers of this library cannot allocate device memory: a host
 // framework that owns every device allocation and forbids side allocations,

@@ -46,6 +46,7 @@ class Workload:
     top_k: int = 0                # 0: dense
     n_recent: int = 0
     host_resident: bool = False   # past KV and grads in pinned host memory
+    window: int = 0               # > 0: recent-only lists of this many past pages
 
     @property
     def group_size(self) -> int:
@@ -86,6 +87,9 @@ WORKLOADS = {
     "qwen256k_topk": Workload("qwen256k_topk", 28, 4, 128, 64, 4096, 64, seed=1003,
                               shuffle_pages=True, page_direction=0.5, top_k=64,
                               n_recent=2),
+    # recent-only page lists: the last 64 past pages (4096 tokens) + the chunk
+    "qwen256k_local": Workload("qwen256k_local", 28, 4, 128, 64, 4096, 64, seed=1006,
+                               shuffle_pages=True, window=64),
     "qwen1m_topk_offload": Workload("qwen1m_topk_offload", 28, 4, 128, 64, 4096, 256,
                                     seed=1004, shuffle_pages=True, page_direction=0.5,
                                     top_k=64, n_recent=2, host_resident=True),
