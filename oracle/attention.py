@@ -157,6 +157,86 @@ def chunk_backward(q, k_past, v_past, k_cur, v_cur, do, scale):
     return dq, dk_past, dv_past, dk_cur, dv_cur
 
 
+def _block_logits(qh, row0, kp, kc, scale):
+    """Logits of one head's row block (chunk rows row0 .. row0 + T - 1) against
+    [its past keys | the chunk's keys 0 .. row0 + T - 1], causal on the latter."""
+    T = qh.shape[0]
+    kc = kc[: row0 + T]
+    s_past = scale * (qh @ kp.T)
+    s_cur = scale * (qh @ kc.T)
+    keep = np.arange(row0 + T)[None, :] <= (row0 + np.arange(T))[:, None]
+    s_cur = np.where(keep, s_cur, -np.inf)
+    return np.concatenate([s_past, s_cur], axis=1)
+
+
+def chunk_forward_blocks(q, block_rows, k_past, v_past, k_cur, v_cur, scale):
+    """Forward of one chunk whose rows come in blocks of ``block_rows`` with a
+    key set each: the pages relevant to each query page ([pt] §2C).
+
+    ``k_past[b][g]``, ``v_past[b][g]`` ``[n_bg][d]`` are the past keys group g
+    attends to from rows of block b; the chunk's own keys are causal as in
+    :func:`chunk_forward`.  Returns O ``[C][Hq][d]`` and LSE ``[Hq][C]``."""
+    q, k_cur, v_cur = _f64(q), _f64(k_cur), _f64(v_cur)
+    C, Hq, d = q.shape
+    Hkv = k_cur.shape[1]
+    G = Hq // Hkv
+    dv_dim = v_cur.shape[2]
+    o = np.zeros((C, Hq, dv_dim))
+    lse = np.zeros((Hq, C))
+    for b in range((C + block_rows - 1) // block_rows):
+        r0, r1 = b * block_rows, min(C, (b + 1) * block_rows)
+        for h in range(Hq):
+            g = h // G
+            kp = _f64(k_past[b][g]).reshape(-1, d)
+            vp = _f64(v_past[b][g]).reshape(-1, dv_dim)
+            s = _block_logits(q[r0:r1, h, :], r0, kp, k_cur[:, g, :], scale)
+            pm, lse[h, r0:r1] = _softmax_rows(s)
+            o[r0:r1, h, :] = pm @ np.concatenate([vp, v_cur[:r1, g, :]], axis=0)
+    return o, lse
+
+
+def chunk_backward_blocks(q, block_rows, k_past, v_past, k_cur, v_cur, do, scale):
+    """Backward of :func:`chunk_forward_blocks` for the loss sum(O * dO).
+
+    Returns dq, dk_past / dv_past (``[b][g]`` lists: block b's contribution to
+    its own past key set) and dk_cur / dv_cur ``[C][Hkv][d]``."""
+    q, k_cur, v_cur, do = _f64(q), _f64(k_cur), _f64(v_cur), _f64(do)
+    C, Hq, d = q.shape
+    Hkv = k_cur.shape[1]
+    G = Hq // Hkv
+    dv_dim = v_cur.shape[2]
+    nb = (C + block_rows - 1) // block_rows
+    dq = np.zeros_like(q)
+    dk_cur, dv_cur = np.zeros_like(k_cur), np.zeros_like(v_cur)
+    dk_past = [[np.zeros((np.asarray(k_past[b][g]).reshape(-1, d).shape[0], d))
+                for g in range(Hkv)] for b in range(nb)]
+    dv_past = [[np.zeros((np.asarray(v_past[b][g]).reshape(-1, dv_dim).shape[0], dv_dim))
+                for g in range(Hkv)] for b in range(nb)]
+    for b in range(nb):
+        r0, r1 = b * block_rows, min(C, (b + 1) * block_rows)
+        for h in range(Hq):
+            g = h // G
+            kp = _f64(k_past[b][g]).reshape(-1, d)
+            vp = _f64(v_past[b][g]).reshape(-1, dv_dim)
+            n = kp.shape[0]
+            kk = np.concatenate([kp, k_cur[:r1, g, :]], axis=0)
+            vv = np.concatenate([vp, v_cur[:r1, g, :]], axis=0)
+            s = _block_logits(q[r0:r1, h, :], r0, kp, k_cur[:, g, :], scale)
+            pm, _ = _softmax_rows(s)
+            o = pm @ vv
+            D = np.sum(do[r0:r1, h, :] * o, axis=1)
+            dp = do[r0:r1, h, :] @ vv.T
+            ds = pm * (dp - D[:, None])
+            dq[r0:r1, h, :] = scale * (ds @ kk)
+            dkk = scale * (ds.T @ q[r0:r1, h, :])
+            dvv = pm.T @ do[r0:r1, h, :]
+            dk_past[b][g] += dkk[:n]
+            dv_past[b][g] += dvv[:n]
+            dk_cur[:r1, g, :] += dkk[n:]
+            dv_cur[:r1, g, :] += dvv[n:]
+    return dq, dk_past, dv_past, dk_cur, dv_cur
+
+
 def chunk_rows_forward(q_rows, row_pos, k_keys, v_keys, key_pos, scale):
     """Forward for a few sampled rows of ONE head, used at sizes where a whole
     chunk is too slow in fp64.

@@ -10,7 +10,8 @@ import torch
 
 from oracle.attention import (causal_attention, causal_attention_backward,
                               chunk_backward, chunk_forward, chunk_rows_forward)
-from oracle.recurrent import run_sequence
+from oracle.recurrent import run_sequence, run_sequence_blocks
+from oracle.sparse import topk_for_chunk
 
 
 def _rand(shape, seed, scale=1.0):
@@ -224,3 +225,74 @@ def test_sampled_rows_match_full_chunk():
     o_s, lse_s = chunk_rows_forward(q[rows, 1], rows, k[:, 0], v[:, 0], np.arange(L), 0.3)
     np.testing.assert_allclose(o_s, o[rows, 1], rtol=1e-13)
     np.testing.assert_allclose(lse_s, lse[1, rows], rtol=1e-13)
+
+
+def _block_selections(L, C, P, Hkv, T, seed):
+    rng = np.random.default_rng(seed)
+    sels = []
+    for c in range(L // C):
+        n_past = c * C // P
+        sels.append([[sorted(rng.choice(n_past, size=int(rng.integers(0, n_past + 1)),
+                                        replace=False).tolist()) if n_past else []
+                      for _ in range(Hkv)] for _ in range((C + T - 1) // T)])
+    return sels
+
+
+@pytest.mark.parametrize("T", [8, 6])
+def test_row_block_selections_match_torch_masked_attention_and_autograd(T):
+    """Per-row-block key sets against a whole-sequence masked softmax in torch
+    (fp64) and its autograd gradients; T = 6 leaves a ragged last block."""
+    L, C, P, Hq, Hkv, d, scale = 48, 16, 4, 4, 2, 8, 0.3
+    q, k, v, do = (_rand((L, Hq, d), 131), _rand((L, Hkv, d), 132), _rand((L, Hkv, d), 133),
+                   _rand((L, Hq, d), 134))
+    sels = _block_selections(L, C, P, Hkv, T, 135)
+    ref = run_sequence_blocks(q, k, v, do, C, P, scale, T, selections=sels)
+    G = Hq // Hkv
+    mask = np.zeros((Hkv, L, L), dtype=bool)
+    for i in range(L):
+        c, b = i // C, (i % C) // T
+        for g in range(Hkv):
+            for pg in sels[c][b][g]:
+                mask[g, i, pg * P:(pg + 1) * P] = True
+            mask[g, i, c * C:i + 1] = True
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    outs, lses = [], []
+    for h in range(Hq):
+        g = h // G
+        s = scale * (tq[:, h] @ tk[:, g].T)
+        s = torch.where(torch.tensor(mask[g]), s, torch.tensor(float("-inf"), dtype=s.dtype))
+        lses.append(torch.logsumexp(s, 1))
+        outs.append(torch.softmax(s, 1) @ tv[:, g])
+    o_t = torch.stack(outs, 1)
+    np.testing.assert_allclose(ref["o"], o_t.detach().numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(ref["lse"], torch.stack(lses).detach().numpy(), rtol=1e-12,
+                               atol=1e-12)
+    (o_t * torch.tensor(do)).sum().backward()
+    np.testing.assert_allclose(ref["dq"], tq.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(ref["dk"], tk.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(ref["dv"], tv.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_row_blocks_with_one_shared_selection_equal_the_chunk_form():
+    L, C, P, Hq, Hkv, d = 48, 16, 4, 4, 2, 8
+    q, k, v, do = (_rand((L, Hq, d), 141), _rand((L, Hkv, d), 142), _rand((L, Hkv, d), 143),
+                   _rand((L, Hq, d), 144))
+    chunk_sels = [s[0] for s in _block_selections(L, C, P, Hkv, C, 145)]
+    blocks = [[s] * 2 for s in chunk_sels]                  # two 8-row blocks, same lists
+    a = run_sequence(q, k, v, do, C, P, 0.3, selections=chunk_sels)
+    b = run_sequence_blocks(q, k, v, do, C, P, 0.3, 8, selections=blocks)
+    for key in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_allclose(b[key], a[key], rtol=1e-12, atol=1e-13)
+
+
+def test_row_block_topk_is_the_selection_of_the_block_rows():
+    L, C, P, Hq, Hkv, d, T = 48, 16, 4, 4, 2, 8, 8
+    q, k, v, do = (_rand((L, Hq, d), 151), _rand((L, Hkv, d), 152), _rand((L, Hkv, d), 153),
+                   _rand((L, Hq, d), 154))
+    r = run_sequence_blocks(q, k, v, do, C, P, 0.3, T, top_k=2, n_recent=1, with_backward=False)
+    for c in range(1, L // C):
+        for b in range(C // T):
+            rows = slice(c * C + b * T, c * C + (b + 1) * T)
+            want, _ = topk_for_chunk(q[rows], k[:c * C], P, 2, 1)
+            assert r["selected"][c][b] == want
+
