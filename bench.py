@@ -158,12 +158,24 @@ class Run:
             self.loc_p = [torch.zeros((Hkv, w.window), dtype=torch.int32, device=device)
                           for _ in range(N)]
             self.loc_n = [torch.zeros((Hkv,), dtype=torch.int32, device=device) for _ in range(N)]
+        self.qtile = sparse and w.qtile_topk
         if sparse:
             ms = w.top_k + w.n_recent
-            self.sel_l = [torch.zeros((Hkv, ms), dtype=torch.int32, device=device) for _ in range(N)]
-            self.sel_p = [torch.zeros((Hkv, ms), dtype=torch.int32, device=device) for _ in range(N)]
-            self.sel_n = [torch.zeros((Hkv,), dtype=torch.int32, device=device) for _ in range(N)]
-            ws = pk.page_topk_workspace_size(C, Hq, Hkv, d, (N - 1) * ppc)
+            nq = (C + 127) // 128 if self.qtile else None
+            lead = (nq, Hkv) if self.qtile else (Hkv,)
+            self.sel_l = [torch.zeros(lead + (ms,), dtype=torch.int32, device=device)
+                          for _ in range(N)]
+            self.sel_p = [torch.zeros(lead + (ms,), dtype=torch.int32, device=device)
+                          for _ in range(N)]
+            self.sel_n = [torch.zeros(lead, dtype=torch.int32, device=device) for _ in range(N)]
+            if self.qtile:
+                ws = pk.page_topk_batched_workspace_size(nq, Hkv, d, (N - 1) * ppc)
+                self.row_start = torch.arange(0, (nq + 1) * 128, 128, dtype=torch.int32,
+                                              device=device).clamp_(max=C)
+                self.npast = [torch.full((nq,), c * ppc, dtype=torch.int32, device=device)
+                              for c in range(N)]
+            else:
+                ws = pk.page_topk_workspace_size(C, Hq, Hkv, d, (N - 1) * ppc)
             self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         # algorithmic FLOPs per chunk (per kernel class) and per step
         self.flops = {"fwd": [], "dkdv": [], "dq": []}
@@ -180,9 +192,10 @@ class Run:
             self.flops["dq"].append(2.0 * pairs * d)
         self.step_flops = sum(sum(v) for v in self.flops.values())
         # per chunk: append, forward, preprocess, dK/dV, dQ; Top-K adds query
-        # mean, page scores and select per chunk with a past; local lists one
+        # mean, page scores and select per chunk with a past (per-query-tile
+        # lists: and a second dK/dV launch); local lists one
         self.launches_per_step = N * 5 + ((N - 1) * 3 if sparse else 0) + \
-            ((N - 1) if self.local else 0)
+            ((N - 1) if self.local else 0) + ((N - 1) if self.qtile else 0)
 
     def step(self, timers=None):
         """One pass over all chunks.  With concurrent_bwd, chunk c's dQ launch
@@ -221,6 +234,13 @@ class Run:
                                                       n_past, self.loc_p[c], self.loc_n[c],
                                                       stream=stream))
                 past, cnt = self.loc_p[c], self.loc_n[c]
+            elif self.qtile:
+                n_past = c * ppc
+                timed("topk", lambda: pk.page_topk_batched(
+                    self.pool, x["q"], self.row_start, 128, self.npast[c], n_past,
+                    self.page_table_dev[:n_past], w.top_k, w.n_recent, self.sel_l[c],
+                    self.sel_p[c], self.sel_n[c], self.ws, stream=stream))
+                past, cnt = self.sel_p[c], self.sel_n[c]
             elif self.sparse:
                 n_past = c * ppc
                 timed("topk", lambda: pk.page_topk(
@@ -659,6 +679,8 @@ def main():
     ap.add_argument("--no-hbm", action="store_true", help="skip the batched HBM/host-link kernels")
     ap.add_argument("--no-local", action="store_true", help="skip the recent-only page-list run")
     ap.add_argument("--local-workload", default="qwen256k_local")
+    ap.add_argument("--no-qtile", action="store_true", help="skip the per-query-tile Top-K run")
+    ap.add_argument("--qtile-workload", default="qwen256k_topk_qtile")
     ap.add_argument("--serial-bwd", action="store_true",
                     help="run each chunk's dQ launch after its dK/dV launch on one stream")
     ap.add_argument("--offload-workload", default="qwen1m_topk_offload")
@@ -803,6 +825,21 @@ def main():
         del lr
         torch.cuda.empty_cache()
 
+    qtile_obj = None
+    if not a.no_qtile:
+        wq = synth.WORKLOADS[a.qtile_workload]
+        qr = Run(wq, True, device)
+        qr.concurrent_bwd = not a.serial_bwd
+        ms_q, kt_q = time_steps(qr, a.steps, a.warmup, dist_on, device)
+        qtile_obj = {"workload": wq.name, "selection": "Top-K per 128-row query tile",
+                     "value": qr.step_flops * world / (ms_q / 1e3) / 1e12, "unit": "TFLOP/s",
+                     "ms_per_step": ms_q, "tokens_per_s": wq.context * world / (ms_q / 1e3),
+                     "kernels": {k: {"ms_per_step": v} for k, v in kt_q.items()},
+                     "device_status": pk.get_device_status(qr.pool)}
+        qr.close()
+        del qr
+        torch.cuda.empty_cache()
+
     offload_obj = None
     if not a.no_offload:
         offload_obj = offload_run(synth.WORKLOADS[a.offload_workload], max(1, min(a.steps, 2)),
@@ -857,6 +894,7 @@ def main():
         "roofline": roof,
         "sparse": sparse_obj,
         "local": local_obj,
+        "qtile_topk": qtile_obj,
         "offload": offload_obj,
         "hbm_kernels": hbm_obj,
         "e2e": e2e,

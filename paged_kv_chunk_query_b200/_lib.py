@@ -59,7 +59,8 @@ class AttnArgs(ctypes.Structure):
                 ("delta_ws", ctypes.c_void_p), ("chunk_len", ctypes.c_int32),
                 ("num_q_heads", ctypes.c_int32), ("past_pages", ctypes.c_void_p),
                 ("past_counts", ctypes.c_void_p), ("max_past", ctypes.c_int32),
-                ("cur_pages", ctypes.c_void_p), ("softmax_scale", ctypes.c_float)]
+                ("cur_pages", ctypes.c_void_p), ("softmax_scale", ctypes.c_float),
+                ("lists_per_qtile", ctypes.c_int32)]
 
 
 _lib = None
@@ -258,8 +259,17 @@ def kv_append(pool: int, page_ids: torch.Tensor, k: torch.Tensor, v: torch.Tenso
 
 def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o=None, dq=None,
                delta_ws=None):
+    """past_pages [Hkv][max_past] (one list per group) or [n_qtiles][Hkv][max_past]
+    (one list per 128-row query tile and group; counts [n_qtiles][Hkv])."""
     C, Hq, _ = q.shape
-    max_past = past_pages.shape[1] if past_pages is not None and past_pages.numel() else 0
+    per_qtile = past_pages is not None and past_pages.dim() == 3
+    max_past = past_pages.shape[-1] if past_pages is not None and past_pages.numel() else 0
+    if per_qtile and max_past:
+        n_qt = (C + 127) // 128
+        if past_pages.shape[0] != n_qt or past_counts is None or \
+                tuple(past_counts.shape) != tuple(past_pages.shape[:2]):
+            raise ValueError(f"per-query-tile lists need past_pages [{n_qt}][Hkv][max_past] and "
+                             f"past_counts [{n_qt}][Hkv]")
     return AttnArgs(
         _dev_tensor(q, torch.bfloat16, "q"), _dev_tensor(o, torch.bfloat16, "o"),
         _dev_tensor(lse, torch.float32, "lse"),
@@ -269,7 +279,8 @@ def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o
         C, Hq,
         _dev_tensor(past_pages, torch.int32, "past_pages") if max_past else None,
         _dev_tensor(past_counts, torch.int32, "past_counts") if max_past else None,
-        max_past, _dev_tensor(cur_pages, torch.int32, "cur_pages"), softmax_scale)
+        max_past, _dev_tensor(cur_pages, torch.int32, "cur_pages"), softmax_scale,
+        int(per_qtile))
 
 
 def chunk_attn_fwd(pool, q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,

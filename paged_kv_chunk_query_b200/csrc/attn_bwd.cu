@@ -36,6 +36,7 @@ struct BwdParams {
   const int32_t* cur_pages;
   uint32_t* status;
   int max_past, C, Hq, Hkv, G, P, num_pool_pages, max_past_tiles;
+  int lpq;  // 1: one past list per (query tile, group); dK/dV: blockIdx.z = query tile
   float scale, scale_log2;
 };
 
@@ -93,14 +94,19 @@ __global__ void __launch_bounds__(320, 1)
                     const __grid_constant__ CUtensorMap kvmap) {
   using Cfg = KvCfg<D>;
   const int g = blockIdx.y;
-  const KvSchedule sch = kv_schedule(p.past_counts, g, p.max_past, p.P, p.status);
+  // with one list per query tile this CTA serves query tile blockIdx.z only
+  // (the chunk's own tiles then come from a separate launch without lists)
+  const int qsel = p.lpq ? static_cast<int>(blockIdx.z) : 0;
+  const int li = (p.lpq ? qsel * p.Hkv : 0) + g;
+  const KvSchedule sch = kv_schedule(p.past_counts ? p.past_counts + (li - g) : nullptr, g,
+                                     p.max_past, p.P, p.status);
   const bool is_past = static_cast<int>(blockIdx.x) < p.max_past_tiles;
   if (is_past && static_cast<int>(blockIdx.x) >= sch.n_past_tiles) return;  // beyond the list
   const int u = is_past ? 0 : static_cast<int>(blockIdx.x) - p.max_past_tiles;  // current tile
   const int j = is_past ? static_cast<int>(blockIdx.x) : sch.n_past_tiles + u;    // schedule index
   const int n_qtiles = (p.C + kTile - 1) / kTile;
-  const int t0 = is_past ? 0 : u;  // first query tile that can see these keys
-  const int n_qt = n_qtiles - t0;
+  const int t0 = p.lpq ? qsel : (is_past ? 0 : u);  // first query tile that can see these keys
+  const int n_qt = p.lpq ? 1 : n_qtiles - t0;
   const int n_iter = p.G * n_qt;
   const int n_cur_pages = p.C / p.P;
 
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
-  const int32_t* past_list = p.past_pages ? p.past_pages + static_cast<size_t>(g) * p.max_past
+  const int32_t* past_list = p.past_pages ? p.past_pages + static_cast<size_t>(li) * p.max_past
                                           : nullptr;
 
   if (warp == 8) {
@@ -439,7 +445,9 @@ __global__ void __launch_bounds__(352, 1)
 
   const int warp = warp_id(), lane = lane_id();
   const int qt = blockIdx.x, h = blockIdx.y, g = h / p.G;
-  const KvSchedule sch = kv_schedule(p.past_counts, g, p.max_past, p.P, p.status);
+  const int li = (p.lpq ? qt * p.Hkv : 0) + g;
+  const KvSchedule sch = kv_schedule(p.past_counts ? p.past_counts + (li - g) : nullptr, g,
+                                     p.max_past, p.P, p.status);
   const int T = sch.n_past_tiles + qt + 1;
   const int n_cur_pages = p.C / p.P;
 
@@ -488,7 +496,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       prefetch_tensormap(&kvmap);
       const int32_t* past_list =
-          p.past_pages ? p.past_pages + static_cast<size_t>(g) * p.max_past : nullptr;
+          p.past_pages ? p.past_pages + static_cast<size_t>(li) * p.max_past : nullptr;
       const int per = kTile / p.P;
       const int nst = is_k ? Cfg::kNK : Cfg::kNV;
       uint64_t* full = is_k ? bar_kf : bar_vf;
@@ -750,6 +758,7 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.max_past_tiles = (a->max_past * s.P + kTile - 1) / kTile;
   p.scale = a->softmax_scale;
   p.scale_log2 = a->softmax_scale * kLog2e;
+  p.lpq = a->lists_per_qtile;
 
   if (step < 0 || step == OOMB_BWD_PREPROCESS) {
     constexpr int RPB = 256 / (D / 8);
@@ -762,10 +771,26 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
     if (!make_row_map(&qmap, a->q, D, s.Hq, s.C) || !make_row_map(&domap, a->d_o, D, s.Hq, s.C) ||
         !make_pool_map(&kvmap, pool))
       return OOMB_ERR_CUDA;
-    if (step < 0 || step == OOMB_BWD_DKDV) {
+    if ((step < 0 || step == OOMB_BWD_DKDV) && !p.lpq) {
       dim3 grid(p.max_past_tiles + s.n_qtiles, s.Hkv);
       bwd_dkdv_kernel<D><<<grid, 320, KvCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
       if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+    }
+    if ((step < 0 || step == OOMB_BWD_DKDV) && p.lpq) {
+      // the chunk's own tiles, for every query tile that reaches them
+      BwdParams pc = p;
+      pc.lpq = 0;
+      pc.max_past = pc.max_past_tiles = 0;
+      pc.past_pages = pc.past_counts = nullptr;
+      bwd_dkdv_kernel<D><<<dim3(s.n_qtiles, s.Hkv), 320, KvCfg<D>::kSmem, stream>>>(
+          pc, qmap, domap, kvmap);
+      if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+      // each query tile's listed pages: one z-slice per query tile
+      if (p.max_past_tiles > 0) {
+        bwd_dkdv_kernel<D><<<dim3(p.max_past_tiles, s.Hkv, s.n_qtiles), 320, KvCfg<D>::kSmem,
+                             stream>>>(p, qmap, domap, kvmap);
+        if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+      }
     }
     if (step < 0 || step == OOMB_BWD_DQ) {
       dim3 grid(s.n_qtiles, s.Hq);

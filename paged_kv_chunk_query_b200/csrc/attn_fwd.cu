@@ -45,6 +45,7 @@ struct FwdParams {
   const int32_t* cur_pages;
   uint32_t* status;
   int max_past, C, Hq, G, P, num_pool_pages;
+  int lpq;  // 1: one past list per (query tile, group)
   float scale_log2;
 };
 
@@ -81,7 +82,10 @@ __global__ void __launch_bounds__(224, 1)
 
   const int warp = warp_id(), lane = lane_id();
   const int qt = blockIdx.x, h = blockIdx.y, g = h / p.G;
-  const KvSchedule sch = kv_schedule(p.past_counts, g, p.max_past, p.P, p.status);
+  // list of (query tile, group) or of the group
+  const int li = (p.lpq ? qt * (p.Hq / p.G) : 0) + g;
+  const KvSchedule sch = kv_schedule(p.past_counts ? p.past_counts + (li - g) : nullptr, g,
+                                     p.max_past, p.P, p.status);
   const int T = sch.n_past_tiles + qt + 1;  // past tiles + current tiles up to the diagonal
   const int n_cur_pages = p.C / p.P;
 
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(224, 1)
           tma_load_3d(sQ + hf * kTile * 128, &qmap, &bar_q, hf * 64, h, qt * kTile);
       }
       prefetch_tensormap(&kvmap);
-      const int32_t* past_list = p.past_pages + static_cast<size_t>(g) * p.max_past;
+      const int32_t* past_list = p.past_pages + static_cast<size_t>(li) * p.max_past;
       const int per = kTile / p.P;
       const int nst = is_k ? Cfg::kNK : Cfg::kNV;
       uint64_t* full = is_k ? bar_kf : bar_vf;
@@ -399,6 +403,7 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.P = s.P;
   p.num_pool_pages = pool->desc.num_pages;
   p.scale_log2 = a->softmax_scale * kLog2e;
+  p.lpq = a->lists_per_qtile;
   dim3 grid(s.n_qtiles, s.Hq);
   attn_fwd_kernel<D><<<grid, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
   return check_launch();

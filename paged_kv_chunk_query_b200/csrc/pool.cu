@@ -250,6 +250,7 @@ oomb_status validate_attn(const oomb_pool* pool, const oomb_attn_args* a, bool b
   if (a->num_q_heads <= 0 || a->num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
   if (a->max_past < 0 || (a->max_past > 0 && (!a->past_pages || !a->past_counts)))
     return OOMB_ERR_INVALID_ARG;
+  if (a->lists_per_qtile != 0 && a->lists_per_qtile != 1) return OOMB_ERR_INVALID_ARG;
   if (!a->q || !a->o || !a->lse || !a->cur_pages) return OOMB_ERR_INVALID_ARG;
   if (!aligned16(a->q) || !aligned16(a->o)) return OOMB_ERR_INVALID_ARG;
   if (!(a->softmax_scale > 0.f)) return OOMB_ERR_INVALID_ARG;

@@ -47,6 +47,7 @@ class Workload:
     n_recent: int = 0
     host_resident: bool = False   # past KV and grads in pinned host memory
     window: int = 0               # > 0: recent-only lists of this many past pages
+    qtile_topk: bool = False      # Top-K per 128-row query tile instead of per chunk
 
     @property
     def group_size(self) -> int:
@@ -87,6 +88,10 @@ WORKLOADS = {
     "qwen256k_topk": Workload("qwen256k_topk", 28, 4, 128, 64, 4096, 64, seed=1003,
                               shuffle_pages=True, page_direction=0.5, top_k=64,
                               n_recent=2),
+    # one Top-K selection per 128-row query tile (per-query-page sparsity)
+    "qwen256k_topk_qtile": Workload("qwen256k_topk_qtile", 28, 4, 128, 64, 4096, 64, seed=1007,
+                                    shuffle_pages=True, page_direction=0.5, top_k=64,
+                                    n_recent=2, qtile_topk=True),
     # recent-only page lists: the last 64 past pages (4096 tokens) + the chunk
     "qwen256k_local": Workload("qwen256k_local", 28, 4, 128, 64, 4096, 64, seed=1006,
                                shuffle_pages=True, window=64),
