@@ -201,7 +201,7 @@ oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk
  * OOMB_TOPK_STATIC_SCRATCH_BYTES inside the library, held on every GPU that
  * loads it until the process exits.  Returns OOMB_ERR_UNSUPPORTED when
  * oomb_page_topk_workspace_size() of the call exceeds that size (e.g. with
- * Hkv = 4 and d = 128, n_past up to 24,576 pages fits).  It allocates nothing.
+ * Hkv = 4 and d = 128, n_past up to 24,512 pages fits).  It allocates nothing.
  * The first call on a device looks up the array's device address (with that
  * device current); make that first call before any stream capture.  All calls
  * share the one array: calls that overlap on the GPU (different streams) race

@@ -13,13 +13,14 @@
 // The kernels take a batch of independent problems (blockIdx.z / .y), each a
 // range of query rows and its own number of past pages; the per-chunk entry
 // points run a batch of one.
-// Kernel 1 (qmean_partial): grid (slices, Hkv, problems); each CTA streams a
-//   slice of its problem's rows with 16-byte loads, 8 in flight per thread,
-//   and writes one fp32 partial sum per d.
-// Kernel 2 (page_score): grid (pages / 64, Hkv, problems); each CTA reduces
-//   the partials in a fixed order into q_bar, then each warp scores 8 pages
-//   (float4 loads of the summaries, shuffle reduction).
-// Kernel 3 (select): one CTA per (group, problem); finds the K-th largest
+// Kernel 1 (qmean_partial): grid (slices, problems); each CTA streams whole
+//   token rows (all heads, contiguous) of a slice of its problem's rows, one
+//   thread per 16-byte column, and writes one fp32 partial per (group, d).
+// Kernel 2 (qbar): grid (problems, Hkv); sums the slice partials in a fixed
+//   order into q_bar.
+// Kernel 3 (page_score): grid (pages / 64, Hkv, problems); each warp scores 8
+//   pages (float4 loads of the summaries, shuffle reduction).
+// Kernel 4 (select): one CTA per (group, problem); finds the K-th largest
 //   64-bit key (ordered score, inverted id) by 8-bit radix passes from the top
 //   with a parallel bin scan, stopping once the boundary bin is kept whole,
 //   then compacts the kept ids in ascending order.
@@ -32,7 +33,7 @@
 namespace {
 
 constexpr int kSplits = 128;         // max query-mean slices per (problem, group)
-constexpr int kMeanThreads = 256;
+constexpr int kMeanThreadsMax = 1024;  // query mean: one thread per 16-byte column of a token
 constexpr int kScoreThreads = 256;   // 8 warps x 8 pages per CTA
 constexpr int kPagesPerScoreCta = 64;
 constexpr int kSelectThreads = 1024;
@@ -84,56 +85,72 @@ __device__ __forceinline__ int problem_npast(const Problems& pb, int b) {
 }
 
 // ---------------------------------------------------------------- query mean
-// grid (splits, Hkv, problems): CTA (s, g, b) sums rows (token, head in g) of
-// slice s of problem b's tokens.  Each thread keeps 8 independent 16-byte
-// loads in flight (about 32 KiB per CTA), enough with 3-4 CTAs per SM to
-// stream Q at HBM speed.
+// grid (splits, problems): CTA (s, b) streams slice s of problem b's tokens,
+// whole token rows (every head: Hq * d * 2 contiguous bytes), one thread per
+// 16-byte column, 4 rows in flight per thread; then sums the G heads of each
+// group in shared memory (fixed order) and writes one fp32 partial per
+// (group, d).  Reading whole rows keeps every DRAM page opened once.
 template <int D>
-__global__ void __launch_bounds__(kMeanThreads) qmean_partial_kernel(
+__global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
     const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, const Problems pb, int Hq,
     int G) {
-  constexpr int VPR = D / 8;               // 16-byte vectors per row
-  constexpr int RG = kMeanThreads / VPR;   // rows per pass
-  constexpr int U = 8;                     // loads in flight per thread
-  __shared__ float red[RG][D];
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
-  const int vec = t % VPR, rg = t / VPR;
+  extern __shared__ float col_sum[];  // [Hq][D]
+  constexpr int VPR = D / 8;          // 16-byte vectors per (token, head) row
+  constexpr int U = 4;                // rows in flight per thread
+  const int split = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const int ncol = Hq * VPR;          // 16-byte vectors per token
   int r0, r1;
   problem_rows(pb, b, r0, r1);
   const int per = (r1 - r0 + pb.splits - 1) / pb.splits;
   const int tok0 = r0 + split * per, tok1 = min(r1, tok0 + per);
-  const int rows = max(0, tok1 - tok0) * G;
-  float acc[8];
+  const uint4* base = reinterpret_cast<const uint4*>(q);
+  for (int col = t; col < ncol; col += blockDim.x) {
+    float acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int base = rg; base < rows; base += RG * U) {
-    uint4 v[U];
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    int tok = tok0;
+    for (; tok + U <= tok1; tok += U) {
+      uint4 v[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int rr = base + u * RG;
-      if (rr < rows) {
-        const int tok = tok0 + rr / G, hh = g * G + rr % G;
-        v[u] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<size_t>(tok) * Hq + hh) * D +
-                                                    vec * 8));
-      } else {
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; u < U; ++u) v[u] = __ldg(base + static_cast<size_t>(tok + u) * ncol + col);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(bv[e]);
       }
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
+    for (; tok < tok1; ++tok) {
+      const uint4 v = __ldg(base + static_cast<size_t>(tok) * ncol + col);
+      const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(bv[e]);
     }
-  }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[rg][vec * 8 + e] = acc[e];
-  __syncthreads();
-  if (t < D) {
-    float s = 0.f;
-    for (int r = 0; r < RG; ++r) s += red[r][t];  // fixed order: deterministic
-    partial[((static_cast<size_t>(b) * pb.splits + split) * gridDim.y + g) * D + t] = s;
+    for (int e = 0; e < 8; ++e) col_sum[col * 8 + e] = acc[e];  // (head, d) = col * 8 + e
   }
+  __syncthreads();
+  const int Hkv = Hq / G;
+  for (int i = t; i < Hkv * D; i += blockDim.x) {
+    const int g = i / D, dd = i % D;
+    float s = 0.f;
+    for (int hh = 0; hh < G; ++hh) s += col_sum[(g * G + hh) * D + dd];  // fixed order
+    partial[((static_cast<size_t>(b) * pb.splits + split) * Hkv + g) * D + dd] = s;
+  }
+}
+
+// grid (problems, Hkv), D threads: q_bar = (sum of the slice partials in slice
+// order) / (rows * G), once per (problem, group).
+__global__ void qbar_kernel(const float* __restrict__ partial, float* __restrict__ qbar,
+                            const Problems pb, int G, int D) {
+  const int b = blockIdx.x, g = blockIdx.y, Hkv = gridDim.y, dd = threadIdx.x;
+  int r0, r1;
+  problem_rows(pb, b, r0, r1);
+  const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
+  const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D;
+  float s = 0.f;
+  for (int i = 0; i < pb.splits; ++i) s += __ldg(pp + (static_cast<size_t>(i) * Hkv + g) * D + dd);
+  qbar[(static_cast<size_t>(b) * Hkv + g) * D + dd] = rows > 0.f ? s / rows : 0.f;
 }
 
 __device__ __forceinline__ uint32_t order_f32(float f) {
@@ -149,41 +166,19 @@ __device__ __forceinline__ uint32_t order_f32(float f) {
 // (~logical id), stored at [problem][group][max_past].
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads) page_score_kernel(
-    const float* __restrict__ partial, const float* __restrict__ summary,
-    const int32_t* __restrict__ page_table, const Problems pb, int Hkv, int G,
+    const float* __restrict__ qbar, const float* __restrict__ summary,
+    const int32_t* __restrict__ page_table, const Problems pb, int Hkv,
     int num_pool_pages, unsigned long long* __restrict__ keys, float* __restrict__ out_scores) {
-  constexpr int kParts = kScoreThreads / D;  // threads per d in the q_bar reduction
-  __shared__ float part_sum[kParts][D];
-  __shared__ float qbar[D];
-  const int g = blockIdx.y, b = blockIdx.z, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = blockIdx.y, b = blockIdx.z, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n_past = problem_npast(pb, b);
   if (static_cast<int>(blockIdx.x) * kPagesPerScoreCta >= n_past) return;  // whole CTA
-  {
-    int r0, r1;
-    problem_rows(pb, b, r0, r1);
-    const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
-    const float inv_rows = rows > 0.f ? 1.0f / rows : 0.f;
-    const int d = t % D, part = t / D;
-    const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D;
-    float s = 0.f;
-#pragma unroll 8
-    for (int i = part; i < pb.splits; i += kParts) s += __ldg(pp + (static_cast<size_t>(i) * Hkv + g) * D + d);
-    part_sum[part][d] = s;
-    __syncthreads();
-    if (t < D) {
-      float s2 = 0.f;
-#pragma unroll
-      for (int i = 0; i < kParts; ++i) s2 += part_sum[i][t];
-      qbar[t] = s2 * inv_rows;
-    }
-    __syncthreads();
-  }
+  const float* qb = qbar + (static_cast<size_t>(b) * Hkv + g) * D;
   constexpr int PW = kPagesPerScoreCta / (kScoreThreads / 32);  // pages per warp
   const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
   constexpr int EPL = D / 32;  // elements per lane
   float qv[EPL];
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) qv[e] = qbar[lane * EPL + e];
+  for (int e = 0; e < EPL; ++e) qv[e] = __ldg(qb + lane * EPL + e);
   float acc[PW];
 #pragma unroll
   for (int i = 0; i < PW; ++i) {
@@ -334,12 +329,13 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
   if (t == 0) out_count[row] = min(running_sh, max_sel);
 }
 
-// Workspace: partials [problems][splits <= 128][Hkv][d] fp32, then keys
-// [problems][Hkv][max(max_past, 1)] u64.
+// Workspace: partials [problems][splits <= 128][Hkv][d] fp32, q_bar
+// [problems][Hkv][d] fp32, then keys [problems][Hkv][max(max_past, 1)] u64.
 size_t workspace_bytes_for(int64_t problems, int Hkv, int D, int max_past) {
   const size_t partial = static_cast<size_t>(problems) * kSplits * Hkv * D * 4;
+  const size_t qbar = static_cast<size_t>(problems) * Hkv * D * 4;
   const size_t keys = static_cast<size_t>(problems) * Hkv * (max_past > 0 ? max_past : 1) * 8;
-  return align256(partial) + align256(keys);
+  return align256(partial) + align256(qbar) + align256(keys);
 }
 
 // Launches the three kernels for `n_problems` problems on `s`.
@@ -352,25 +348,31 @@ oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
   const int Hkv = d.num_kv_heads, D = d.head_dim, G = num_q_heads / Hkv;
   Problems pb = pb_in;
   pb.status = pool->d_status;
+  const size_t partial_bytes = align256(static_cast<size_t>(n_problems) * kSplits * Hkv * D * 4);
+  const size_t qbar_bytes = align256(static_cast<size_t>(n_problems) * Hkv * D * 4);
   float* partial = static_cast<float*>(scratch);
+  float* qbar = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + partial_bytes);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(
-      static_cast<uint8_t*>(scratch) +
-      align256(static_cast<size_t>(n_problems) * kSplits * Hkv * D * 4));
+      static_cast<uint8_t*>(scratch) + partial_bytes + qbar_bytes);
   const auto* q = static_cast<const __nv_bfloat16*>(d_q);
-  dim3 g1(pb.splits, Hkv, n_problems);
+  // one thread per 16-byte column of a token row, a multiple of 32, at most 1024
+  const int ncol = num_q_heads * D / 8;
+  const int mean_threads = ncol >= kMeanThreadsMax ? kMeanThreadsMax : ((ncol + 31) / 32) * 32;
+  const size_t mean_smem = static_cast<size_t>(num_q_heads) * D * 4;
+  dim3 g1(pb.splits, n_problems);
   dim3 g2((pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv, n_problems);
-  if (D == 128) {
-    qmean_partial_kernel<128><<<g1, kMeanThreads, 0, s>>>(q, partial, pb, num_q_heads, G);
-    if (pb.max_past > 0)
-      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
-                                                          pb, Hkv, G, d.num_pages, keys,
-                                                          d_out_scores);
-  } else {
-    qmean_partial_kernel<64><<<g1, kMeanThreads, 0, s>>>(q, partial, pb, num_q_heads, G);
-    if (pb.max_past > 0)
-      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(partial, pool->summary, d_page_table,
-                                                         pb, Hkv, G, d.num_pages, keys,
-                                                         d_out_scores);
+  if (D == 128)
+    qmean_partial_kernel<128><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G);
+  else
+    qmean_partial_kernel<64><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G);
+  qbar_kernel<<<dim3(n_problems, Hkv), D, 0, s>>>(partial, qbar, pb, G, D);
+  if (pb.max_past > 0) {
+    if (D == 128)
+      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(qbar, pool->summary, d_page_table, pb,
+                                                          Hkv, d.num_pages, keys, d_out_scores);
+    else
+      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(qbar, pool->summary, d_page_table, pb,
+                                                         Hkv, d.num_pages, keys, d_out_scores);
   }
   topk_select_kernel<<<dim3(Hkv, n_problems), kSelectThreads, 0, s>>>(
       keys, d_page_table, pb, top_k, n_recent, d.num_pages, d_out_logical, d_out_physical,
@@ -387,6 +389,9 @@ oomb_status check_topk_args(const oomb_pool* pool, const void* d_q, int num_q_he
   const int Hkv = pool->desc.num_kv_heads;
   if (!d_q || !d_out_logical || !d_out_count) return OOMB_ERR_INVALID_ARG;
   if (num_q_heads <= 0 || num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
+  // the query mean keeps one fp32 row of every head in 48 KiB of shared memory
+  if (static_cast<size_t>(num_q_heads) * pool->desc.head_dim * 4 > 48 * 1024)
+    return OOMB_ERR_UNSUPPORTED;
   if (max_past < 0 || max_past > 65536 || top_k < 0 || n_recent < 0 ||
       top_k + n_recent > 4096 || top_k + n_recent == 0)
     return OOMB_ERR_INVALID_ARG;

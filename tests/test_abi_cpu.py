@@ -133,5 +133,6 @@ def test_compute_calls_reject_host_pools_without_touching_cuda():
 def test_topk_workspace_size_formula():
     ws = L.page_topk_workspace_size(4096, 28, 4, 128, 4094)
     # 128 slices x 4 groups x 128 d fp32 partials + 4 x 4094 64-bit keys, 256-byte aligned
-    assert ws == 128 * 4 * 128 * 4 + ((4 * 4094 * 8 + 255) // 256) * 256
+    # query-mean partials (128 slices), q_bar, then the 64-bit page keys
+    assert ws == 128 * 4 * 128 * 4 + 4 * 128 * 4 + ((4 * 4094 * 8 + 255) // 256) * 256
     assert L.page_topk_workspace_size(0, 28, 4, 128, 10) == 0
