@@ -146,7 +146,29 @@ typedef struct oomb_attn_args {
    *    outputs of oomb_page_topk_batched with one problem per query tile have
    *    exactly this layout. */
   int32_t lists_per_qtile;
+  /* Segmented attention: the past streamed through a bounded device window
+   * ([pt] §2D: pages move between host and GPU while computation runs; a
+   * dense chunk then takes its past in pieces).
+   *   OOMB_SEG_WHOLE (0): the call covers the listed past pages and the chunk
+   *     itself (causal); outputs as described above.
+   *   OOMB_SEG_FIRST (1) / OOMB_SEG_NEXT (2): the call covers only the listed
+   *     past pages (not the chunk).  Forward: writes (FIRST) or merges into
+   *     (NEXT) the running normalised output o_acc and lse; o is not written.
+   *     Backward: dK/dV of the listed pages are added to the pool as usual; dQ
+   *     is written to (FIRST) or added into (NEXT) dq_acc; dq is not written.
+   *   OOMB_SEG_LAST (3): the call covers the listed past pages (the list may be
+   *     empty) and the chunk itself, merges into o_acc / lse and writes o and
+   *     the final lse (forward), adds into dq_acc and writes dq (backward).
+   * Segments of one chunk: every forward segment (FIRST, NEXT..., LAST), then
+   * the backward segments in any order that starts with FIRST and ends with
+   * LAST (the backward needs the final o and lse).  Per-query-tile lists
+   * cannot be combined with segments. */
+  int32_t segment;
+  float* o_acc;   /* device fp32 [chunk_len][num_q_heads][head_dim]: running O  */
+  float* dq_acc;  /* device fp32, layout of o_acc: running dQ (backward)         */
 } oomb_attn_args;
+
+enum { OOMB_SEG_WHOLE = 0, OOMB_SEG_FIRST = 1, OOMB_SEG_NEXT = 2, OOMB_SEG_LAST = 3 };
 
 /* Forward with online softmax; writes o and lse. */
 oomb_status oomb_chunk_attn_fwd(oomb_pool* pool, const oomb_attn_args* args, void* stream);

@@ -26,6 +26,7 @@ OK, ERR_INVALID_ARG, ERR_OUT_OF_PAGES, ERR_BAD_PAGE, ERR_CUDA, ERR_TIMEOUT, ERR_
     ERR_DEVICE_CHECK = range(8)
 LOC_DEVICE, LOC_PINNED_HOST, LOC_HOST = 0, 1, 2
 BWD_PREPROCESS, BWD_DKDV, BWD_DQ = 0, 1, 2
+SEG_WHOLE, SEG_FIRST, SEG_NEXT, SEG_LAST = 0, 1, 2, 3
 
 # Every exported symbol of include/oomb.h.
 EXPORTS = (
@@ -60,7 +61,8 @@ class AttnArgs(ctypes.Structure):
                 ("num_q_heads", ctypes.c_int32), ("past_pages", ctypes.c_void_p),
                 ("past_counts", ctypes.c_void_p), ("max_past", ctypes.c_int32),
                 ("cur_pages", ctypes.c_void_p), ("softmax_scale", ctypes.c_float),
-                ("lists_per_qtile", ctypes.c_int32)]
+                ("lists_per_qtile", ctypes.c_int32), ("segment", ctypes.c_int32),
+                ("o_acc", ctypes.c_void_p), ("dq_acc", ctypes.c_void_p)]
 
 
 _lib = None
@@ -258,7 +260,7 @@ def kv_append(pool: int, page_ids: torch.Tensor, k: torch.Tensor, v: torch.Tenso
 
 
 def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o=None, dq=None,
-               delta_ws=None):
+               delta_ws=None, segment=SEG_WHOLE, o_acc=None, dq_acc=None):
     """past_pages [Hkv][max_past] (one list per group) or [n_qtiles][Hkv][max_past]
     (one list per 128-row query tile and group; counts [n_qtiles][Hkv])."""
     C, Hq, _ = q.shape
@@ -280,20 +282,24 @@ def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o
         _dev_tensor(past_pages, torch.int32, "past_pages") if max_past else None,
         _dev_tensor(past_counts, torch.int32, "past_counts") if max_past else None,
         max_past, _dev_tensor(cur_pages, torch.int32, "cur_pages"), softmax_scale,
-        int(per_qtile))
+        int(per_qtile), segment,
+        _dev_tensor(o_acc, torch.float32, "o_acc") if o_acc is not None else None,
+        _dev_tensor(dq_acc, torch.float32, "dq_acc") if dq_acc is not None else None)
 
 
 def chunk_attn_fwd(pool, q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
-                   stream=None):
-    a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale)
+                   stream=None, segment=SEG_WHOLE, o_acc=None):
+    a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
+                   segment=segment, o_acc=o_acc)
     _check(load().oomb_chunk_attn_fwd(pool, ctypes.byref(a), _stream(stream)),
            "oomb_chunk_attn_fwd")
 
 
 def chunk_attn_bwd(pool, q, o, lse, d_o, dq, delta_ws, past_pages, past_counts, cur_pages,
-                   softmax_scale, stream=None, step=None):
+                   softmax_scale, stream=None, step=None, segment=SEG_WHOLE, o_acc=None,
+                   dq_acc=None):
     a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o, dq,
-                   delta_ws)
+                   delta_ws, segment=segment, o_acc=o_acc, dq_acc=dq_acc)
     if step is None:
         _check(load().oomb_chunk_attn_bwd(pool, ctypes.byref(a), _stream(stream)),
                "oomb_chunk_attn_bwd")

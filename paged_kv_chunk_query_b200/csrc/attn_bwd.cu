@@ -37,6 +37,8 @@ struct BwdParams {
   uint32_t* status;
   int max_past, C, Hq, Hkv, G, P, num_pool_pages, max_past_tiles;
   int lpq;  // 1: one past list per (query tile, group); dK/dV: blockIdx.z = query tile
+  int seg;  // OOMB_SEG_*: whole key set, or a segment accumulated into dq_acc
+  float* dq_acc;
   float scale, scale_log2;
 };
 
@@ -448,7 +450,9 @@ __global__ void __launch_bounds__(352, 1)
   const int li = (p.lpq ? qt * p.Hkv : 0) + g;
   const KvSchedule sch = kv_schedule(p.past_counts ? p.past_counts + (li - g) : nullptr, g,
                                      p.max_past, p.P, p.status);
-  const int T = sch.n_past_tiles + qt + 1;
+  // past tiles + (unless this call is a past-only segment) the chunk's tiles
+  const bool with_cur = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
+  const int T = sch.n_past_tiles + (with_cur ? qt + 1 : 0);
   const int n_cur_pages = p.C / p.P;
 
   if (threadIdx.x == 0) {
@@ -559,7 +563,7 @@ __global__ void __launch_bounds__(352, 1)
         return true;
       };
       bool ok = mbar_wait(&bar_qt, 0, abort_flag);  // Q and dO are in TMEM
-      ok = ok && issue_s(0) && issue_dp(0);
+      if (T > 0) ok = ok && issue_s(0) && issue_dp(0);
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
           if (!(ok = mbar_wait(&bar_sl, j & 1, abort_flag))) break;  // S(j) in registers
@@ -667,22 +671,46 @@ __global__ void __launch_bounds__(352, 1)
     } else {
       tc_fence_after();
       const int d0 = half * (D / 2);
-      __nv_bfloat16* row = p.dq + (static_cast<size_t>(q_local) * p.Hq + h) * D + d0;
+      const size_t ridx = (static_cast<size_t>(q_local) * p.Hq + h) * D + d0;
+      // segments: FIRST writes dq_acc, NEXT adds into it, LAST adds and writes dq
+      const bool add = p.seg == OOMB_SEG_NEXT || p.seg == OOMB_SEG_LAST;
+      const bool write_bf16 = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t a[32];
-        tmem_ld32(tmem + lane_off + Cfg::kColDQ + d0 + c * 32, a);
-        tmem_ld_wait();
+        if (T > 0) {  // no tile: this call's dQ is zero (TMEM never written)
+          tmem_ld32(tmem + lane_off + Cfg::kColDQ + d0 + c * 32, a);
+          tmem_ld_wait();
+        }
         if (row_valid) {
-          uint32_t pk[16];
+          float x[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16(__uint_as_float(a[2 * e]) * p.scale,
-                              __uint_as_float(a[2 * e + 1]) * p.scale);
-          uint4* dst = reinterpret_cast<uint4*>(row + c * 32);
+          for (int e = 0; e < 32; ++e) x[e] = T > 0 ? __uint_as_float(a[e]) * p.scale : 0.f;
+          if (add) {
+            const float4* acc = reinterpret_cast<const float4*>(p.dq_acc + ridx + c * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int e = 0; e < 8; ++e) {
+              const float4 a4 = acc[e];
+              x[4 * e] += a4.x;
+              x[4 * e + 1] += a4.y;
+              x[4 * e + 2] += a4.z;
+              x[4 * e + 3] += a4.w;
+            }
+          }
+          if (write_bf16) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(p.dq + ridx + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.dq_acc + ridx + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+          }
         }
       }
     }
@@ -759,6 +787,8 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.scale = a->softmax_scale;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.lpq = a->lists_per_qtile;
+  p.seg = a->segment;
+  p.dq_acc = a->dq_acc;
 
   if (step < 0 || step == OOMB_BWD_PREPROCESS) {
     constexpr int RPB = 256 / (D / 8);
@@ -772,9 +802,13 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
         !make_pool_map(&kvmap, pool))
       return OOMB_ERR_CUDA;
     if ((step < 0 || step == OOMB_BWD_DKDV) && !p.lpq) {
-      dim3 grid(p.max_past_tiles + s.n_qtiles, s.Hkv);
-      bwd_dkdv_kernel<D><<<grid, 320, KvCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
-      if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+      // a past-only segment has no tile of the chunk itself
+      const bool with_cur = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
+      dim3 grid(p.max_past_tiles + (with_cur ? s.n_qtiles : 0), s.Hkv);
+      if (grid.x > 0) {
+        bwd_dkdv_kernel<D><<<grid, 320, KvCfg<D>::kSmem, stream>>>(p, qmap, domap, kvmap);
+        if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;
+      }
     }
     if ((step < 0 || step == OOMB_BWD_DKDV) && p.lpq) {
       // the chunk's own tiles, for every query tile that reaches them

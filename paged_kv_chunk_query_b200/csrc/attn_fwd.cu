@@ -46,6 +46,8 @@ struct FwdParams {
   uint32_t* status;
   int max_past, C, Hq, G, P, num_pool_pages;
   int lpq;  // 1: one past list per (query tile, group)
+  int seg;  // OOMB_SEG_*: whole key set, or a segment merged into o_acc / lse
+  float* o_acc;
   float scale_log2;
 };
 
@@ -86,7 +88,10 @@ __global__ void __launch_bounds__(224, 1)
   const int li = (p.lpq ? qt * (p.Hq / p.G) : 0) + g;
   const KvSchedule sch = kv_schedule(p.past_counts ? p.past_counts + (li - g) : nullptr, g,
                                      p.max_past, p.P, p.status);
-  const int T = sch.n_past_tiles + qt + 1;  // past tiles + current tiles up to the diagonal
+  // past tiles + (unless this call is a past-only segment) the chunk's tiles up
+  // to the diagonal; a past-only segment with an empty list has no tile
+  const bool with_cur = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
+  const int T = sch.n_past_tiles + (with_cur ? qt + 1 : 0);
   const int n_cur_pages = p.C / p.P;
 
   if (threadIdx.x == 0) {
@@ -313,32 +318,76 @@ __global__ void __launch_bounds__(224, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_p[b]);
     }
-    if (ok) ok = warp_wait(&bar_fin, 0, abort_flag);
+    if (ok && T > 0) ok = warp_wait(&bar_fin, 0, abort_flag);
     if (!ok) {
       *abort_flag = 1;
       if (lane == 0) atomicOr(p.status, OOMB_DEV_WAIT_LIMIT);
     } else {
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool valid = q_local < p.C;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D;
+      // this call's result: O_s = O_tmem / l with LSE_s (natural log)
+      const float lse_s = (T > 0 && l > 0.f) ? kLn2 * (m_used + log2f(l)) : -INFINITY;
+      float* lse_ptr = p.lse + static_cast<size_t>(h) * p.C + q_local;
+      // merge with the running (o_acc, lse) of earlier segments:
+      //   LSE = ln(e^LSE_old + e^LSE_s), O = e^(LSE_old - LSE) O_old + e^(LSE_s - LSE) O_s
+      const bool merge = p.seg == OOMB_SEG_NEXT || p.seg == OOMB_SEG_LAST;
+      float w_o = 0.f, w_s = 1.f, lse_new = lse_s;
+      if (merge && valid) {
+        const float lse_o = *lse_ptr;
+        const float mx = fmaxf(lse_o, lse_s);
+        if (mx == -INFINITY) {
+          lse_new = -INFINITY;
+          w_s = 0.f;
+        } else {
+          const float eo = lse_o == -INFINITY ? 0.f : expf(lse_o - mx);
+          const float es = lse_s == -INFINITY ? 0.f : expf(lse_s - mx);
+          lse_new = mx + logf(eo + es);
+          w_o = eo / (eo + es);
+          w_s = es / (eo + es);
+        }
+      }
+      const float scale_s = (T > 0 && l > 0.f) ? w_s / l : 0.f;
+      const size_t ridx = (static_cast<size_t>(q_local) * p.Hq + h) * D;
+      const bool write_bf16 = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
-        tmem_ld_wait();
+        if (T > 0) {
+          tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
+          tmem_ld_wait();
+        }
         if (valid) {
-          uint32_t pk[16];
+          float x[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          for (int e = 0; e < 32; ++e) x[e] = T > 0 ? __uint_as_float(o[e]) * scale_s : 0.f;
+          if (merge && w_o > 0.f) {
+            const float4* acc = reinterpret_cast<const float4*>(p.o_acc + ridx + c * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int e = 0; e < 8; ++e) {
+              const float4 a4 = acc[e];
+              x[4 * e] = fmaf(a4.x, w_o, x[4 * e]);
+              x[4 * e + 1] = fmaf(a4.y, w_o, x[4 * e + 1]);
+              x[4 * e + 2] = fmaf(a4.z, w_o, x[4 * e + 2]);
+              x[4 * e + 3] = fmaf(a4.w, w_o, x[4 * e + 3]);
+            }
+          }
+          if (write_bf16) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(p.o + ridx + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.o_acc + ridx + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+          }
         }
       }
-      if (valid) p.lse[static_cast<size_t>(h) * p.C + q_local] = kLn2 * (m_used + log2f(l));
+      if (valid) *lse_ptr = merge ? lse_new : lse_s;
     }
   }
 
@@ -404,6 +453,8 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.num_pool_pages = pool->desc.num_pages;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.lpq = a->lists_per_qtile;
+  p.seg = a->segment;
+  p.o_acc = a->o_acc;
   dim3 grid(s.n_qtiles, s.Hq);
   attn_fwd_kernel<D><<<grid, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
   return check_launch();

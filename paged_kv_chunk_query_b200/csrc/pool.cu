@@ -251,6 +251,12 @@ oomb_status validate_attn(const oomb_pool* pool, const oomb_attn_args* a, bool b
   if (a->max_past < 0 || (a->max_past > 0 && (!a->past_pages || !a->past_counts)))
     return OOMB_ERR_INVALID_ARG;
   if (a->lists_per_qtile != 0 && a->lists_per_qtile != 1) return OOMB_ERR_INVALID_ARG;
+  if (a->segment < OOMB_SEG_WHOLE || a->segment > OOMB_SEG_LAST) return OOMB_ERR_INVALID_ARG;
+  if (a->segment != OOMB_SEG_WHOLE) {
+    if (a->lists_per_qtile) return OOMB_ERR_INVALID_ARG;
+    if (!a->o_acc || !aligned16(a->o_acc)) return OOMB_ERR_INVALID_ARG;
+    if (backward && (!a->dq_acc || !aligned16(a->dq_acc))) return OOMB_ERR_INVALID_ARG;
+  }
   if (!a->q || !a->o || !a->lse || !a->cur_pages) return OOMB_ERR_INVALID_ARG;
   if (!aligned16(a->q) || !aligned16(a->o)) return OOMB_ERR_INVALID_ARG;
   if (!(a->softmax_scale > 0.f)) return OOMB_ERR_INVALID_ARG;

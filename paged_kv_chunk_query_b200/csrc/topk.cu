@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
   }
 }
 
-// grid (problems, Hkv), D threads: q_bar = (sum of the slice partials in slice
-// order) / (rows * G), once per (problem, group).
+// grid (problems, Hkv), D threads: q_bar = (sum of the slice partials, in a
+// fixed order) / (rows * G), once per (problem, group).
 __global__ void qbar_kernel(const float* __restrict__ partial, float* __restrict__ qbar,
                             const Problems pb, int G, int D) {
   const int b = blockIdx.x, g = blockIdx.y, Hkv = gridDim.y, dd = threadIdx.x;
@@ -148,8 +148,17 @@ __global__ void qbar_kernel(const float* __restrict__ partial, float* __restrict
   problem_rows(pb, b, r0, r1);
   const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
   const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D;
-  float s = 0.f;
-  for (int i = 0; i < pb.splits; ++i) s += __ldg(pp + (static_cast<size_t>(i) * Hkv + g) * D + dd);
+  // eight independent chains (eight loads in flight), combined in a fixed order
+  float s8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+  int i = 0;
+  for (; i + 8 <= pb.splits; i += 8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s8[e] += __ldg(pp + (static_cast<size_t>(i + e) * Hkv + g) * D + dd);
+  }
+  for (; i < pb.splits; ++i) s8[i & 7] += __ldg(pp + (static_cast<size_t>(i) * Hkv + g) * D + dd);
+  const float s = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
   qbar[(static_cast<size_t>(b) * Hkv + g) * D + dd] = rows > 0.f ? s / rows : 0.f;
 }
 
