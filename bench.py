@@ -480,6 +480,46 @@ def offload_run(w, steps, device, dist_on):
             "device_status": status}
 
 
+def dense_offload_run(w, window, device, dist_on, grad_path="host"):
+    """Dense 256K with KV and gradients in pinned host memory and a window of
+    `window` past pages (two slots) on the device; one step = all chunks,
+    timed with CUDA events on the compute stream (1 warm-up step)."""
+    from paged_kv_chunk_query_b200 import synth
+    from paged_kv_chunk_query_b200.offload import DenseOffloadRun
+    ins = [synth.device_chunk_inputs(w, c, device) for c in range(w.num_chunks)]
+    run = DenseOffloadRun(w, device, window, grad_path)
+    try:
+        run.run(lambda c: ins[c])
+        run.sync()
+        run.h2d_bytes = run.d2h_bytes = 0
+        _barrier(dist_on)
+        comp = torch.cuda.current_stream()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        run.run(lambda c: ins[c])
+        b.record(comp)
+        run.sync()
+        ms = _max_over_ranks(a.elapsed_time(b), dist_on, device)
+        import paged_kv_chunk_query_b200 as pk
+        status = pk.get_device_status(run.stage) | pk.get_device_status(run.host)
+        P, Hkv, d = w.page_size, w.num_kv_heads, w.head_dim
+        dev_bytes = (2 * window + w.pages_per_chunk) * Hkv * 2 * P * d * (2 + 4)
+        full_bytes = w.num_pages * Hkv * 2 * P * d * (2 + 4)
+        h2d, d2h = run.h2d_bytes, run.d2h_bytes
+    finally:
+        run.close()
+        del ins
+        torch.cuda.empty_cache()
+    return {"workload": w.name, "window_pages": window, "grad_path": grad_path,
+            "ms_per_step": ms,
+            "tokens_per_s": w.context / (ms / 1e3),
+            "device_window_bytes": dev_bytes, "full_pool_bytes": full_bytes,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "h2d_gbs": h2d / (ms / 1e3) / 1e9, "d2h_gbs": d2h / (ms / 1e3) / 1e9,
+            "device_status": status}
+
+
 # ------------------------------------------------------------------ HBM / host-link kernels
 def _event_ms(fn, reps=5, warmup=2):
     stream = torch.cuda.current_stream()
@@ -680,6 +720,11 @@ def main():
     ap.add_argument("--no-local", action="store_true", help="skip the recent-only page-list run")
     ap.add_argument("--local-workload", default="qwen256k_local")
     ap.add_argument("--no-qtile", action="store_true", help="skip the per-query-tile Top-K run")
+    ap.add_argument("--no-dense-offload", action="store_true",
+                    help="skip the dense run with host-resident KV and a device window")
+    ap.add_argument("--dense-window", type=int, default=512, help="window pages (two slots)")
+    ap.add_argument("--dense-grad-path", choices=["gpu", "host"], default="host",
+                    help="gradient write-back of the dense offload run")
     ap.add_argument("--qtile-workload", default="qwen256k_topk_qtile")
     ap.add_argument("--serial-bwd", action="store_true",
                     help="run each chunk's dQ launch after its dK/dV launch on one stream")
@@ -852,6 +897,13 @@ def main():
                 offload_obj["ms_per_chunk"] / per_chunk_dev - 1.0)
         offload_obj["tokens_per_s"] *= world
 
+    dense_off_obj = None
+    if not a.no_dense_offload:
+        dense_off_obj = dense_offload_run(w, a.dense_window, device, dist_on, a.dense_grad_path)
+        dense_off_obj["ms_per_step_device_resident"] = ms
+        dense_off_obj["overhead_vs_device_resident"] = dense_off_obj["ms_per_step"] / ms - 1.0
+        dense_off_obj["tokens_per_s"] *= world
+
     hbm_obj = None
     if not a.no_hbm:
         hbm_obj = hbm_kernels(w, device, peaks)
@@ -896,6 +948,7 @@ def main():
         "local": local_obj,
         "qtile_topk": qtile_obj,
         "offload": offload_obj,
+        "dense_offload": dense_off_obj,
         "hbm_kernels": hbm_obj,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -194,3 +194,217 @@ class OffloadRun:
         h2d = sel * kv_block + ((sel + own) * g_block if backward else 0)
         d2h = own * kv_block + ((sel + own) * g_block if backward else 0)
         return h2d, d2h
+
+
+class DenseOffloadRun:
+    """Dense attention with KV and gradients in pinned host memory and a
+    bounded device window ([pt] §2D: pages move between host and GPU on
+    dedicated streams while computation runs; the pages' dense-model case).
+
+    The device holds two slots of ``window`` pages each plus the chunk's own
+    pages.  A chunk's past is taken in segments of ``window`` pages: the
+    forward merges them into an fp32 running output (oomb segment modes,
+    FIRST / NEXT / LAST, the last with the chunk itself), then the backward
+    streams the same segments again, and each segment's gradient blocks are
+    added into the host pool (and zeroed) as soon as its backward is done.
+    While one slot computes, the copy stream (higher priority) fills the
+    other; the chunk's own pages are appended on the device, stored to the
+    host pool, and their gradients added back after the chunk's backward.
+
+    Host pages are taken in logical order (and the slots' pages in order), so
+    a segment is one contiguous range in both pools: its K/V travel as one
+    copy-engine transfer (oomb_page_prefetch merges consecutive blocks), which
+    takes no SM from the attention kernels; only the gradient additions run
+    as (small) kernels over the host link.
+    """
+
+    def __init__(self, w, device, window, grad_path="host"):
+        """grad_path "gpu": a kernel adds each segment's gradient blocks into the
+        pinned host pages over the host link; "host": they are copied
+        device -> host (copy engine) and a library worker thread adds them with
+        CPU threads (oomb_grad_writeback), leaving the link's host -> device
+        direction to the K/V."""
+        self.w, self.dev, self.window = w, device, window
+        self.grad_path = grad_path
+        P, Hkv, d, N = w.page_size, w.num_kv_heads, w.head_dim, w.num_chunks
+        C, Hq = w.chunk_len, w.num_q_heads
+        self.ppc = w.pages_per_chunk
+        self.host = L.pool_create(w.num_pages, P, Hkv, d, L.LOC_PINNED_HOST, True, 0,
+                                  device.index or 0)
+        # two slots of `window` pages and two sets of the chunk's own pages (used
+        # by chunks in turn, so chunk c+1 appends while chunk c's drain)
+        n_stage = 2 * window + 2 * self.ppc
+        self.stage = L.pool_create(n_stage, P, Hkv, d, L.LOC_DEVICE, True, 0, device.index or 0)
+        sp = np.array([L.pool_alloc_page(self.stage) for _ in range(n_stage)], dtype=np.int64)
+        self.table = np.array([L.pool_alloc_page(self.host) for _ in range(N * self.ppc)],
+                              dtype=np.int64)
+        i32 = dict(dtype=torch.int32, device=device)
+        heads = np.arange(Hkv, dtype=np.int64)
+
+        def blocks(pages):
+            return (np.asarray(pages, dtype=np.int64)[:, None] * Hkv + heads[None, :]).reshape(-1)
+
+        slots = [sp[:window], sp[window:2 * window]]
+        curs = [sp[2 * window:2 * window + self.ppc], sp[2 * window + self.ppc:]]
+        self.slot_blocks = [torch.tensor(blocks(x), **i32) for x in slots]
+        self.slot_blocks_host = [blocks(x) for x in slots]
+        # the past list of a slot: its pages, the same for every group
+        self.slot_lists = [torch.tensor(np.tile(x, (Hkv, 1)), **i32) for x in slots]
+        self.counts = torch.tensor(np.repeat(np.arange(window + 1)[:, None], Hkv, 1), **i32)
+        self.cur_dev = [torch.tensor(x, **i32) for x in curs]
+        self.cur_blocks = [torch.tensor(blocks(x), **i32) for x in curs]
+        self.cur_blocks_host = [blocks(x) for x in curs]
+        n_seg = max(1, -(-(N - 1) * self.ppc // window))
+        # host blocks of segment s (logical pages [s W, (s + 1) W)), page-major
+        self.seg_blocks, self.seg_blocks_host = [], []
+        for s in range(n_seg):
+            pages = self.table[s * window:(s + 1) * window]
+            self.seg_blocks.append(torch.tensor(blocks(pages), **i32))
+            self.seg_blocks_host.append(blocks(pages))
+        self.own_blocks = torch.tensor(blocks(self.table).reshape(N, -1), **i32)
+        self.own_blocks_host = blocks(self.table).reshape(N, -1)
+        self.copy = torch.cuda.Stream(device=device, priority=-1)
+        self.o_acc = torch.empty((C, Hq, d), dtype=torch.float32, device=device)
+        self.dq_acc = torch.empty_like(self.o_acc)
+        self.delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        self.h2d_bytes = self.d2h_bytes = 0
+
+    def close(self):
+        self.sync()
+        L.pool_destroy(self.stage)
+        L.pool_destroy(self.host)
+
+    def _grads_back(self, src_dev, dst_dev, src_host, dst_host, X):
+        """Gradient blocks of the staging pool into the host pool (zeroed here)."""
+        if self.grad_path == "host":
+            L.grad_writeback(self.stage, self.host, src_host, dst_host, stream=X)
+        else:
+            L.grad_block_add(self.stage, self.host, src_dev, dst_dev, True, stream=X)
+
+    def _segments(self, c):
+        """(mode, first page, pages) of chunk c's calls; the last carries the chunk."""
+        n_past = c * self.ppc
+        segs = [(a, min(self.window, n_past - a)) for a in range(0, n_past, self.window)]
+        if len(segs) <= 1:
+            return [(L.SEG_WHOLE,) + (segs[0] if segs else (0, 0))]
+        modes = [L.SEG_FIRST] + [L.SEG_NEXT] * (len(segs) - 2) + [L.SEG_LAST]
+        return [(m, a, n) for m, (a, n) in zip(modes, segs)]
+
+    def run(self, chunks, outputs=None, backward=True):
+        w = self.w
+        Hkv = w.num_kv_heads
+        comp = torch.cuda.current_stream(self.dev)
+        X = self.copy
+        kv_blk, g_blk = 2 * w.page_size * w.head_dim * 2, 2 * w.page_size * w.head_dim * 4
+        slot_used = [None, None]   # event: last compute on the slot has finished
+        use = 0                    # slots alternate over every segment call
+        cur_free = [None, None]    # event: a chunk-page set's store and write-back are done
+        next_first = None          # chunk c+1's first fetch, issued during chunk c
+        X.wait_stream(comp)
+        scratch = None
+        for c in range(w.num_chunks):
+            x = chunks(c)
+            if outputs is not None:
+                o, lse, dq = outputs(c)
+            else:
+                if scratch is None:
+                    scratch = (torch.empty_like(x["q"]),
+                               torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32,
+                                           device=self.dev), torch.empty_like(x["q"]))
+                o, lse, dq = scratch
+            cb = c % 2
+            cur = self.cur_dev[cb]
+            if cur_free[cb] is not None:
+                comp.wait_event(cur_free[cb])
+            L.kv_append(self.stage, cur, x["k"], x["v"], comp)
+            ev = torch.cuda.Event()
+            ev.record(comp)
+            X.wait_event(ev)
+            L.page_prefetch(self.stage, self.host, self.cur_blocks_host[cb], self.own_blocks_host[c],
+                            stream=X)
+            self.d2h_bytes += self.ppc * Hkv * kv_blk
+            segs = self._segments(c)
+            # every call of the chunk in order: the forward segments, then the
+            # backward ones; each needs its segment's pages in a slot
+            calls = [("fwd",) + sg for sg in segs] + \
+                ([("bwd",) + sg for sg in segs] if backward else [])
+
+            def fetch(a, n):
+                """Segment pages into the next slot on the copy stream; returns
+                (slot, event after the copy)."""
+                nonlocal use
+                slot = use % 2
+                use += 1
+                if slot_used[slot] is not None:
+                    X.wait_event(slot_used[slot])
+                if n:
+                    s = a // self.window
+                    L.page_prefetch(self.host, self.stage, self.seg_blocks_host[s][:n * Hkv],
+                                    self.slot_blocks_host[slot][:n * Hkv], stream=X)
+                    self.h2d_bytes += n * Hkv * kv_blk
+                e = torch.cuda.Event()
+                e.record(X)
+                return slot, e
+
+            def lists(slot, n):
+                return (self.slot_lists[slot], self.counts[n]) if n else (None, None)
+
+            # prefetch one call ahead: call i+1's pages are queued on the copy
+            # stream before call i's gradient write-back, so they arrive while
+            # call i computes
+            fetched = {0: next_first if next_first is not None else fetch(calls[0][2], calls[0][3])}
+            next_first = None
+            for i, (kind, mode, a, n) in enumerate(calls):
+                if i + 1 < len(calls):
+                    fetched[i + 1] = fetch(calls[i + 1][2], calls[i + 1][3])
+                slot, e = fetched.pop(i)
+                comp.wait_event(e)
+                past, cnt = lists(slot, n)
+                if kind == "fwd":
+                    L.chunk_attn_fwd(self.stage, x["q"], o, lse, past, cnt, cur,
+                                     w.softmax_scale, comp, segment=mode, o_acc=self.o_acc)
+                else:
+                    if calls[i - 1][0] == "fwd":
+                        L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, self.delta,
+                                         None, None, cur, w.softmax_scale, comp,
+                                         step=L.BWD_PREPROCESS)
+                    for st in (L.BWD_DKDV, L.BWD_DQ):
+                        L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, self.delta,
+                                         past, cnt, cur, w.softmax_scale, comp,
+                                         step=st, segment=mode, o_acc=self.o_acc,
+                                         dq_acc=self.dq_acc)
+                done = torch.cuda.Event()
+                done.record(comp)
+                slot_used[slot] = done
+                if kind == "bwd" and n:
+                    # the segment's gradients into the host pool, zeroed here
+                    X.wait_event(done)
+                    s = a // self.window
+                    self._grads_back(self.slot_blocks[slot][:n * Hkv],
+                                     self.seg_blocks[s][:n * Hkv],
+                                     self.slot_blocks_host[slot][:n * Hkv],
+                                     self.seg_blocks_host[s][:n * Hkv], X)
+                    if self.grad_path == "gpu":
+                        self.h2d_bytes += n * Hkv * g_blk
+                    self.d2h_bytes += n * Hkv * g_blk
+            last_slot = (use - 1) % 2
+            if c + 1 < w.num_chunks:
+                # the next chunk's first segment comes in while this one drains
+                _, a1, n1 = self._segments(c + 1)[0]
+                next_first = fetch(a1, n1)
+            if backward:
+                X.wait_event(slot_used[last_slot])
+                self._grads_back(self.cur_blocks[cb], self.own_blocks[c], self.cur_blocks_host[cb],
+                                 self.own_blocks_host[c], X)
+                if self.grad_path == "gpu":
+                    self.h2d_bytes += self.ppc * Hkv * g_blk
+                self.d2h_bytes += self.ppc * Hkv * g_blk
+            cur_free[cb] = torch.cuda.Event()
+            cur_free[cb].record(X)
+        comp.wait_stream(X)
+
+    def sync(self):
+        """Waits for the device and, on the host path, every queued addition."""
+        torch.cuda.synchronize(self.dev)
+        if self.grad_path == "host":
+            L.grad_writeback_sync(self.stage)

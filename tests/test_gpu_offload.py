@@ -135,3 +135,41 @@ def test_offloaded_topk_run_matches_device_resident_run():
     assert rel_l2(dk_off, orc["dk"]) <= 1e-2 and rel_l2(dv_off, orc["dv"]) <= 1e-2
     o = np.concatenate([to64(x[0]) for x in outs])
     assert rel_l2(o, orc["o"]) <= 5e-3
+
+
+@pytest.mark.parametrize("window,grad_path", [(3, "gpu"), (20, "gpu"), (3, "host")])
+def test_dense_offload_matches_device_resident_run(window, grad_path):
+    """Dense attention with KV and gradients in pinned host memory and a
+    window of `window` past pages on the device (segments merged in fp32)
+    against the device-resident dense run and the oracle."""
+    from paged_kv_chunk_query_b200.offload import DenseOffloadRun
+    dev = torch.device("cuda", 0)
+    w = synth.Workload("doff", 14, 2, 128, 64, 256, 5, seed=67, shuffle_pages=True)
+    ins = [{k: v.to(dev) for k, v in synth.chunk_inputs(w, c).items()} for c in range(w.num_chunks)]
+    C, Hq = w.chunk_len, w.num_q_heads
+    outs = [(torch.empty_like(x["q"]), torch.empty((Hq, C), dtype=torch.float32, device=dev),
+             torch.empty_like(x["q"])) for x in ins]
+    run = DenseOffloadRun(w, dev, window, grad_path)
+    try:
+        run.run(lambda c: ins[c], lambda c: outs[c])
+        run.sync()
+        assert pk.get_device_status(run.stage) == 0 and pk.get_device_status(run.host) == 0
+        _, gh, _ = pk.pool_views(run.host)
+        ids = torch.tensor(run.table, dtype=torch.long)
+        g = gh[ids].permute(0, 3, 1, 2, 4).reshape(w.context, w.num_kv_heads, 2, w.head_dim)
+        dk_off, dv_off = g[:, :, 0].double().numpy(), g[:, :, 1].double().numpy()
+    finally:
+        run.close()
+    with PagedRun(w) as r:
+        ref = [r.chunk(c, synth.chunk_inputs(w, c)) for c in range(w.num_chunks)]
+        torch.cuda.synchronize()
+        dk_dev, dv_dev = r.grads_by_token(w.context)
+    for c in range(w.num_chunks):
+        for i, key in enumerate(("o", "lse", "dq")):
+            assert rel_l2(to64(outs[c][i]), to64(ref[c][key])) <= 5e-3, (c, key)
+    assert rel_l2(dk_off, dk_dev) <= 5e-3 and rel_l2(dv_off, dv_dev) <= 5e-3
+    inp = synth.sequence_inputs(w)
+    orc = run_sequence(inp["q"], inp["k"], inp["v"], inp["do"], C, w.page_size, w.softmax_scale)
+    assert rel_l2(dk_off, orc["dk"]) <= 1e-2 and rel_l2(dv_off, orc["dv"]) <= 1e-2
+    o = np.concatenate([to64(x[0]) for x in outs])
+    assert rel_l2(o, orc["o"]) <= 5e-3
