@@ -188,6 +188,30 @@ typedef enum oomb_bwd_step {
 oomb_status oomb_chunk_attn_bwd_step(oomb_pool* pool, const oomb_attn_args* args, int32_t step,
                                      void* stream);
 
+/* ---------------------------------------------------------------- projection
+ * Q/K/V projection of one chunk with a paged epilogue ([pt] §2D: the pages a
+ * sparse chunk needs are known once its queries exist, so their transfer can
+ * overlap the rest of its work — here the K/V projection; [es] §2B).
+ *   Y = X W^T, X = d_x [chunk_len][hidden] bf16 (token-major), W = d_w
+ *   [(num_q_heads + 2 num_kv_heads) head_dim][hidden] bf16 with rows: the Q
+ *   heads, then the K heads, then the V heads; fp32 accumulation, outputs
+ *   rounded to bf16 (tcgen05 GEMM, 128 x 128 tiles, TMA, 6 stages).
+ *   part OOMB_PROJ_Q: writes d_q [chunk_len][num_q_heads][head_dim] (if not
+ *     NULL) and, if d_qsum is not NULL, sets d_qsum [num_kv_heads][head_dim]
+ *     fp32 to the sum of the rounded Q over the chunk's rows and each group's
+ *     G heads (q_bar = qsum / (chunk_len G), the Top-K query side).
+ *   part OOMB_PROJ_KV: writes token t's K and V into page d_page_ids[t /
+ *     page_size] of the pool (as oomb_kv_append does), sets those pages' fp32
+ *     mean keys and zero-fills their gradient blocks.
+ *   part OOMB_PROJ_QKV: both in one launch.
+ * Requires a device pool, hidden a multiple of 64, chunk_len a multiple of
+ * page_size, 16-byte aligned X, W and Q.  Page ids out of the pool are
+ * skipped and set bit 0 of the device status word. */
+enum { OOMB_PROJ_Q = 0, OOMB_PROJ_KV = 1, OOMB_PROJ_QKV = 2 };
+oomb_status oomb_qkv_project(oomb_pool* pool, const void* d_x, const void* d_w, int32_t chunk_len,
+                             int32_t hidden, int32_t num_q_heads, int32_t part, void* d_q,
+                             float* d_qsum, const int32_t* d_page_ids, void* stream);
+
 /* ---------------------------------------------------------------- Top-K
  * Page-level selection for one chunk ([pt] §2C, [es] §2B, [it] §2D):
  *   q_bar_g   = fp32 mean of the chunk's rows over the G query heads of group g

@@ -27,6 +27,7 @@ OK, ERR_INVALID_ARG, ERR_OUT_OF_PAGES, ERR_BAD_PAGE, ERR_CUDA, ERR_TIMEOUT, ERR_
 LOC_DEVICE, LOC_PINNED_HOST, LOC_HOST = 0, 1, 2
 BWD_PREPROCESS, BWD_DKDV, BWD_DQ = 0, 1, 2
 SEG_WHOLE, SEG_FIRST, SEG_NEXT, SEG_LAST = 0, 1, 2, 3
+PROJ_Q, PROJ_KV, PROJ_QKV = 0, 1, 2
 
 # Every exported symbol of include/oomb.h.
 EXPORTS = (
@@ -38,6 +39,7 @@ EXPORTS = (
     "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
     "oomb_selftest_wait_limit", "oomb_page_topk_batched_workspace_size", "oomb_page_topk_batched",
     "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists", "oomb_local_pages",
+    "oomb_qkv_project",
 )
 
 
@@ -104,6 +106,7 @@ def load() -> ctypes.CDLL:
         "oomb_grad_block_add": [vp, vp, vp, vp, i32, i32, vp],
         "oomb_prefetch_lists": [vp, vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp],
         "oomb_local_pages": [vp, vp, i32, i32, vp, vp, vp],
+        "oomb_qkv_project": [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):  # completeness is checked by the export test
@@ -361,6 +364,19 @@ def local_pages(pool, page_table, n_past, out_pages, out_count, stream=None):
         pool, _dev_tensor(page_table, torch.int32, "page_table") if n_past else None, n_past,
         window, _dev_tensor(out_pages, torch.int32, "out_pages"),
         _dev_tensor(out_count, torch.int32, "out_count"), _stream(stream)), "oomb_local_pages")
+
+
+def qkv_project(pool, x, w, num_q_heads, part, q=None, qsum=None, page_ids=None, stream=None):
+    """oomb_qkv_project: x [C][hidden] bf16, w [(Hq + 2 Hkv) d][hidden] bf16;
+    part PROJ_Q (q and/or qsum), PROJ_KV (K/V into the pages page_ids, page
+    means, zeroed gradients) or PROJ_QKV."""
+    C, hidden = x.shape
+    _check(load().oomb_qkv_project(
+        pool, _dev_tensor(x, torch.bfloat16, "x"), _dev_tensor(w, torch.bfloat16, "w"), C, hidden,
+        num_q_heads, part, _dev_tensor(q, torch.bfloat16, "q") if q is not None else None,
+        _dev_tensor(qsum, torch.float32, "qsum") if qsum is not None else None,
+        _dev_tensor(page_ids, torch.int32, "page_ids") if page_ids is not None else None,
+        _stream(stream)), "oomb_qkv_project")
 
 
 TOPK_STATIC_SCRATCH_BYTES = 1 << 20
