@@ -133,14 +133,6 @@ def _check(status: int, where: str):
         raise OombError(status, where)
 
 
-def _ptr(t):
-    if t is None:
-        return None
-    if isinstance(t, int):
-        return t
-    return t.data_ptr()
-
-
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None

@@ -73,9 +73,6 @@ class Workload:
     def alloc_seed(self) -> int:
         return self.seed if self.shuffle_pages else 0
 
-    def scaled(self, **kw) -> "Workload":
-        return dataclasses.replace(self, **kw)
-
 
 WORKLOADS = {
     "tiny": Workload("tiny", 4, 1, 64, 16, 64, 8, seed=1000),
