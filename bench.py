@@ -149,7 +149,9 @@ class Run:
         # delta while chunk c+1's preprocess runs
         self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(N)]
         self.side = torch.cuda.Stream(device=device)
+        self.fwd_stream = torch.cuda.Stream(device=device)
         self.concurrent_bwd = True
+        self.fwd_overlap = False
         self.dense_past = [None] + [pt[:c * ppc].repeat(Hkv, 1).contiguous() for c in range(1, N)]
         self.dense_cnt = [None] + [torch.full((Hkv,), c * ppc, dtype=torch.int32, device=device)
                                    for c in range(1, N)]
@@ -198,6 +200,90 @@ class Run:
             ((N - 1) if self.local else 0) + ((N - 1) if self.qtile else 0)
 
     def step(self, timers=None):
+        if self.fwd_overlap and self.concurrent_bwd:
+            return self._step3(timers)
+        return self._step2(timers)
+
+    def _step3(self, timers=None):
+        """One pass over all chunks on three streams: the forward stream runs
+        chunk c's selection, forward and preprocess; then chunk c's dQ (side
+        stream) and dK/dV (main stream) run while the forward stream already
+        takes chunk c+1 (its forward reads only K/V, which no backward writes).
+        Appends stay on the main stream."""
+        pk, w = self.pk, self.w
+        M = torch.cuda.current_stream()
+        S, F = self.side, self.fwd_stream
+
+        def timed(name, fn, st):
+            if timers is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            timers.setdefault(name, []).append((a, b))
+
+        ppc = w.pages_per_chunk
+        S.wait_stream(M)
+        F.wait_stream(M)
+        timed("append", lambda: pk.kv_append(self.pool, self.cur[0], self.inputs[0]["k"],
+                                             self.inputs[0]["v"], M), M)
+        appended = torch.cuda.Event()
+        appended.record(M)
+        for c in range(w.num_chunks):
+            x = self.inputs[c]
+            F.wait_event(appended)    # chunk c's pages (and earlier summaries) appended
+            if c == 0:
+                past, cnt = None, None
+            elif self.local:
+                n_past = c * ppc
+                timed("lists", lambda: pk.local_pages(self.pool, self.page_table_dev[:n_past],
+                                                      n_past, self.loc_p[c], self.loc_n[c],
+                                                      stream=F), F)
+                past, cnt = self.loc_p[c], self.loc_n[c]
+            elif self.qtile:
+                n_past = c * ppc
+                timed("topk", lambda: pk.page_topk_batched(
+                    self.pool, x["q"], self.row_start, 128, self.npast[c], n_past,
+                    self.page_table_dev[:n_past], w.top_k, w.n_recent, self.sel_l[c],
+                    self.sel_p[c], self.sel_n[c], self.ws, stream=F), F)
+                past, cnt = self.sel_p[c], self.sel_n[c]
+            elif self.sparse:
+                n_past = c * ppc
+                timed("topk", lambda: pk.page_topk(
+                    self.pool, x["q"], self.page_table_dev[:n_past], n_past, w.top_k, w.n_recent,
+                    self.sel_l[c], self.sel_p[c], self.sel_n[c], self.ws, stream=F), F)
+                past, cnt = self.sel_p[c], self.sel_n[c]
+            else:
+                past, cnt = self.dense_past[c], self.dense_cnt[c]
+            o, lse, dq = self.o[c], self.lse[c], self.dq[c]
+            sc = w.softmax_scale
+            delta = self.deltas[c]
+            timed("fwd", lambda: pk.chunk_attn_fwd(self.pool, x["q"], o, lse, past, cnt,
+                                                   self.cur[c], sc, F), F)
+            timed("preprocess", lambda: pk.chunk_attn_bwd(
+                self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, F,
+                step=pk.BWD_PREPROCESS), F)
+            if c + 1 < w.num_chunks:
+                xn = self.inputs[c + 1]
+                timed("append", lambda: pk.kv_append(self.pool, self.cur[c + 1], xn["k"], xn["v"],
+                                                     M), M)
+                appended = torch.cuda.Event()
+                appended.record(M)
+            S.wait_stream(F)
+            M.wait_stream(F)
+            timed("dq", lambda: pk.chunk_attn_bwd(
+                self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, S,
+                step=pk.BWD_DQ), S)
+            timed("dkdv", lambda: pk.chunk_attn_bwd(
+                self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, M,
+                step=pk.BWD_DKDV), M)
+        M.wait_stream(S)
+        M.wait_stream(F)
+
+    def _step2(self, timers=None):
         """One pass over all chunks.  With concurrent_bwd, chunk c's dQ launch
         runs on a second stream next to its dK/dV launch (the two only read
         what the forward and preprocess wrote and write disjoint outputs), so
@@ -790,6 +876,8 @@ def main():
     ap.add_argument("--dense-grad-path", choices=["gpu", "host"], default="host",
                     help="gradient write-back of the dense offload run")
     ap.add_argument("--qtile-workload", default="qwen256k_topk_qtile")
+    ap.add_argument("--fwd-overlap", action="store_true",
+                    help="run each chunk's forward on a third stream beside the previous backward")
     ap.add_argument("--serial-bwd", action="store_true",
                     help="run each chunk's dQ launch after its dK/dV launch on one stream")
     ap.add_argument("--offload-workload", default="qwen1m_topk_offload")
@@ -841,6 +929,7 @@ def main():
     clocks = Clocks(local)
     dense = Run(w, False, device)
     dense.concurrent_bwd = not a.serial_bwd
+    dense.fwd_overlap = a.fwd_overlap
     clocks.start()
     ms, kt = time_steps(dense, a.steps, a.warmup, dist_on, device)
     clk = clocks.stop()
@@ -891,6 +980,7 @@ def main():
         ws = synth.WORKLOADS[ws_name]
         sp = Run(ws, True, device)
         sp.concurrent_bwd = not a.serial_bwd
+        sp.fwd_overlap = a.fwd_overlap
         ms_s, kt_s = time_steps(sp, a.steps, a.warmup, dist_on, device)
         sparse_status = pk.get_device_status(sp.pool)
         topk_bytes = 0.0
@@ -924,6 +1014,7 @@ def main():
         wl = synth.WORKLOADS[a.local_workload]
         lr = Run(wl, False, device)
         lr.concurrent_bwd = not a.serial_bwd
+        lr.fwd_overlap = a.fwd_overlap
         ms_l, kt_l = time_steps(lr, a.steps, a.warmup, dist_on, device)
         local_obj = {"workload": wl.name, "window_pages": wl.window,
                      "value": lr.step_flops * world / (ms_l / 1e3) / 1e12, "unit": "TFLOP/s",
@@ -939,6 +1030,7 @@ def main():
         wq = synth.WORKLOADS[a.qtile_workload]
         qr = Run(wq, True, device)
         qr.concurrent_bwd = not a.serial_bwd
+        qr.fwd_overlap = a.fwd_overlap
         ms_q, kt_q = time_steps(qr, a.steps, a.warmup, dist_on, device)
         qtile_obj = {"workload": wq.name, "selection": "Top-K per 128-row query tile",
                      "value": qr.step_flops * world / (ms_q / 1e3) / 1e12, "unit": "TFLOP/s",
