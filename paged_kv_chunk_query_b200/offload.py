@@ -196,6 +196,18 @@ class OffloadRun:
         return h2d, d2h
 
 
+def plan_segments(n_past, window):
+    """The calls that take a chunk's past of n_past pages through a window of
+    `window` pages: [(segment mode, first page, pages)], in order, covering
+    [0, n_past) once; the last call also carries the chunk itself.  No past or
+    a single segment is one whole-key-set call."""
+    segs = [(a, min(window, n_past - a)) for a in range(0, n_past, window)]
+    if len(segs) <= 1:
+        return [(L.SEG_WHOLE,) + (segs[0] if segs else (0, 0))]
+    modes = [L.SEG_FIRST] + [L.SEG_NEXT] * (len(segs) - 2) + [L.SEG_LAST]
+    return [(m, a, n) for m, (a, n) in zip(modes, segs)]
+
+
 class DenseOffloadRun:
     """Dense attention with KV and gradients in pinned host memory and a
     bounded device window ([pt] §2D: pages move between host and GPU on
@@ -283,12 +295,7 @@ class DenseOffloadRun:
 
     def _segments(self, c):
         """(mode, first page, pages) of chunk c's calls; the last carries the chunk."""
-        n_past = c * self.ppc
-        segs = [(a, min(self.window, n_past - a)) for a in range(0, n_past, self.window)]
-        if len(segs) <= 1:
-            return [(L.SEG_WHOLE,) + (segs[0] if segs else (0, 0))]
-        modes = [L.SEG_FIRST] + [L.SEG_NEXT] * (len(segs) - 2) + [L.SEG_LAST]
-        return [(m, a, n) for m, (a, n) in zip(modes, segs)]
+        return plan_segments(c * self.ppc, self.window)
 
     def run(self, chunks, outputs=None, backward=True):
         w = self.w
