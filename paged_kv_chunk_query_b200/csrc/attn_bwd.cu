@@ -756,15 +756,15 @@ bool make_pool_map(CUtensorMap* m, const oomb_pool* pool) {
 template <int D>
 oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape& s, int step,
                        cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             KvCfg<D>::kSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             QCfg<D>::kSmem) != cudaSuccess)
-      return OOMB_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (!once_per_device(attr_done, [] {
+        return cudaFuncSetAttribute(bwd_dkdv_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    KvCfg<D>::kSmem) == cudaSuccess &&
+               cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    QCfg<D>::kSmem) == cudaSuccess;
+      }))
+    return OOMB_ERR_CUDA;
   BwdParams p;
   p.o = static_cast<const __nv_bfloat16*>(a->o);
   p.d_o = static_cast<const __nv_bfloat16*>(a->d_o);

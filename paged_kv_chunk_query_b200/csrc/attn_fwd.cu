@@ -411,13 +411,13 @@ template <int D>
 oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape& s,
                        cudaStream_t stream) {
   using Cfg = FwdCfg<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmem) != cudaSuccess)
-      return OOMB_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (!once_per_device(attr_done, [] {
+        return cudaFuncSetAttribute(attn_fwd_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::kSmem) == cudaSuccess;
+      }))
+    return OOMB_ERR_CUDA;
   CUtensorMap qmap, kvmap;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(s.Hq),

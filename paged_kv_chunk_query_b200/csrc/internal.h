@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 #include <vector>
@@ -70,6 +71,21 @@ struct DeviceGuard {
     if (changed) cudaSetDevice(prev);
   }
 };
+
+// Runs `set` (a per-device setting such as a kernel's shared-memory limit) the
+// first time it is needed on the current device and remembers success in
+// `done` (one bit per device ordinal < 64; later devices run it every call).
+// Concurrent first calls may both run `set`, which must be idempotent.
+template <class F>
+inline bool once_per_device(std::atomic<uint64_t>& done, F set) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+  if (!set()) return false;
+  if (bit) done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
 
 // Common validation of an attention call; fills the derived sizes.
 struct AttnShape {

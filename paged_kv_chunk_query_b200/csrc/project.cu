@@ -276,13 +276,12 @@ extern "C" oomb_status oomb_qkv_project(oomb_pool* pool, const void* d_x, const 
   if (do_kv && !d_page_ids) return OOMB_ERR_INVALID_ARG;
   if (!aligned16(d_x) || !aligned16(d_w) || (d_q && !aligned16(d_q))) return OOMB_ERR_INVALID_ARG;
   DeviceGuard guard(d.device);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kProjSmem) != cudaSuccess)
-      return OOMB_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (!once_per_device(attr_done, [] {
+        return cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kProjSmem) == cudaSuccess;
+      }))
+    return OOMB_ERR_CUDA;
   const int nq = num_q_heads * D, n_out = nq + 2 * Hkv * D;
   CUtensorMap xmap, wmap;
   if (!make_rows_map(&xmap, d_x, hidden, chunk_len) || !make_rows_map(&wmap, d_w, hidden, n_out))
