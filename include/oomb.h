@@ -195,7 +195,7 @@ oomb_status oomb_chunk_attn_bwd_step(oomb_pool* pool, const oomb_attn_args* args
  *   Y = X W^T, X = d_x [chunk_len][hidden] bf16 (token-major), W = d_w
  *   [(num_q_heads + 2 num_kv_heads) head_dim][hidden] bf16 with rows: the Q
  *   heads, then the K heads, then the V heads; fp32 accumulation, outputs
- *   rounded to bf16 (tcgen05 GEMM, 128 x 128 tiles, TMA, 6 stages).
+ *   rounded to bf16 (tcgen05 GEMM, 128 x 256 tiles, TMA, 4 stages).
  *   part OOMB_PROJ_Q: writes d_q [chunk_len][num_q_heads][head_dim] (if not
  *     NULL) and, if d_qsum is not NULL, sets d_qsum [num_kv_heads][head_dim]
  *     fp32 to the sum of the rounded Q over the chunk's rows and each group's

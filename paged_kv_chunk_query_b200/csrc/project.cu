@@ -11,8 +11,10 @@
 //
 // Y = X W^T with X [C][hidden] bf16 and W [(Hq + 2 Hkv) d][hidden] bf16 (rows:
 // Q heads, K heads, V heads), fp32 accumulation, outputs rounded to bf16.
-// One CTA per 128 x 128 output tile: warp 0 loads X and W slices of 64 hidden
-// elements by TMA into a ring of 6 stages, warp 1 issues the UMMAs (both
+// One CTA per 128 x 256 output tile (tokens x outputs; each k-step loads 48 KB
+// for 128 x 256 x 64 products, a quarter less L2 traffic per FLOP than 128 x
+// 128): warp 0 loads X and W slices of 64 hidden elements by TMA into a ring
+// of 4 stages, warp 1 issues the UMMAs (both
 // operands K-major in shared memory, accumulator in TMEM), warps 2-5 read the
 // accumulator (TMEM lane = token) and write Q rows, or K/V rows into pool
 // pages, and add their sums: the page means of K (over the page's P tokens)
@@ -25,8 +27,8 @@ namespace {
 
 using namespace oomb;
 
-constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kStages = 6;
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 4;
 constexpr int kTileA = kBM * kBK * 2, kTileB = kBN * kBK * 2;
 constexpr int kStageBytes = kTileA + kTileB;
 constexpr int kProjSmem = kStages * kStageBytes + 1024;
@@ -251,10 +253,10 @@ __global__ void proj_prepare_kernel(const int32_t* __restrict__ page_ids, float*
   }
 }
 
-bool make_rows_map(CUtensorMap* m, const void* base, int inner, int rows) {
+bool make_rows_map(CUtensorMap* m, const void* base, int inner, int rows, int box_rows) {
   const uint64_t dims[2] = {static_cast<uint64_t>(inner), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(inner) * 2};
-  const uint32_t box[2] = {kBK, kBM};
+  const uint32_t box[2] = {kBK, static_cast<uint32_t>(box_rows)};
   return make_bf16_map(m, base, 2, dims, strides, box);
 }
 
@@ -284,7 +286,8 @@ extern "C" oomb_status oomb_qkv_project(oomb_pool* pool, const void* d_x, const 
     return OOMB_ERR_CUDA;
   const int nq = num_q_heads * D, n_out = nq + 2 * Hkv * D;
   CUtensorMap xmap, wmap;
-  if (!make_rows_map(&xmap, d_x, hidden, chunk_len) || !make_rows_map(&wmap, d_w, hidden, n_out))
+  if (!make_rows_map(&xmap, d_x, hidden, chunk_len, kBM) ||
+      !make_rows_map(&wmap, d_w, hidden, n_out, kBN))
     return OOMB_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ProjParams p;
