@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(320, 1)
   };
 
   __shared__ uint64_t bar_kv, bar_qf[Cfg::kNS], bar_qe[Cfg::kNS];
-  __shared__ uint64_t bar_st, bar_sl, bar_dpt, bar_pds, bar_acc, bar_drain;
+  __shared__ uint64_t bar_st, bar_sl, bar_dpt, bar_p, bar_ds, bar_acc, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh, q_issued_sh, q_used_sh, kv_issued_sh;
 
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&bar_st, 1);
     mbar_init(&bar_sl, 8);
     mbar_init(&bar_dpt, 1);
-    mbar_init(&bar_pds, 8);
+    mbar_init(&bar_p, 8);
+    mbar_init(&bar_ds, 8);
     mbar_init(&bar_acc, 1);
     mbar_init(&bar_drain, 1);
     fence_mbar_init();
@@ -201,7 +202,8 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 9) {
     if (lane == 0) {
       // Order per query tile i: S^T_{i+1} as soon as the compute warps hold S^T_i
-      // in registers; dV_i, dK_i once P^T_i, dS^T_i are in TMEM; then dP^T_{i+1}.
+      // in registers; dV_i once P^T_i is in TMEM, dK_i once dS^T_i is; then
+      // dP^T_{i+1}.
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
@@ -242,15 +244,19 @@ __global__ void __launch_bounds__(320, 1)
           if (!(ok = mbar_wait(&bar_sl, i & 1, abort_flag))) break;
           if (!(ok = issue_s(i + 1))) break;
         }
-        if (!(ok = mbar_wait(&bar_pds, i & 1, abort_flag))) break;
+        // dV += P^T_i dO_i as soon as P^T_i is in TMEM (while the compute warps
+        // still form dS^T_i); dK += dS^T_i Q_i once dS^T_i is there.  Both A
+        // operands are packed in the (already read) dP^T columns.
+        if (!(ok = mbar_wait(&bar_p, i & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQ(s)), do_addr = smem_u32(sDO(s));
-        // dV += P^T_i dO_i ; dK += dS^T_i Q_i  (A operands packed in the dP^T columns)
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           umma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColDPT + (kk / 4) * 64 + (kk % 4) * 8,
                   sw128_desc(do_addr + kk * 16 * 128, kTile * 128, 1024), idesc_acc,
                   (i > 0 || kk > 0) ? 1u : 0u);
+        if (!(ok = mbar_wait(&bar_ds, i & 1, abort_flag))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPT + (kk / 4) * 64 + 32 + (kk % 4) * 8,
@@ -319,6 +325,19 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(tmem + lane_off + Cfg::kColDPT + cs, dp);
       tmem_ld32(tmem + lane_off + Cfg::kColDPT + cs + 32, dp + 32);
       tmem_ld_wait();
+      {
+        // P^T (bf16) into this half's first 32 dP^T columns, already read: the
+        // dV product can start while dS^T is formed
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+        tmem_st16(tmem + lane_off + Cfg::kColDPT + cs, pk);
+        tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 16, pk + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p);
+      }
       const float* Dl = sDl(s) + cs;
       uint32_t dsk[32];
 #pragma unroll
@@ -336,18 +355,13 @@ __global__ void __launch_bounds__(320, 1)
         dsk[2 * e4] = pack_bf16(ds[0], ds[1]);
         dsk[2 * e4 + 1] = pack_bf16(ds[2], ds[3]);
       }
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-      // P^T and dS^T (bf16) into this half's dP^T columns, already read
-      tmem_st16(tmem + lane_off + Cfg::kColDPT + cs, pk);
-      tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 16, pk + 16);
+      // dS^T (bf16) into this half's last 32 dP^T columns, already read
       tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 32, dsk);
       tmem_st16(tmem + lane_off + Cfg::kColDPT + cs + 48, dsk + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_pds);
+      if (lane == 0) mbar_arrive(&bar_ds);
     }
     if (ok && n_iter > 0) ok = warp_wait(&bar_acc, 0, abort_flag);
     if (!ok) {
