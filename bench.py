@@ -58,6 +58,24 @@ def pairs_of_chunk(C, n_past_keys):
     return C * n_past_keys + C * (C + 1) // 2
 
 
+def chunk_past_keys(w, c, sparse):
+    """Past keys each row of chunk c attends to: every earlier token (dense),
+    the kept pages (Top-K: min(K, n_past - R) + min(R, n_past) pages, per
+    chunk or per query tile alike), or the last `window` pages (recent-only)."""
+    ppc, P = w.pages_per_chunk, w.page_size
+    if sparse and c:
+        return (min(w.top_k, max(0, c * ppc - w.n_recent)) + min(w.n_recent, c * ppc)) * P
+    if w.window > 0:
+        return min(w.window, c * ppc) * P
+    return c * w.chunk_len
+
+
+def step_pairs(w, sparse):
+    """(query row, key) pairs of one step over all chunks and query heads."""
+    return sum(pairs_of_chunk(w.chunk_len, chunk_past_keys(w, c, sparse)) * w.num_q_heads
+               for c in range(w.num_chunks))
+
+
 class Clocks:
     """Samples nvidia-smi every 200 ms while running."""
 
@@ -182,13 +200,7 @@ class Run:
         # algorithmic FLOPs per chunk (per kernel class) and per step
         self.flops = {"fwd": [], "dkdv": [], "dq": []}
         for c in range(N):
-            if sparse and c:
-                n_keys = (min(w.top_k, max(0, c * ppc - w.n_recent)) + min(w.n_recent, c * ppc)) * P
-            elif self.local:
-                n_keys = min(w.window, c * ppc) * P
-            else:
-                n_keys = c * C
-            pairs = pairs_of_chunk(C, n_keys) * Hq
+            pairs = pairs_of_chunk(C, chunk_past_keys(w, c, sparse)) * Hq
             self.flops["fwd"].append(4.0 * pairs * d)
             self.flops["dkdv"].append(8.0 * pairs * d)
             self.flops["dq"].append(2.0 * pairs * d)

@@ -56,3 +56,26 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_flop_accounting_matches_the_published_workload_figures():
+    """pairs and FLOPs per step (fwd 4 pairs d, bwd 10 pairs d) against the
+    figures derived for each workload: 32K dense, 256K dense, 256K Top-K,
+    1M Top-K offload."""
+    import bench
+    from paged_kv_chunk_query_b200 import synth
+    W = synth.WORKLOADS
+    cases = [("qwen32k", False, 536_887_296, 26.94),
+             ("qwen256k", False, 34_359_869_440, 1724.0),
+             ("qwen256k_topk", True, 1_626_472_448, 81.6),
+             ("qwen1m_topk_offload", True, 6_559_367_168, 329.1)]
+    for name, sparse, pairs_per_head, tflop in cases:
+        w = W[name]
+        pairs = bench.step_pairs(w, sparse)
+        assert pairs == pairs_per_head * w.num_q_heads, name
+        total = 14.0 * pairs * w.head_dim / 1e12
+        assert abs(total - tflop) <= 0.06 * max(1.0, tflop / 100), (name, total)
+    # a recent-only window covering the whole past is dense
+    w = W["qwen256k"]
+    assert bench.step_pairs(synth.Workload("x", 28, 4, 128, 64, 4096, 64, seed=1,
+                                           window=4096), False) == bench.step_pairs(w, False)
