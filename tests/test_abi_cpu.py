@@ -136,3 +136,39 @@ def test_topk_workspace_size_formula():
     # query-mean partials (128 slices), q_bar, then the 64-bit page keys
     assert ws == 128 * 4 * 128 * 4 + 4 * 128 * 4 + ((4 * 4094 * 8 + 255) // 256) * 256
     assert L.page_topk_workspace_size(0, 28, 4, 128, 10) == 0
+
+
+def test_newer_entry_points_reject_host_pools_without_touching_cuda():
+    """Block moves, list builders, batched / static Top-K and the projection
+    check their pools' locations on the host first."""
+    lib = L.load()
+    pool = L.pool_create(8, 16, 1, 64, L.LOC_HOST, True, 0)
+    try:
+        assert lib.oomb_block_copy(pool, pool, None, None, 1, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_grad_block_add(pool, pool, None, None, 1, 1, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_prefetch_lists(pool, pool, None, None, 4, None, 0, None, None, None,
+                                       None, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_local_pages(pool, None, 0, 4, None, None, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_page_topk_batched(pool, None, 64, 4, 1, None, 64, None, 0, None, 4, 2,
+                                          None, None, None, None, None, 0,
+                                          None) == L.ERR_INVALID_ARG
+        assert lib.oomb_page_topk_static(pool, None, 64, 4, None, 0, 4, 2, None, None, None,
+                                         None, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_qkv_project(pool, None, None, 128, 64, 4, L.PROJ_QKV, None, None, None,
+                                    None) == L.ERR_INVALID_ARG
+        assert lib.oomb_block_copy(None, pool, None, None, 0, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_selftest_wait_limit(pool, None) == L.ERR_INVALID_ARG
+    finally:
+        L.pool_destroy(pool)
+
+
+def test_batched_topk_workspace_size_formula():
+    def a256(x):
+        return (x + 255) // 256 * 256
+    B, Hkv, d, mp = 64, 4, 128, 4032
+    want = a256(B * 128 * Hkv * d * 4) + a256(B * Hkv * d * 4) + a256(B * Hkv * mp * 8)
+    assert L.page_topk_batched_workspace_size(B, Hkv, d, mp) == want
+    # one problem is the per-chunk workspace
+    assert L.page_topk_batched_workspace_size(1, Hkv, d, mp) == \
+        L.page_topk_workspace_size(4096, 28, Hkv, d, mp)
+    assert L.page_topk_batched_workspace_size(0, Hkv, d, mp) == 0
