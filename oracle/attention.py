@@ -250,3 +250,53 @@ def chunk_rows_forward(q_rows, row_pos, k_keys, v_keys, key_pos, scale):
     s = np.where(keep, scale * (q_rows @ k_keys.T), -np.inf)
     p, lse = _softmax_rows(s)
     return p @ v_keys, lse
+
+
+def chunk_rows_backward(q_rows, do_rows, row_pos, k_keys, v_keys, key_pos, scale):
+    """Forward and dQ for a few sampled rows of ONE head (the sizes where a
+    whole chunk is too slow in fp64).
+
+    Same arguments as :func:`chunk_rows_forward` plus dO of those rows
+    ``[R][d]``.  dq_i needs only row i's own softmax: D_i = dO_i . O_i,
+    dP_ij = dO_i . v_j, dS_ij = P_ij (dP_ij - D_i), dq_i = scale sum_j dS_ij k_j.
+    Returns O ``[R][d]``, LSE ``[R]`` and dQ ``[R][d]``."""
+    q_rows, do_rows = _f64(q_rows), _f64(do_rows)
+    k_keys, v_keys = _f64(k_keys), _f64(v_keys)
+    keep = np.asarray(key_pos)[None, :] <= np.asarray(row_pos)[:, None]
+    s = np.where(keep, scale * (q_rows @ k_keys.T), -np.inf)
+    p, lse = _softmax_rows(s)
+    o = p @ v_keys
+    D = np.sum(do_rows * o, axis=1)
+    dp = do_rows @ v_keys.T
+    ds = p * (dp - D[:, None])
+    return o, lse, scale * (ds @ k_keys)
+
+
+def chunk_keys_backward(q, do, row_pos, k_keys, v_keys, key_pos, key_idx, scale):
+    """One chunk's contribution to dK and dV of a few sampled keys of ONE
+    KV-head group, summed over the group's query heads.
+
+    q, do ``[R][G][d]``: every query row of the chunk for the G heads of the
+    group (absolute positions ``row_pos`` ``[R]``); k_keys, v_keys ``[n][d]``:
+    every key the chunk's rows may see (positions ``key_pos``; row i sees key
+    j iff key_pos[j] <= row_pos[i]); ``key_idx``: indices into those keys.
+    Each head's softmax needs every key (LSE_i and D_i = dO_i . O_i);
+    then, for the sampled keys j only, dK_j = scale sum_i dS_ij q_i and
+    dV_j = sum_i P_ij dO_i.  Returns dK, dV ``[len(key_idx)][d]``."""
+    q, do = _f64(q), _f64(do)
+    k_keys, v_keys = _f64(k_keys), _f64(v_keys)
+    key_idx = np.asarray(key_idx, dtype=np.int64)
+    keep = np.asarray(key_pos)[None, :] <= np.asarray(row_pos)[:, None]
+    dk = np.zeros((len(key_idx), k_keys.shape[1]))
+    dv = np.zeros((len(key_idx), v_keys.shape[1]))
+    for h in range(q.shape[1]):
+        s = np.where(keep, scale * (q[:, h, :] @ k_keys.T), -np.inf)
+        p, _ = _softmax_rows(s)
+        o = p @ v_keys
+        D = np.sum(do[:, h, :] * o, axis=1)
+        p_j = p[:, key_idx]
+        dp_j = do[:, h, :] @ v_keys[key_idx].T
+        ds_j = p_j * (dp_j - D[:, None])
+        dk += scale * (ds_j.T @ q[:, h, :])
+        dv += p_j.T @ do[:, h, :]
+    return dk, dv

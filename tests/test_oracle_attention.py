@@ -9,7 +9,8 @@ import pytest
 import torch
 
 from oracle.attention import (causal_attention, causal_attention_backward,
-                              chunk_backward, chunk_forward, chunk_rows_forward)
+                              chunk_backward, chunk_forward, chunk_keys_backward,
+                              chunk_rows_backward, chunk_rows_forward)
 from oracle.recurrent import run_sequence, run_sequence_blocks
 from oracle.sparse import topk_for_chunk
 
@@ -296,3 +297,72 @@ def test_row_block_topk_is_the_selection_of_the_block_rows():
             want, _ = topk_for_chunk(q[rows], k[:c * C], P, 2, 1)
             assert r["selected"][c][b] == want
 
+
+
+def _torch_positions_attention(q, k, v, row_pos, key_pos, scale):
+    """fp64 torch SDPA of rows [R][Hh][d] against keys [n][d] (one KV head)
+    with the mask key_pos <= row_pos; tensors require grad."""
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(k, requires_grad=True)
+    tv = torch.tensor(v, requires_grad=True)
+    mask = torch.tensor(np.asarray(key_pos)[None, :] <= np.asarray(row_pos)[:, None])
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq.permute(1, 0, 2), tk[None], tv[None], attn_mask=mask[None], scale=scale)
+    return tq, tk, tv, o.permute(1, 0, 2)
+
+
+def test_sampled_rows_backward_matches_torch_autograd():
+    """O, LSE and dQ of sampled rows against torch SDPA + autograd on the same
+    position mask: rows at the chunk start (only past keys + itself), inside,
+    and at the end; keys out of order in memory."""
+    n, d, scale = 70, 16, 0.29
+    rng = np.random.default_rng(131)
+    key_pos = rng.permutation(n)                       # absolute positions, shuffled
+    row_pos = np.array([40, 41, 55, 69])
+    q, do = _rand((4, d), 132), _rand((4, d), 133)
+    k, v = _rand((n, d), 134), _rand((n, d), 135)
+    o, lse, dq = chunk_rows_backward(q, do, row_pos, k, v, key_pos, scale)
+    tq, tk, tv, ref = _torch_positions_attention(q[:, None], k, v, row_pos, key_pos, scale)
+    np.testing.assert_allclose(o, ref[:, 0].detach().numpy(), rtol=1e-12, atol=1e-13)
+    (ref[:, 0] * torch.tensor(do)).sum().backward()
+    np.testing.assert_allclose(dq, tq.grad[:, 0].numpy(), rtol=1e-10, atol=1e-12)
+    s = (torch.tensor(q) @ torch.tensor(k).T) * scale
+    s = s.masked_fill(~torch.tensor(key_pos[None, :] <= row_pos[:, None]), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=1).numpy(), rtol=1e-12)
+
+
+def test_sampled_keys_backward_matches_torch_autograd_and_finite_differences():
+    """dK/dV of sampled keys of one group (three heads, causal chunk over a
+    past) against torch autograd of the whole set, and against central
+    finite differences of sum(O * dO) on two of the sampled keys."""
+    past, C, G, d, scale = 24, 12, 3, 8, 0.41
+    n = past + C
+    key_pos = np.arange(n)
+    row_pos = past + np.arange(C)
+    q, do = _rand((C, G, d), 141), _rand((C, G, d), 142)
+    k, v = _rand((n, d), 143), _rand((n, d), 144)
+    idx = np.array([0, 7, 23, 24, 30, 35])            # past and current-chunk keys
+    dk, dv = chunk_keys_backward(q, do, row_pos, k, v, key_pos, idx, scale)
+    tq, tk, tv, ref = _torch_positions_attention(q, k, v, row_pos, key_pos, scale)
+    (ref * torch.tensor(do)).sum().backward()
+    np.testing.assert_allclose(dk, tk.grad.numpy()[idx], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy()[idx], rtol=1e-10, atol=1e-12)
+
+    def loss(kk, vv):
+        o = np.stack([chunk_rows_forward(q[:, h], row_pos, kk, vv, key_pos, scale)[0]
+                      for h in range(G)], 1)
+        return float(np.sum(o * do))
+    h = 1e-6
+    for j, which in ((1, "k"), (4, "v")):
+        for e in range(d):
+            kp, km, vp, vm = k.copy(), k.copy(), v.copy(), v.copy()
+            if which == "k":
+                kp[idx[j], e] += h
+                km[idx[j], e] -= h
+                fd = (loss(kp, v) - loss(km, v)) / (2 * h)
+                assert abs(fd - dk[j, e]) <= 1e-6 * max(1.0, abs(dk[j, e]))
+            else:
+                vp[idx[j], e] += h
+                vm[idx[j], e] -= h
+                fd = (loss(k, vp) - loss(k, vm)) / (2 * h)
+                assert abs(fd - dv[j, e]) <= 1e-6 * max(1.0, abs(dv[j, e]))
