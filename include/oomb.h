@@ -252,7 +252,10 @@ oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk
  * device current); make that first call before any stream capture.  All calls
  * share the one array: calls that overlap on the GPU (different streams) race
  * on it and must be ordered by the caller.  No scratch word needs clearing:
- * each call writes what it reads. */
+ * each call writes what it reads.  The looked-up address is kept per device
+ * ordinal for the life of the process, so resetting a device
+ * (cudaDeviceReset, or tearing down and re-creating its primary context)
+ * while this library is loaded is not supported for this entry point. */
 #define OOMB_TOPK_STATIC_SCRATCH_BYTES (1u << 20)
 oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* d_q, int32_t chunk_len,
                                   int32_t num_q_heads, const int32_t* d_page_table,
@@ -330,14 +333,26 @@ oomb_status oomb_page_prefetch(const oomb_pool* src_pool, oomb_pool* dst_pool,
  * pool with up to 16 CPU threads, in submission order, without holding up the
  * stream.  The call itself blocks only while both slots are still being
  * added (OOMB_ERR_TIMEOUT after 120 s).  Destination blocks must be distinct
- * within one call.  The host gradients include a call's blocks once
- * oomb_grad_writeback_sync() has returned OOMB_OK. */
+ * within one call: a repeated destination returns OOMB_ERR_INVALID_ARG (an id
+ * outside its pool OOMB_ERR_BAD_PAGE) before any CUDA call.  The host
+ * gradients include a call's blocks once oomb_grad_writeback_sync() has
+ * returned OOMB_OK.
+ * Failures: if a device -> host copy cannot be queued, the call returns
+ * OOMB_ERR_CUDA, adds nothing, and leaves every device block as it was (the
+ * zero-fills are queued only after all copies were); the staging slot is
+ * reused only once copies already queued into it have finished.  If a copy
+ * fails on the device, the worker skips that call's additions and the next
+ * oomb_grad_writeback_sync() returns OOMB_ERR_CUDA.  If a zero-fill cannot be
+ * queued, the additions still happen but some device blocks may keep their
+ * values (OOMB_ERR_CUDA). */
 oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* host_pool,
                                 const int32_t* h_src_blocks, const int32_t* h_dst_blocks,
                                 int32_t n_blocks, void* stream);
 /* Waits until every gradient addition queued by oomb_grad_writeback for this
  * device pool has been applied to the host pool (OOMB_ERR_TIMEOUT after
- * timeout_us microseconds). */
+ * timeout_us microseconds).  OOMB_ERR_CUDA: the copy of some call since the
+ * previous sync failed and that call's blocks were not added (the report is
+ * cleared by this call). */
 oomb_status oomb_grad_writeback_sync(oomb_pool* device_pool, int64_t timeout_us);
 
 /* ---------------------------------------------------------------- block moves with device lists
@@ -406,6 +421,15 @@ const char* oomb_status_string(oomb_status status);
  * word, exactly as a kernel whose arrival was lost would.  Device or
  * pinned-host pools only. */
 oomb_status oomb_selftest_wait_limit(oomb_pool* pool, void* stream);
+/* Self-test of the gradient write-back worker (no counterpart in the paper;
+ * host only, makes no CUDA call): a staging slot of n_blocks blocks of
+ * block_floats floats, all 1.0, goes through the worker into host_grad
+ * blocks 0 .. n_blocks-1, its copy reported as completed (fail_copy == 0) or
+ * as failed (fail_copy != 0).  Returns what oomb_grad_writeback_sync would:
+ * OOMB_OK with host_grad incremented by 1.0, or OOMB_ERR_CUDA with host_grad
+ * untouched. */
+oomb_status oomb_selftest_writeback_copy(float* host_grad, int32_t n_blocks,
+                                         int32_t block_floats, int32_t fail_copy);
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t oomb_version(void);
 

@@ -39,7 +39,7 @@ EXPORTS = (
     "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
     "oomb_selftest_wait_limit", "oomb_page_topk_batched_workspace_size", "oomb_page_topk_batched",
     "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists", "oomb_local_pages",
-    "oomb_qkv_project",
+    "oomb_qkv_project", "oomb_selftest_writeback_copy",
 )
 
 
@@ -107,6 +107,7 @@ def load() -> ctypes.CDLL:
         "oomb_prefetch_lists": [vp, vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp],
         "oomb_local_pages": [vp, vp, i32, i32, vp, vp, vp],
         "oomb_qkv_project": [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp],
+        "oomb_selftest_writeback_copy": [vp, i32, i32, i32],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):  # completeness is checked by the export test

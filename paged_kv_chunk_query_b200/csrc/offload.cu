@@ -37,6 +37,19 @@ bool blocks_valid(const oomb_pool* pool, const int32_t* blocks, int n) {
   return true;
 }
 
+// One pass over a destination list, in order: OOMB_ERR_BAD_PAGE at the first
+// id outside the pool, OOMB_ERR_INVALID_ARG at the first id seen twice.
+oomb_status distinct_blocks(const oomb_pool* pool, const int32_t* blocks, int n) {
+  const int64_t nb = static_cast<int64_t>(pool->desc.num_pages) * pool->desc.num_kv_heads;
+  std::vector<uint8_t> seen(static_cast<size_t>(nb), 0);
+  for (int i = 0; i < n; ++i) {
+    if (blocks[i] < 0 || blocks[i] >= nb) return OOMB_ERR_BAD_PAGE;
+    if (seen[blocks[i]]) return OOMB_ERR_INVALID_ARG;
+    seen[blocks[i]] = 1;
+  }
+  return OOMB_OK;
+}
+
 // Runs [i, j) with src and dst both consecutive.
 template <class F>
 void for_each_run(const int32_t* src, const int32_t* dst, int n, F f) {
@@ -60,11 +73,13 @@ int host_threads() {
 // in turn, and one worker thread that, job by job in submission order, waits
 // for a slot's device->host copy to finish and adds the slot into the host
 // pool with several CPU threads.  The worker never calls back into a stream,
-// so the copy stream is not held up by the additions.
+// so the copy stream is not held up by the additions.  A job whose copy did
+// not complete is not added: the worker only frees its slot and records the
+// failure, which the next oomb_grad_writeback_sync reports.
 struct oomb_wb_engine {
   struct Job {
     int slot;
-    float* host_grad;
+    float* host_grad;           // nullptr: nothing to add, only wait and free the slot
     std::vector<int32_t> dst;
     size_t block_floats;
   };
@@ -73,16 +88,25 @@ struct oomb_wb_engine {
   std::deque<Job> jobs;
   bool stop = false;
   int pending = 0;              // jobs submitted and not yet added
+  bool failed = false;          // a job's copy failed since the last sync
   float* slot_ptr[2] = {nullptr, nullptr};
   size_t slot_bytes[2] = {0, 0};
   bool slot_busy[2] = {false, false};
   cudaEvent_t slot_ev[2] = {nullptr, nullptr};
   int next_slot = 0;
   int device = 0;
+  // host-only self-test: no CUDA call; every copy "completes" with this status
+  bool fake_copies = false;
+  cudaError_t fake_copy_status = cudaSuccess;
   std::thread worker;
 
+  cudaError_t wait_copy(int slot) {
+    if (fake_copies) return fake_copy_status;
+    return cudaEventSynchronize(slot_ev[slot]);
+  }
+
   void run() {
-    cudaSetDevice(device);
+    if (!fake_copies) cudaSetDevice(device);
     while (true) {
       Job job;
       {
@@ -92,28 +116,50 @@ struct oomb_wb_engine {
         job = std::move(jobs.front());
         jobs.pop_front();
       }
-      cudaEventSynchronize(slot_ev[job.slot]);
-      const float* stage = slot_ptr[job.slot];
-      const size_t n = job.dst.size();
-      const int T = std::max(1, std::min<int>(host_threads(), static_cast<int>(n)));
-      auto work = [&](int t) {
-        for (size_t b = t; b < n; b += T) {
-          float* out = job.host_grad + static_cast<size_t>(job.dst[b]) * job.block_floats;
-          const float* in = stage + b * job.block_floats;
-          for (size_t e = 0; e < job.block_floats; ++e) out[e] += in[e];
-        }
-      };
-      std::vector<std::thread> pool;
-      for (int t = 1; t < T; ++t) pool.emplace_back(work, t);
-      work(0);
-      for (auto& th : pool) th.join();
+      const bool copied = wait_copy(job.slot) == cudaSuccess;
+      if (copied && job.host_grad) {
+        const float* stage = slot_ptr[job.slot];
+        const size_t n = job.dst.size();
+        const int T = std::max(1, std::min<int>(host_threads(), static_cast<int>(n)));
+        auto work = [&](int t) {
+          for (size_t b = t; b < n; b += T) {
+            float* out = job.host_grad + static_cast<size_t>(job.dst[b]) * job.block_floats;
+            const float* in = stage + b * job.block_floats;
+            for (size_t e = 0; e < job.block_floats; ++e) out[e] += in[e];
+          }
+        };
+        std::vector<std::thread> pool;
+        for (int t = 1; t < T; ++t) pool.emplace_back(work, t);
+        work(0);
+        for (auto& th : pool) th.join();
+      }
       {
         std::lock_guard<std::mutex> lk(mu);
+        if (!copied) failed = true;
         slot_busy[job.slot] = false;
         --pending;
       }
       cv.notify_all();
     }
+  }
+
+  // Waits for every queued job; reports (and clears) a failed copy.
+  oomb_status sync(int64_t timeout_us) {
+    std::unique_lock<std::mutex> lk(mu);
+    if (!cv.wait_for(lk, std::chrono::microseconds(timeout_us), [&] { return pending == 0; }))
+      return OOMB_ERR_TIMEOUT;
+    const bool f = failed;
+    failed = false;
+    return f ? OOMB_ERR_CUDA : OOMB_OK;
+  }
+
+  void shutdown() {
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      stop = true;
+    }
+    cv.notify_all();
+    if (worker.joinable()) worker.join();
   }
 };
 
@@ -122,12 +168,7 @@ namespace oomb {
 void destroy_wb_engine(oomb_pool* pool) {
   oomb_wb_engine* e = pool->wb;
   if (!e) return;
-  {
-    std::lock_guard<std::mutex> lk(e->mu);
-    e->stop = true;
-  }
-  e->cv.notify_all();
-  if (e->worker.joinable()) e->worker.join();
+  e->shutdown();
   for (int i = 0; i < 2; ++i) {
     if (e->slot_ptr[i]) cudaFreeHost(e->slot_ptr[i]);
     if (e->slot_ev[i]) cudaEventDestroy(e->slot_ev[i]);
@@ -199,13 +240,15 @@ extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* ho
   if (!device_pool || !host_pool || n_blocks < 0) return OOMB_ERR_INVALID_ARG;
   if (n_blocks == 0) return OOMB_OK;
   if (!h_src_blocks || !h_dst_blocks) return OOMB_ERR_INVALID_ARG;
+  if (!same_shape(device_pool, host_pool)) return OOMB_ERR_INVALID_ARG;
+  if (!blocks_valid(device_pool, h_src_blocks, n_blocks)) return OOMB_ERR_BAD_PAGE;
+  // the worker's CPU threads add different blocks at once: a destination
+  // listed twice would lose one of its additions
+  const oomb_status dst_ok = distinct_blocks(host_pool, h_dst_blocks, n_blocks);
+  if (dst_ok != OOMB_OK) return dst_ok;
   if (device_pool->desc.location != OOMB_LOC_DEVICE ||
       host_pool->desc.location != OOMB_LOC_PINNED_HOST || !device_pool->grad || !host_pool->grad)
     return OOMB_ERR_INVALID_ARG;
-  if (!same_shape(device_pool, host_pool)) return OOMB_ERR_INVALID_ARG;
-  if (!blocks_valid(device_pool, h_src_blocks, n_blocks) ||
-      !blocks_valid(host_pool, h_dst_blocks, n_blocks))
-    return OOMB_ERR_BAD_PAGE;
   oomb::DeviceGuard guard(device_pool->desc.device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bfloats = device_pool->block_elems();
@@ -244,8 +287,34 @@ extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* ho
     done += j - i;
     i = j;
   }
-  ok = ok && cudaEventRecord(e->slot_ev[slot], s) == cudaSuccess;
-  // the device blocks start from zero for their next contributions
+  const bool copies_ok = ok;
+  const bool recorded = cudaEventRecord(e->slot_ev[slot], s) == cudaSuccess;
+  if (!copies_ok || !recorded) {
+    // Nothing is added and no device block is zeroed: the device gradients
+    // stay as they were.  Copies already queued may still be writing into
+    // the slot, so it stays busy until they are done.
+    if (recorded) {
+      std::lock_guard<std::mutex> lk(e->mu);
+      e->jobs.push_back(oomb_wb_engine::Job{slot, nullptr, {}, bfloats});
+      ++e->pending;
+    } else {
+      cudaStreamSynchronize(s);
+      std::lock_guard<std::mutex> lk(e->mu);
+      e->slot_busy[slot] = false;
+    }
+    e->cv.notify_all();
+    return OOMB_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lk(e->mu);
+    e->jobs.push_back(oomb_wb_engine::Job{
+        slot, host_pool->grad, std::vector<int32_t>(h_dst_blocks, h_dst_blocks + n_blocks),
+        bfloats});
+    ++e->pending;
+  }
+  e->cv.notify_all();
+  // The device blocks start from zero for their next contributions; the
+  // copies ahead of these fills on the stream have captured the values.
   for (int i = 0; i < n_blocks && ok;) {
     int j = i + 1;
     while (j < n_blocks && h_src_blocks[j] == h_src_blocks[j - 1] + 1) ++j;
@@ -253,18 +322,6 @@ extern "C" oomb_status oomb_grad_writeback(oomb_pool* device_pool, oomb_pool* ho
                          (j - i) * bfloats * 4, s) == cudaSuccess;
     i = j;
   }
-  {
-    std::lock_guard<std::mutex> lk(e->mu);
-    if (!ok) {
-      e->slot_busy[slot] = false;
-    } else {
-      e->jobs.push_back(oomb_wb_engine::Job{
-          slot, host_pool->grad, std::vector<int32_t>(h_dst_blocks, h_dst_blocks + n_blocks),
-          bfloats});
-      ++e->pending;
-    }
-  }
-  e->cv.notify_all();
   return ok ? OOMB_OK : OOMB_ERR_CUDA;
 }
 
@@ -272,8 +329,33 @@ extern "C" oomb_status oomb_grad_writeback_sync(oomb_pool* device_pool, int64_t 
   if (!device_pool) return OOMB_ERR_INVALID_ARG;
   oomb_wb_engine* e = device_pool->wb;
   if (!e) return OOMB_OK;
-  std::unique_lock<std::mutex> lk(e->mu);
-  const bool done = e->cv.wait_for(lk, std::chrono::microseconds(timeout_us),
-                                   [&] { return e->pending == 0; });
-  return done ? OOMB_OK : OOMB_ERR_TIMEOUT;
+  return e->sync(timeout_us);
+}
+
+extern "C" oomb_status oomb_selftest_writeback_copy(float* host_grad, int32_t n_blocks,
+                                                    int32_t block_floats, int32_t fail_copy) {
+  if (!host_grad || n_blocks <= 0 || block_floats <= 0) return OOMB_ERR_INVALID_ARG;
+  // A host-only engine: its staging slot holds 1.0 in every element and its
+  // copy "completes" with success or with an error, as asked.
+  oomb_wb_engine e;
+  e.fake_copies = true;
+  e.fake_copy_status = fail_copy ? cudaErrorLaunchFailure : cudaSuccess;
+  const size_t nf = static_cast<size_t>(n_blocks) * block_floats;
+  std::vector<float> slot(nf, 1.0f);
+  e.slot_ptr[0] = slot.data();
+  e.slot_bytes[0] = nf * 4;
+  e.slot_busy[0] = true;
+  std::vector<int32_t> dst(n_blocks);
+  for (int i = 0; i < n_blocks; ++i) dst[i] = i;
+  e.worker = std::thread([&e] { e.run(); });
+  {
+    std::lock_guard<std::mutex> lk(e.mu);
+    e.jobs.push_back(oomb_wb_engine::Job{0, host_grad, dst, static_cast<size_t>(block_floats)});
+    ++e.pending;
+  }
+  e.cv.notify_all();
+  const oomb_status st = e.sync(10'000'000);
+  e.shutdown();
+  e.slot_ptr[0] = nullptr;
+  return st;
 }

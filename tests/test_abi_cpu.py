@@ -172,3 +172,39 @@ def test_batched_topk_workspace_size_formula():
     assert L.page_topk_batched_workspace_size(1, Hkv, d, mp) == \
         L.page_topk_workspace_size(4096, 28, Hkv, d, mp)
     assert L.page_topk_batched_workspace_size(0, Hkv, d, mp) == 0
+
+
+def test_grad_writeback_rejects_repeated_destinations_before_cuda():
+    """The worker's CPU threads add blocks in parallel, so a destination listed
+    twice would lose an addition: the list is checked in one pass, in order,
+    before the pools' locations (so host pools reach the check here)."""
+    lib = L.load()
+    pool = L.pool_create(8, 16, 1, 64, L.LOC_HOST, True, 0)
+    try:
+        src = (ctypes.c_int32 * 3)(0, 1, 2)
+        dup = (ctypes.c_int32 * 3)(4, 4, 99)     # repeat first, out of range after
+        out = (ctypes.c_int32 * 3)(4, 5, 99)     # out of range, no repeat
+        ok = (ctypes.c_int32 * 3)(4, 5, 6)
+        assert lib.oomb_grad_writeback(pool, pool, src, dup, 3, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_grad_writeback(pool, pool, src, out, 3, None) == L.ERR_BAD_PAGE
+        # a valid distinct list passes the list checks and stops at the location check
+        assert lib.oomb_grad_writeback(pool, pool, src, ok, 3, None) == L.ERR_INVALID_ARG
+        bad_src = (ctypes.c_int32 * 3)(0, 1, 8)
+        assert lib.oomb_grad_writeback(pool, pool, bad_src, ok, 3, None) == L.ERR_BAD_PAGE
+    finally:
+        L.pool_destroy(pool)
+
+
+def test_grad_writeback_worker_skips_a_failed_copy_and_reports_it():
+    """A staging slot whose device->host copy failed is not added into the host
+    gradients, and the sync reports OOMB_ERR_CUDA; a completed copy is added."""
+    import numpy as np
+    lib = L.load()
+    n, bf = 5, 96
+    host = np.full(n * bf + 7, 2.5, dtype=np.float32)
+    ptr = host.ctypes.data_as(ctypes.c_void_p)
+    assert lib.oomb_selftest_writeback_copy(ptr, n, bf, 1) == L.ERR_CUDA
+    assert np.all(host == 2.5)
+    assert lib.oomb_selftest_writeback_copy(ptr, n, bf, 0) == L.OK
+    assert np.all(host[:n * bf] == 3.5) and np.all(host[n * bf:] == 2.5)
+    assert lib.oomb_selftest_writeback_copy(None, n, bf, 0) == L.ERR_INVALID_ARG
