@@ -48,8 +48,27 @@ def _peaks():
         with open(p) as f:
             d = json.load(f)
         return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16": d.get("bf16_tflops", 1590.0),
-                "bf16_sustained": d.get("bf16_tflops_sustained", 1400.0), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+                "bf16_sustained": d.get("bf16_tflops_sustained", 1400.0),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+def clock_scaled_peak(burst, sm_mhz, sm_max_mhz):
+    """The burst tensor peak scaled to the SM clock a run actually held: the
+    tensor pipe's rate is proportional to the SM clock, so this is what the
+    same GEMM would reach at that clock (None without a clock record)."""
+    if not burst or not sm_mhz or not sm_max_mhz:
+        return None
+    return burst * sm_mhz / sm_max_mhz
+
+
+def step_fractions(tflops, peaks, sm_mhz):
+    """A step's TFLOP/s as fractions of the sustained, burst and clock-scaled
+    burst bf16 peaks."""
+    cp = clock_scaled_peak(peaks["bf16"], sm_mhz, peaks.get("sm_max_mhz"))
+    return {"of_sustained": tflops / peaks["bf16_sustained"], "of_burst": tflops / peaks["bf16"],
+            "of_clock_normalised": tflops / cp if cp else None}
 
 
 def pairs_of_chunk(C, n_past_keys):
@@ -146,7 +165,9 @@ class Clocks:
 class Run:
     """All device state of one workload: pool, page tables, inputs, outputs."""
 
-    def __init__(self, w, sparse, device):
+    def __init__(self, w, sparse, device, inputs=None):
+        """inputs: per chunk a dict of device tensors q, k, v, dO (default: the
+        workload's shapes and distributions drawn on the device)."""
         import paged_kv_chunk_query_b200 as pk
         from paged_kv_chunk_query_b200 import synth
         self.pk, self.w, self.sparse, self.dev = pk, w, sparse, device
@@ -159,7 +180,8 @@ class Run:
         pt = torch.tensor(self.page_table, dtype=torch.int32, device=device)
         self.page_table_dev = pt
         self.cur = [pt[c * ppc:(c + 1) * ppc].contiguous() for c in range(N)]
-        self.inputs = [synth.device_chunk_inputs(w, c, device) for c in range(N)]
+        self.inputs = inputs if inputs is not None else \
+            [synth.device_chunk_inputs(w, c, device) for c in range(N)]
         self.o = [torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device) for _ in range(N)]
         self.dq = [torch.empty_like(x) for x in self.o]
         self.lse = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(N)]
@@ -839,6 +861,36 @@ def oracle_sample(w, rows, seed_chunk=None):
     return dt, flops, threads, desc
 
 
+def oracle_tiny_full():
+    """The tiny workload (L 512, Hq 4, Hkv 1, d 64, 16-token pages, 8 chunks of
+    64) run in full by the oracle, fwd+bwd: (seconds, algorithmic FLOPs)."""
+    from oracle.recurrent import run_sequence
+    from paged_kv_chunk_query_b200 import synth
+    w = synth.WORKLOADS["tiny"]
+    inp = synth.sequence_inputs(w)
+    t0 = time.perf_counter()
+    run_sequence(inp["q"], inp["k"], inp["v"], inp["do"], w.chunk_len, w.page_size,
+                 w.softmax_scale)
+    dt = time.perf_counter() - t0
+    return dt, 14.0 * step_pairs(w, False) * w.head_dim
+
+
+def cpu_baseline_obj(w, rows):
+    """The oracle as it stands on a bounded sample of the headline workload,
+    plus the tiny workload in full and the sample's rate extrapolated (and
+    labelled as such) to one whole step."""
+    dt, fl, threads, desc = oracle_sample(w, rows)
+    rate = fl / dt
+    tdt, tfl = oracle_tiny_full()
+    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": desc, "seconds": dt,
+            "tiny_full_run": {"seconds": tdt, "tflops": tfl / tdt / 1e12,
+                              "what": "tiny workload (L 512) fwd+bwd in full, fp64"},
+            "extrapolated_full_step_seconds": step_pairs(w, False) * 14.0 * w.head_dim / rate,
+            "extrapolation_note": "the sample's TFLOP/s applied to the whole dense step's "
+                                  "algorithmic FLOPs; an estimate, not a measurement"}
+
+
 # ------------------------------------------------------------------ roofline bits
 def _traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or
@@ -894,6 +946,8 @@ def main():
                     help="run each chunk's dQ launch after its dK/dV launch on one stream")
     ap.add_argument("--offload-workload", default="qwen1m_topk_offload")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0: auto)")
+    ap.add_argument("--no-32k", action="store_true", help="skip the 32K dense throughput line")
+    ap.add_argument("--small-workload", default="qwen32k")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -908,7 +962,9 @@ def main():
         # The reference arm is the CPU oracle as it stands, rank 0 only.
         if rank != 0:
             return
-        rows = a.cpu_rows or 32
+        # the sample shrinks with the number of steps so the whole run stays
+        # near two minutes (64 rows for 8 steps; rate units are per second)
+        rows = a.cpu_rows or max(16, min(64, 64 * 8 // max(1, a.steps + a.warmup)))
         for _ in range(a.warmup):
             oracle_sample(w, rows)
         secs, flops = [], 0.0
@@ -971,13 +1027,18 @@ def main():
     dom = max(kernel_flops, key=kernel_flops.get)
     dom_ms = kt[dom]
     tr = _traffic(dom)
+    clock_peak = clock_scaled_peak(peaks["bf16"], clk.get("sm_mhz"), peaks.get("sm_max_mhz"))
     if dom in kernel_flops:
         achieved = kernel_flops[dom] / (dom_ms / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
                 "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_sustained"],
                 "frac_of_burst": achieved / peaks["bf16"],
-                "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                "frac_clock_normalised": achieved / clock_peak if clock_peak else None,
+                "clock_normalised_peak": clock_peak,
+                "peak_source": f"bf16_tflops_sustained ({peaks['source']}); burst "
+                               f"{peaks['bf16']:.1f}; clock-normalised = burst x median SM MHz "
+                               "of this run / max SM MHz",
                 "traffic": tr["bytes_per_launch"] if tr else None,
                 "launch_share": dom_ms / ms}
     else:
@@ -1019,6 +1080,29 @@ def main():
                       "device_status": sparse_status}
         sp.close()
         del sp
+        torch.cuda.empty_cache()
+
+    small_obj = None
+    if not a.no_32k:
+        w32 = synth.WORKLOADS[a.small_workload]
+        r32 = Run(w32, False, device)
+        r32.concurrent_bwd = not a.serial_bwd
+        r32.fwd_overlap = a.fwd_overlap
+        clk32 = Clocks(local)
+        clk32.start()
+        ms_32, kt_32 = time_steps(r32, max(a.steps, 5), a.warmup, dist_on, device)
+        c32 = clk32.stop()
+        tf32 = r32.step_flops / (ms_32 / 1e3) / 1e12
+        small_obj = {"workload": w32.name, "context": w32.context,
+                     "value": tf32 * world, "unit": "TFLOP/s", "ms_per_step": ms_32,
+                     "steps": max(a.steps, 5), "tokens_per_s": w32.context * world / (ms_32 / 1e3),
+                     "tflop_per_step": r32.step_flops / 1e12,
+                     "fractions_of_bf16_peak": step_fractions(tf32, _peaks(), c32.get("sm_mhz")),
+                     "clocks": c32,
+                     "kernels": {k: {"ms_per_step": v} for k, v in kt_32.items()},
+                     "device_status": pk.get_device_status(r32.pool)}
+        r32.close()
+        del r32
         torch.cuda.empty_cache()
 
     local_obj = None
@@ -1088,10 +1172,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu:
-        rows = a.cpu_rows or 32
-        dt, fl, threads, desc = oracle_sample(w, rows)
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": desc, "seconds": dt}
+        cpu = cpu_baseline_obj(w, a.cpu_rows or 64)
 
     if dist_on:
         torch.distributed.barrier()
@@ -1116,6 +1197,9 @@ def main():
             k: {"ms_per_step": v, "tflops": (kernel_flops[k] / (v / 1e3) / 1e12)
                 if k in kernel_flops else None} for k, v in kt_serial.items()},
         "roofline": roof,
+        "step_fractions_of_bf16_peak": step_fractions(value / world, peaks, clk.get("sm_mhz")),
+        "ms_x_median_sm_mhz": ms * clk["sm_mhz"] if clk.get("sm_mhz") else None,
+        "qwen32k": small_obj,
         "sparse": sparse_obj,
         "local": local_obj,
         "qtile_topk": qtile_obj,
