@@ -201,24 +201,39 @@ class Run:
                           for _ in range(N)]
             self.loc_n = [torch.zeros((Hkv,), dtype=torch.int32, device=device) for _ in range(N)]
         self.qtile = sparse and w.qtile_topk
+        self.qpage = sparse and w.qpage_topk
+        self.masks = [None] * N
         if sparse:
             ms = w.top_k + w.n_recent
-            nq = (C + 127) // 128 if self.qtile else None
-            lead = (nq, Hkv) if self.qtile else (Hkv,)
+            nq = (C + 127) // 128
+            # selection problems per chunk: query tiles, query pages, or the chunk
+            nprob = nq if self.qtile else (C // P if self.qpage else None)
+            rows = 128 if self.qtile else P
+            lead = (nprob, Hkv) if nprob else (Hkv,)
             self.sel_l = [torch.zeros(lead + (ms,), dtype=torch.int32, device=device)
                           for _ in range(N)]
             self.sel_p = [torch.zeros(lead + (ms,), dtype=torch.int32, device=device)
                           for _ in range(N)]
             self.sel_n = [torch.zeros(lead, dtype=torch.int32, device=device) for _ in range(N)]
-            if self.qtile:
-                ws = pk.page_topk_batched_workspace_size(nq, Hkv, d, (N - 1) * ppc)
-                self.row_start = torch.arange(0, (nq + 1) * 128, 128, dtype=torch.int32,
+            if nprob:
+                ws = pk.page_topk_batched_workspace_size(nprob, Hkv, d, (N - 1) * ppc)
+                self.sel_rows = rows
+                self.row_start = torch.arange(0, (nprob + 1) * rows, rows, dtype=torch.int32,
                                               device=device).clamp_(max=C)
-                self.npast = [torch.full((nq,), c * ppc, dtype=torch.int32, device=device)
+                self.npast = [torch.full((nprob,), c * ppc, dtype=torch.int32, device=device)
                               for c in range(N)]
             else:
                 ws = pk.page_topk_workspace_size(C, Hq, Hkv, d, (N - 1) * ppc)
             self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+            if self.qpage:
+                # per query tile: the union of its query pages' lists + membership masks
+                mu = min(128 // P, C // P) * ms
+                self.u_pages = [torch.zeros((nq, Hkv, mu), dtype=torch.int32, device=device)
+                                for _ in range(N)]
+                self.masks = [torch.zeros((nq, Hkv, mu), dtype=torch.uint8, device=device)
+                              for _ in range(N)]
+                self.u_cnt = [torch.zeros((nq, Hkv), dtype=torch.int32, device=device)
+                              for _ in range(N)]
         # algorithmic FLOPs per chunk (per kernel class) and per step
         self.flops = {"fwd": [], "dkdv": [], "dq": []}
         for c in range(N):
@@ -231,7 +246,38 @@ class Run:
         # mean, page scores and select per chunk with a past (per-query-tile
         # lists: and a second dK/dV launch); local lists one
         self.launches_per_step = N * 5 + ((N - 1) * 3 if sparse else 0) + \
-            ((N - 1) if self.local else 0) + ((N - 1) if self.qtile else 0)
+            ((N - 1) if self.local else 0) + ((N - 1) if self.qtile else 0) + \
+            ((N - 1) * 2 if self.qpage else 0)
+
+    def select(self, c, st, timed):
+        """Chunk c's past lists on stream st: (pages, counts, masks)."""
+        pk, w = self.pk, self.w
+        ppc = w.pages_per_chunk
+        x = self.inputs[c]
+        if c == 0:
+            return None, None, None
+        n_past = c * ppc
+        if self.local:
+            timed("lists", lambda: pk.local_pages(self.pool, self.page_table_dev[:n_past], n_past,
+                                                  self.loc_p[c], self.loc_n[c], stream=st), st)
+            return self.loc_p[c], self.loc_n[c], None
+        if self.qtile or self.qpage:
+            timed("topk", lambda: pk.page_topk_batched(
+                self.pool, x["q"], self.row_start, self.sel_rows, self.npast[c], n_past,
+                self.page_table_dev[:n_past], w.top_k, w.n_recent, self.sel_l[c], self.sel_p[c],
+                self.sel_n[c], self.ws, stream=st), st)
+            if self.qtile:
+                return self.sel_p[c], self.sel_n[c], None
+            timed("lists", lambda: pk.qpage_lists(
+                self.pool, self.sel_l[c], self.sel_p[c], self.sel_n[c], w.chunk_len,
+                self.u_pages[c], self.masks[c], self.u_cnt[c], stream=st), st)
+            return self.u_pages[c], self.u_cnt[c], self.masks[c]
+        if self.sparse:
+            timed("topk", lambda: pk.page_topk(
+                self.pool, x["q"], self.page_table_dev[:n_past], n_past, w.top_k, w.n_recent,
+                self.sel_l[c], self.sel_p[c], self.sel_n[c], self.ws, stream=st), st)
+            return self.sel_p[c], self.sel_n[c], None
+        return self.dense_past[c], self.dense_cnt[c], None
 
     def step(self, timers=None):
         if self.fwd_overlap and self.concurrent_bwd:
@@ -269,37 +315,15 @@ class Run:
         for c in range(w.num_chunks):
             x = self.inputs[c]
             F.wait_event(appended)    # chunk c's pages (and earlier summaries) appended
-            if c == 0:
-                past, cnt = None, None
-            elif self.local:
-                n_past = c * ppc
-                timed("lists", lambda: pk.local_pages(self.pool, self.page_table_dev[:n_past],
-                                                      n_past, self.loc_p[c], self.loc_n[c],
-                                                      stream=F), F)
-                past, cnt = self.loc_p[c], self.loc_n[c]
-            elif self.qtile:
-                n_past = c * ppc
-                timed("topk", lambda: pk.page_topk_batched(
-                    self.pool, x["q"], self.row_start, 128, self.npast[c], n_past,
-                    self.page_table_dev[:n_past], w.top_k, w.n_recent, self.sel_l[c],
-                    self.sel_p[c], self.sel_n[c], self.ws, stream=F), F)
-                past, cnt = self.sel_p[c], self.sel_n[c]
-            elif self.sparse:
-                n_past = c * ppc
-                timed("topk", lambda: pk.page_topk(
-                    self.pool, x["q"], self.page_table_dev[:n_past], n_past, w.top_k, w.n_recent,
-                    self.sel_l[c], self.sel_p[c], self.sel_n[c], self.ws, stream=F), F)
-                past, cnt = self.sel_p[c], self.sel_n[c]
-            else:
-                past, cnt = self.dense_past[c], self.dense_cnt[c]
+            past, cnt, msk = self.select(c, F, timed)
             o, lse, dq = self.o[c], self.lse[c], self.dq[c]
             sc = w.softmax_scale
             delta = self.deltas[c]
             timed("fwd", lambda: pk.chunk_attn_fwd(self.pool, x["q"], o, lse, past, cnt,
-                                                   self.cur[c], sc, F), F)
+                                                   self.cur[c], sc, F, past_masks=msk), F)
             timed("preprocess", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, F,
-                step=pk.BWD_PREPROCESS), F)
+                step=pk.BWD_PREPROCESS, past_masks=msk), F)
             if c + 1 < w.num_chunks:
                 xn = self.inputs[c + 1]
                 timed("append", lambda: pk.kv_append(self.pool, self.cur[c + 1], xn["k"], xn["v"],
@@ -310,10 +334,10 @@ class Run:
             M.wait_stream(F)
             timed("dq", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, S,
-                step=pk.BWD_DQ), S)
+                step=pk.BWD_DQ, past_masks=msk), S)
             timed("dkdv", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, M,
-                step=pk.BWD_DKDV), M)
+                step=pk.BWD_DKDV, past_masks=msk), M)
         M.wait_stream(S)
         M.wait_stream(F)
 
@@ -346,37 +370,15 @@ class Run:
             if c == 0:
                 timed("append", lambda: pk.kv_append(self.pool, self.cur[0], x["k"], x["v"],
                                                      stream))
-            if c == 0:
-                past, cnt = None, None
-            elif self.local:
-                n_past = c * ppc
-                timed("lists", lambda: pk.local_pages(self.pool, self.page_table_dev[:n_past],
-                                                      n_past, self.loc_p[c], self.loc_n[c],
-                                                      stream=stream))
-                past, cnt = self.loc_p[c], self.loc_n[c]
-            elif self.qtile:
-                n_past = c * ppc
-                timed("topk", lambda: pk.page_topk_batched(
-                    self.pool, x["q"], self.row_start, 128, self.npast[c], n_past,
-                    self.page_table_dev[:n_past], w.top_k, w.n_recent, self.sel_l[c],
-                    self.sel_p[c], self.sel_n[c], self.ws, stream=stream))
-                past, cnt = self.sel_p[c], self.sel_n[c]
-            elif self.sparse:
-                n_past = c * ppc
-                timed("topk", lambda: pk.page_topk(
-                    self.pool, x["q"], self.page_table_dev[:n_past], n_past, w.top_k, w.n_recent,
-                    self.sel_l[c], self.sel_p[c], self.sel_n[c], self.ws, stream=stream))
-                past, cnt = self.sel_p[c], self.sel_n[c]
-            else:
-                past, cnt = self.dense_past[c], self.dense_cnt[c]
+            past, cnt, msk = self.select(c, stream, timed)
             o, lse, dq = self.o[c], self.lse[c], self.dq[c]
             s = w.softmax_scale
             delta = self.deltas[c]
             timed("fwd", lambda: pk.chunk_attn_fwd(self.pool, x["q"], o, lse, past, cnt,
-                                                   self.cur[c], s, stream))
+                                                   self.cur[c], s, stream, past_masks=msk))
             timed("preprocess", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], s, stream,
-                step=pk.BWD_PREPROCESS))
+                step=pk.BWD_PREPROCESS, past_masks=msk))
             if c + 1 < w.num_chunks:
                 # chunk c+1's pages: nothing of chunk c reads or writes them
                 xn = self.inputs[c + 1]
@@ -386,10 +388,10 @@ class Run:
                 side.wait_stream(stream)
             timed("dq", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], s, side,
-                step=pk.BWD_DQ), side)
+                step=pk.BWD_DQ, past_masks=msk), side)
             timed("dkdv", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], s, stream,
-                step=pk.BWD_DKDV))
+                step=pk.BWD_DKDV, past_masks=msk))
         if side is not stream:
             stream.wait_stream(side)
 
@@ -940,6 +942,8 @@ def main():
     ap.add_argument("--dense-grad-path", choices=["gpu", "host"], default="host",
                     help="gradient write-back of the dense offload run")
     ap.add_argument("--qtile-workload", default="qwen256k_topk_qtile")
+    ap.add_argument("--no-qpage", action="store_true", help="skip the per-query-page Top-K run")
+    ap.add_argument("--qpage-workload", default="qwen256k_topk_qpage")
     ap.add_argument("--fwd-overlap", action="store_true",
                     help="run each chunk's forward on a third stream beside the previous backward")
     ap.add_argument("--serial-bwd", action="store_true",
@@ -1137,6 +1141,25 @@ def main():
         del qr
         torch.cuda.empty_cache()
 
+    qpage_obj = None
+    if not a.no_qpage:
+        wp = synth.WORKLOADS[a.qpage_workload]
+        qp = Run(wp, True, device)
+        qp.concurrent_bwd = not a.serial_bwd
+        qp.fwd_overlap = a.fwd_overlap
+        ms_p, kt_p = time_steps(qp, a.steps, a.warmup, dist_on, device)
+        qpage_obj = {"workload": wp.name,
+                     "selection": f"Top-K per {wp.page_size}-token query page; per 128-row "
+                                  "query tile the union of its query pages' lists with "
+                                  "membership masks",
+                     "value": qp.step_flops * world / (ms_p / 1e3) / 1e12, "unit": "TFLOP/s",
+                     "ms_per_step": ms_p, "tokens_per_s": wp.context * world / (ms_p / 1e3),
+                     "kernels": {k: {"ms_per_step": v} for k, v in kt_p.items()},
+                     "device_status": pk.get_device_status(qp.pool)}
+        qp.close()
+        del qp
+        torch.cuda.empty_cache()
+
     offload_obj = None
     if not a.no_offload:
         offload_obj = offload_run(synth.WORKLOADS[a.offload_workload], max(1, min(a.steps, 2)),
@@ -1203,6 +1226,7 @@ def main():
         "sparse": sparse_obj,
         "local": local_obj,
         "qtile_topk": qtile_obj,
+        "qpage_topk": qpage_obj,
         "offload": offload_obj,
         "dense_offload": dense_off_obj,
         "projection": proj_obj,

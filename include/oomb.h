@@ -144,7 +144,16 @@ typedef struct oomb_attn_args {
    *    past_counts [n_qtiles][num_kv_heads], n_qtiles = ceil(chunk_len / 128);
    *    rows of query tile t attend to list t (plus the chunk, causally).  The
    *    outputs of oomb_page_topk_batched with one problem per query tile have
-   *    exactly this layout. */
+   *    exactly this layout.
+   * 2: one past list per QUERY PAGE (page_size consecutive rows of the chunk)
+   *    and group ([pt] §2C), given per 128-row query tile as the union of the
+   *    lists of its 128/page_size query pages: past_pages and past_counts as
+   *    for 1 (the union, ascending logical page order), and past_masks
+   *    [n_qtiles][num_kv_heads][max_past] with bit b of entry i set iff that
+   *    page is in the list of the tile's query page b (rows 128 t + b page_size
+   *    .. + page_size - 1).  A row attends to the entries whose bit for its
+   *    query page is set (plus the chunk, causally).  oomb_qpage_lists builds
+   *    these from oomb_page_topk_batched's per-query-page selections. */
   int32_t lists_per_qtile;
   /* Segmented attention: the past streamed through a bounded device window
    * ([pt] §2D: pages move between host and GPU while computation runs; a
@@ -166,6 +175,7 @@ typedef struct oomb_attn_args {
   int32_t segment;
   float* o_acc;   /* device fp32 [chunk_len][num_q_heads][head_dim]: running O  */
   float* dq_acc;  /* device fp32, layout of o_acc: running dQ (backward)         */
+  const uint8_t* past_masks;  /* lists_per_qtile == 2 only (else ignored), see above */
 } oomb_attn_args;
 
 enum { OOMB_SEG_WHOLE = 0, OOMB_SEG_FIRST = 1, OOMB_SEG_NEXT = 2, OOMB_SEG_LAST = 3 };
@@ -237,6 +247,27 @@ oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, int32_t chunk
                            int32_t top_k, int32_t n_recent, int32_t* d_out_logical,
                            int32_t* d_out_physical, int32_t* d_out_count, float* d_out_scores,
                            void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* Per-query-page lists for the attention ([pt] §2C: the key pages relevant to
+ * each query page).  Input: one selection per query page of a chunk, as
+ * oomb_page_topk_batched returns them with one problem per query page (rows
+ * b page_size .. b page_size + page_size - 1): d_sel_logical and
+ * d_sel_physical [n_qpages][num_kv_heads][max_sel] (ascending logical ids),
+ * d_sel_count [n_qpages][num_kv_heads], n_qpages = chunk_len / page_size.
+ * Output per 128-row query tile t and group g: the union of the selections
+ * of the tile's query pages in ascending logical order, as physical ids
+ * d_out_pages [n_qtiles][num_kv_heads][max_union], the membership bits
+ * d_out_masks (uint8, same layout; bit b: in the list of the tile's query
+ * page b) and d_out_count [n_qtiles][num_kv_heads] — the past_pages,
+ * past_masks and past_counts of oomb_attn_args with lists_per_qtile = 2.
+ * max_union must be at least min(128 / page_size, n_qpages) * max_sel.
+ * One launch on `stream`; a count outside [0, max_sel] is clamped and sets
+ * bit 2 of the pool's device status word. */
+oomb_status oomb_qpage_lists(oomb_pool* pool, const int32_t* d_sel_logical,
+                             const int32_t* d_sel_physical, const int32_t* d_sel_count,
+                             int32_t chunk_len, int32_t max_sel, int32_t* d_out_pages,
+                             uint8_t* d_out_masks, int32_t* d_out_count, int32_t max_union,
+                             void* stream);
 
 /* Allocation-free variant of oomb_page_topk (this one has no counterpart in
  * the paper; it exists for callers that cannot allocate device memory, e.g.

@@ -15,7 +15,7 @@ from ._lib import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, LOC_DEVICE, LOC_HOST, LOC_P
                    page_topk, page_topk_batched, page_topk_batched_workspace_size,
                    page_topk_workspace_size, pool_alloc_page, pool_buffers, pool_create,
                    pool_destroy, pool_free_page, pool_get_desc, pool_num_free, pool_views,
-                   prefetch_lists, qkv_project, status_string, version, wait)
+                   prefetch_lists, qkv_project, qpage_lists, status_string, version, wait)
 from .synth import WORKLOADS, Workload
 
 __all__ = [
@@ -27,6 +27,6 @@ __all__ = [
     "get_device_status", "status_string", "version",
     "LOC_DEVICE", "LOC_PINNED_HOST", "LOC_HOST", "BWD_PREPROCESS", "BWD_DKDV", "BWD_DQ",
     "SEG_WHOLE", "SEG_FIRST", "SEG_NEXT", "SEG_LAST", "PROJ_Q", "PROJ_KV", "PROJ_QKV",
-    "qkv_project",
+    "qkv_project", "qpage_lists",
     "WORKLOADS", "Workload",
 ]

@@ -39,7 +39,7 @@ EXPORTS = (
     "oomb_version", "oomb_page_topk_static", "oomb_grad_writeback_sync",
     "oomb_selftest_wait_limit", "oomb_page_topk_batched_workspace_size", "oomb_page_topk_batched",
     "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists", "oomb_local_pages",
-    "oomb_qkv_project", "oomb_selftest_writeback_copy",
+    "oomb_qkv_project", "oomb_selftest_writeback_copy", "oomb_qpage_lists",
 )
 
 
@@ -64,7 +64,8 @@ class AttnArgs(ctypes.Structure):
                 ("past_counts", ctypes.c_void_p), ("max_past", ctypes.c_int32),
                 ("cur_pages", ctypes.c_void_p), ("softmax_scale", ctypes.c_float),
                 ("lists_per_qtile", ctypes.c_int32), ("segment", ctypes.c_int32),
-                ("o_acc", ctypes.c_void_p), ("dq_acc", ctypes.c_void_p)]
+                ("o_acc", ctypes.c_void_p), ("dq_acc", ctypes.c_void_p),
+                ("past_masks", ctypes.c_void_p)]
 
 
 _lib = None
@@ -108,6 +109,7 @@ def load() -> ctypes.CDLL:
         "oomb_local_pages": [vp, vp, i32, i32, vp, vp, vp],
         "oomb_qkv_project": [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp],
         "oomb_selftest_writeback_copy": [vp, i32, i32, i32],
+        "oomb_qpage_lists": [vp, vp, vp, vp, i32, i32, vp, vp, vp, i32, vp],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):  # completeness is checked by the export test
@@ -256,18 +258,25 @@ def kv_append(pool: int, page_ids: torch.Tensor, k: torch.Tensor, v: torch.Tenso
 
 
 def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o=None, dq=None,
-               delta_ws=None, segment=SEG_WHOLE, o_acc=None, dq_acc=None):
+               delta_ws=None, segment=SEG_WHOLE, o_acc=None, dq_acc=None, past_masks=None):
     """past_pages [Hkv][max_past] (one list per group) or [n_qtiles][Hkv][max_past]
-    (one list per 128-row query tile and group; counts [n_qtiles][Hkv])."""
+    (one list per 128-row query tile and group; counts [n_qtiles][Hkv]); with
+    past_masks (uint8, layout of past_pages) the per-tile lists are unions of
+    per-query-page lists (oomb_qpage_lists)."""
     C, Hq, _ = q.shape
     per_qtile = past_pages is not None and past_pages.dim() == 3
     max_past = past_pages.shape[-1] if past_pages is not None and past_pages.numel() else 0
+    if past_masks is not None and not per_qtile:
+        raise ValueError("past_masks need per-query-tile past_pages [n_qtiles][Hkv][max_past]")
     if per_qtile and max_past:
         n_qt = (C + 127) // 128
         if past_pages.shape[0] != n_qt or past_counts is None or \
                 tuple(past_counts.shape) != tuple(past_pages.shape[:2]):
             raise ValueError(f"per-query-tile lists need past_pages [{n_qt}][Hkv][max_past] and "
                              f"past_counts [{n_qt}][Hkv]")
+        if past_masks is not None and tuple(past_masks.shape) != tuple(past_pages.shape):
+            raise ValueError("past_masks must have the shape of past_pages")
+    mode = (2 if past_masks is not None else 1) if per_qtile else 0
     return AttnArgs(
         _dev_tensor(q, torch.bfloat16, "q"), _dev_tensor(o, torch.bfloat16, "o"),
         _dev_tensor(lse, torch.float32, "lse"),
@@ -278,24 +287,26 @@ def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o
         _dev_tensor(past_pages, torch.int32, "past_pages") if max_past else None,
         _dev_tensor(past_counts, torch.int32, "past_counts") if max_past else None,
         max_past, _dev_tensor(cur_pages, torch.int32, "cur_pages"), softmax_scale,
-        int(per_qtile), segment,
+        mode, segment,
         _dev_tensor(o_acc, torch.float32, "o_acc") if o_acc is not None else None,
-        _dev_tensor(dq_acc, torch.float32, "dq_acc") if dq_acc is not None else None)
+        _dev_tensor(dq_acc, torch.float32, "dq_acc") if dq_acc is not None else None,
+        _dev_tensor(past_masks, torch.uint8, "past_masks") if past_masks is not None and max_past
+        else None)
 
 
 def chunk_attn_fwd(pool, q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
-                   stream=None, segment=SEG_WHOLE, o_acc=None):
+                   stream=None, segment=SEG_WHOLE, o_acc=None, past_masks=None):
     a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
-                   segment=segment, o_acc=o_acc)
+                   segment=segment, o_acc=o_acc, past_masks=past_masks)
     _check(load().oomb_chunk_attn_fwd(pool, ctypes.byref(a), _stream(stream)),
            "oomb_chunk_attn_fwd")
 
 
 def chunk_attn_bwd(pool, q, o, lse, d_o, dq, delta_ws, past_pages, past_counts, cur_pages,
                    softmax_scale, stream=None, step=None, segment=SEG_WHOLE, o_acc=None,
-                   dq_acc=None):
+                   dq_acc=None, past_masks=None):
     a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o, dq,
-                   delta_ws, segment=segment, o_acc=o_acc, dq_acc=dq_acc)
+                   delta_ws, segment=segment, o_acc=o_acc, dq_acc=dq_acc, past_masks=past_masks)
     if step is None:
         _check(load().oomb_chunk_attn_bwd(pool, ctypes.byref(a), _stream(stream)),
                "oomb_chunk_attn_bwd")
@@ -347,6 +358,21 @@ def page_topk_batched(pool, q, row_start, max_rows, n_past, max_past, page_table
         _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
         _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "oomb_page_topk_batched")
+
+
+def qpage_lists(pool, sel_logical, sel_physical, sel_count, chunk_len, out_pages, out_masks,
+                out_count, stream=None):
+    """oomb_qpage_lists: per-query-page selections [n_qpages][Hkv][max_sel] ->
+    per-query-tile union lists [n_qtiles][Hkv][max_union] (physical ids), their
+    membership masks (uint8) and counts [n_qtiles][Hkv]."""
+    _check(load().oomb_qpage_lists(
+        pool, _dev_tensor(sel_logical, torch.int32, "sel_logical"),
+        _dev_tensor(sel_physical, torch.int32, "sel_physical"),
+        _dev_tensor(sel_count, torch.int32, "sel_count"), chunk_len, sel_logical.shape[-1],
+        _dev_tensor(out_pages, torch.int32, "out_pages"),
+        _dev_tensor(out_masks, torch.uint8, "out_masks"),
+        _dev_tensor(out_count, torch.int32, "out_count"), out_pages.shape[-1], _stream(stream)),
+        "oomb_qpage_lists")
 
 
 def local_pages(pool, page_table, n_past, out_pages, out_count, stream=None):

@@ -37,8 +37,11 @@ struct BwdParams {
   uint32_t* status;
   int max_past, C, Hq, Hkv, G, P, num_pool_pages, max_past_tiles;
   int lpq;  // 1: one past list per (query tile, group); dK/dV: blockIdx.z = query tile
+            // 2: per query page (union lists + membership masks), as 1 otherwise
   int seg;  // OOMB_SEG_*: whole key set, or a segment accumulated into dq_acc
   float* dq_acc;
+  const uint8_t* masks;  // lpq 2: query-page membership bits of each list entry
+  int lg_p;              // log2(P)
   float scale, scale_log2;
 };
 
@@ -283,6 +286,18 @@ __global__ void __launch_bounds__(320, 1)
     if (is_past) key_valid = j * kTile + r < sch.n_past_pages * p.P;
     else key_valid = u * kTile + r < p.C;
     const int key_local = u * kTile + r;  // causal position (current tiles only)
+    // Groups of 16 query columns of this half that may hold a valid (key,
+    // query) pair, constant over the loop (P >= 16, so a group lies in one
+    // query page): none for a key row past the list; with per-query-page
+    // lists, the groups whose query page listed this key row's page (bit
+    // (cs + 16 k) / P of the entry's membership mask).
+    uint32_t grp = key_valid ? 0xFu : 0u;
+    if (p.masks && is_past && key_valid) {
+      const uint32_t qm =
+          p.masks[static_cast<size_t>(li) * p.max_past + ((j * kTile + r) >> p.lg_p)];
+      grp = 0;
+      for (int k = 0; k < 4; ++k) grp |= ((qm >> ((half * 64 + 16 * k) >> p.lg_p)) & 1u) << k;
+    }
     bool ok = true;
     for (int i = 0; i < n_iter; ++i) {
       const int s = i % Cfg::kNS;
@@ -303,7 +318,7 @@ __global__ void __launch_bounds__(320, 1)
       // chunk's own keys, causally at or after the key
       const int cmax = min(kTile, p.C - t * kTile) - static_cast<int>(cs);
       const int cmin = (is_past ? 0 : key_local - t * kTile) - static_cast<int>(cs);
-      const bool full = key_valid && cmin <= 0 && cmax >= 64;
+      const bool full = grp == 0xFu && cmin <= 0 && cmax >= 64;
       // P^T = 2^(S^T*scale*log2e - LSE*log2e); LSE read 4 at a time (broadcast)
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
@@ -317,7 +332,8 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pr[c] = (key_valid && c < cmax && c >= cmin) ? pr[c] : 0.f;
+        for (int c = 0; c < 64; ++c)
+          pr[c] = (c < cmax && c >= cmin && ((grp >> (c >> 4)) & 1u)) ? pr[c] : 0.f;
       }
       if (!(ok = warp_wait(&bar_dpt, i & 1, abort_flag))) break;
       tc_fence_after();
@@ -660,6 +676,22 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) pr[c] = c < lim ? pr[c] : 0.f;
       }
+      if (p.masks && j < sch.n_past_tiles) {
+        // per-query-page lists: pages this row's query page did not select
+        const int per = kTile >> p.lg_p;
+        const uint8_t* mrow = p.masks + static_cast<size_t>(li) * p.max_past + j * per;
+        const int qb = r >> p.lg_p;
+        // bit k: this half's columns [16k, 16k + 16) (one page: P >= 16) are kept
+        uint32_t keep = 0;
+        for (int k = 0; k < 4; ++k) {
+          const int sl = (static_cast<int>(cs) + 16 * k) >> p.lg_p;
+          if (j * per + sl < sch.n_past_pages && ((mrow[sl] >> qb) & 1u)) keep |= 1u << k;
+        }
+        if (keep != 0xFu) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pr[c] = ((keep >> (c >> 4)) & 1u) ? pr[c] : 0.f;
+        }
+      }
       if (!(ok = warp_wait(&bar_dp, j & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t dp[64];
@@ -803,6 +835,8 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.lpq = a->lists_per_qtile;
   p.seg = a->segment;
   p.dq_acc = a->dq_acc;
+  p.masks = a->lists_per_qtile == 2 ? a->past_masks : nullptr;
+  p.lg_p = __builtin_ctz(static_cast<unsigned>(s.P));
 
   if (step < 0 || step == OOMB_BWD_PREPROCESS) {
     constexpr int RPB = 256 / (D / 8);
@@ -830,6 +864,7 @@ oomb_status launch_bwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
       pc.lpq = 0;
       pc.max_past = pc.max_past_tiles = 0;
       pc.past_pages = pc.past_counts = nullptr;
+      pc.masks = nullptr;
       bwd_dkdv_kernel<D><<<dim3(s.n_qtiles, s.Hkv), 320, KvCfg<D>::kSmem, stream>>>(
           pc, qmap, domap, kvmap);
       if (check_launch() != OOMB_OK) return OOMB_ERR_CUDA;

@@ -45,9 +45,11 @@ struct FwdParams {
   const int32_t* cur_pages;
   uint32_t* status;
   int max_past, C, Hq, G, P, num_pool_pages;
-  int lpq;  // 1: one past list per (query tile, group)
+  int lpq;  // 1: one past list per (query tile, group); 2: per query page (union + masks)
   int seg;  // OOMB_SEG_*: whole key set, or a segment merged into o_acc / lse
   float* o_acc;
+  const uint8_t* masks;  // lpq 2: query-page membership bits of each list entry
+  int lg_p;              // log2(P)
   float scale_log2;
 };
 
@@ -267,6 +269,23 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int c = 0; c < kTile; ++c) s[c] = c < lim ? s[c] : -INFINITY;
       }
+      if (p.masks && j < sch.n_past_tiles) {
+        // per-query-page lists: a listed page this row's query page did not
+        // select is masked (its bit in the entry's membership mask is clear)
+        const int per = kTile >> p.lg_p;
+        const uint8_t* mrow = p.masks + static_cast<size_t>(li) * p.max_past + j * per;
+        const int qb = r >> p.lg_p;
+        // bit k: columns [16k, 16k + 16) (one page: P >= 16) are kept
+        uint32_t keep = 0;
+        for (int k = 0; k < kTile / 16; ++k) {
+          const int sl = (16 * k) >> p.lg_p;
+          if (j * per + sl < sch.n_past_pages && ((mrow[sl] >> qb) & 1u)) keep |= 1u << k;
+        }
+        if (keep != 0xFFu) {
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) s[c] = ((keep >> (c >> 4)) & 1u) ? s[c] : -INFINITY;
+        }
+      }
       // row max with 8 independent chains (raw logits; scale > 0 keeps the order)
       float m8[8];
 #pragma unroll
@@ -455,6 +474,8 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.lpq = a->lists_per_qtile;
   p.seg = a->segment;
   p.o_acc = a->o_acc;
+  p.masks = a->lists_per_qtile == 2 ? a->past_masks : nullptr;
+  p.lg_p = __builtin_ctz(static_cast<unsigned>(s.P));
   dim3 grid(s.n_qtiles, s.Hq);
   attn_fwd_kernel<D><<<grid, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
   return check_launch();

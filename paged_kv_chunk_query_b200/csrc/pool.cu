@@ -250,7 +250,8 @@ oomb_status validate_attn(const oomb_pool* pool, const oomb_attn_args* a, bool b
   if (a->num_q_heads <= 0 || a->num_q_heads % Hkv != 0) return OOMB_ERR_INVALID_ARG;
   if (a->max_past < 0 || (a->max_past > 0 && (!a->past_pages || !a->past_counts)))
     return OOMB_ERR_INVALID_ARG;
-  if (a->lists_per_qtile != 0 && a->lists_per_qtile != 1) return OOMB_ERR_INVALID_ARG;
+  if (a->lists_per_qtile < 0 || a->lists_per_qtile > 2) return OOMB_ERR_INVALID_ARG;
+  if (a->lists_per_qtile == 2 && a->max_past > 0 && !a->past_masks) return OOMB_ERR_INVALID_ARG;
   if (a->segment < OOMB_SEG_WHOLE || a->segment > OOMB_SEG_LAST) return OOMB_ERR_INVALID_ARG;
   if (a->segment != OOMB_SEG_WHOLE) {
     if (a->lists_per_qtile) return OOMB_ERR_INVALID_ARG;

@@ -12,20 +12,24 @@
 //
 // The kernels take a batch of independent problems (blockIdx.z / .y), each a
 // range of query rows and its own number of past pages; the per-chunk entry
-// points run a batch of one.
+// points run a batch of one.  Two launches:
 // Kernel 1 (qmean_partial): grid (slices, problems); each CTA streams whole
 //   token rows (all heads, contiguous) of a slice of its problem's rows, one
 //   thread per 16-byte column, and writes one fp32 partial per (group, d).
-// Kernel 2 (qbar): grid (problems, Hkv); sums the slice partials in a fixed
-//   order into q_bar.
-// Kernel 3 (page_score): grid (pages / 64, Hkv, problems); each warp scores 8
-//   pages (float4 loads of the summaries, shuffle reduction).
-// Kernel 4 (select): one CTA per (group, problem); finds the K-th largest
-//   64-bit key (ordered score, inverted id) by 8-bit radix passes from the top
-//   with a parallel bin scan, stopping once the boundary bin is kept whole,
-//   then compacts the kept ids in ascending order.
+//   It also zeroes the tickets kernel 2 counts on.
+// Kernel 2 (page_score_select): grid (pages / 64, Hkv, problems).  Each CTA
+//   sums the slice partials of its (problem, group) in one fixed order into
+//   q_bar (every CTA of a group gets the identical q_bar), then each warp
+//   scores 8 pages (float4 loads of the summaries, shuffle reduction).  The
+//   last CTA of a (problem, group) to finish (a ticket counter; nothing
+//   waits) finds the K-th largest 64-bit key (ordered score, inverted id) by
+//   8-bit radix passes from the top with a parallel bin scan, stopping once
+//   the boundary bin is kept whole, and compacts the kept ids in ascending
+//   order.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <climits>
 #include <mutex>
 
 #include "internal.h"
@@ -36,7 +40,7 @@ constexpr int kSplits = 128;         // max query-mean slices per (problem, grou
 constexpr int kMeanThreadsMax = 1024;  // query mean: one thread per 16-byte column of a token
 constexpr int kScoreThreads = 256;   // 8 warps x 8 pages per CTA
 constexpr int kPagesPerScoreCta = 64;
-constexpr int kSelectThreads = 1024;
+
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -93,11 +97,14 @@ __device__ __forceinline__ int problem_npast(const Problems& pb, int b) {
 template <int D>
 __global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
     const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, const Problems pb, int Hq,
-    int G) {
+    int G, unsigned int* __restrict__ tickets, int n_tickets) {
   extern __shared__ float col_sum[];  // [Hq][D]
   constexpr int VPR = D / 8;          // 16-byte vectors per (token, head) row
   constexpr int U = 4;                // rows in flight per thread
   const int split = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  // the next kernel on the stream counts finished CTAs from zero
+  if (split == 0 && b == 0)
+    for (int i = t; i < n_tickets; i += blockDim.x) tickets[i] = 0u;
   const int ncol = Hq * VPR;          // 16-byte vectors per token
   int r0, r1;
   problem_rows(pb, b, r0, r1);
@@ -139,121 +146,32 @@ __global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
   }
 }
 
-// grid (problems, Hkv), D threads: q_bar = (sum of the slice partials, in a
-// fixed order) / (rows * G), once per (problem, group).
-__global__ void qbar_kernel(const float* __restrict__ partial, float* __restrict__ qbar,
-                            const Problems pb, int G, int D) {
-  const int b = blockIdx.x, g = blockIdx.y, Hkv = gridDim.y, dd = threadIdx.x;
-  int r0, r1;
-  problem_rows(pb, b, r0, r1);
-  const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
-  const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D;
-  // eight independent chains (eight loads in flight), combined in a fixed order
-  float s8[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) s8[e] = 0.f;
-  int i = 0;
-  for (; i + 8 <= pb.splits; i += 8) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s8[e] += __ldg(pp + (static_cast<size_t>(i + e) * Hkv + g) * D + dd);
-  }
-  for (; i < pb.splits; ++i) s8[i & 7] += __ldg(pp + (static_cast<size_t>(i) * Hkv + g) * D + dd);
-  const float s = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-  qbar[(static_cast<size_t>(b) * Hkv + g) * D + dd] = rows > 0.f ? s / rows : 0.f;
-}
-
 __device__ __forceinline__ uint32_t order_f32(float f) {
   // monotone map of fp32 onto uint32 (larger float -> larger integer)
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// ---------------------------------------------------------------- page scores
-// grid (ceil(max_past / 64), Hkv, problems).  Every CTA of a problem reduces
-// its slices' partials in the same fixed order (so all use the identical
-// q_bar), then each warp scores 8 pages.  Key = (ordered score << 32) |
-// (~logical id), stored at [problem][group][max_past].
-template <int D>
-__global__ void __launch_bounds__(kScoreThreads) page_score_kernel(
-    const float* __restrict__ qbar, const float* __restrict__ summary,
-    const int32_t* __restrict__ page_table, const Problems pb, int Hkv,
-    int num_pool_pages, unsigned long long* __restrict__ keys, float* __restrict__ out_scores) {
-  const int g = blockIdx.y, b = blockIdx.z, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n_past = problem_npast(pb, b);
-  if (static_cast<int>(blockIdx.x) * kPagesPerScoreCta >= n_past) return;  // whole CTA
-  const float* qb = qbar + (static_cast<size_t>(b) * Hkv + g) * D;
-  constexpr int PW = kPagesPerScoreCta / (kScoreThreads / 32);  // pages per warp
-  const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
-  constexpr int EPL = D / 32;  // elements per lane
-  float qv[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) qv[e] = __ldg(qb + lane * EPL + e);
-  float acc[PW];
-#pragma unroll
-  for (int i = 0; i < PW; ++i) {
-    const int p = p0 + i;
-    acc[i] = 0.f;
-    if (p < n_past) {
-      int phys = __ldg(page_table + p);
-      if (phys < 0 || phys >= num_pool_pages) {
-        if (lane == 0) atomicOr(pb.status, OOMB_DEV_BAD_PAGE);
-        phys = 0;
-      }
-      const float* srow = summary + (static_cast<size_t>(phys) * Hkv + g) * D + lane * EPL;
-      if (EPL == 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(srow));
-        acc[i] = a.x * qv[0] + a.y * qv[1] + a.z * qv[2] + a.w * qv[3];
-      } else {
-        const float2 a = __ldg(reinterpret_cast<const float2*>(srow));
-        acc[i] = a.x * qv[0] + a.y * qv[1];
-      }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < PW; ++i) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-  }
-  if (lane < PW) {
-    float mine = 0.f;
-#pragma unroll
-    for (int i = 0; i < PW; ++i)
-      if (lane == i) mine = acc[i];
-    const int p = p0 + lane;
-    if (p < n_past) {
-      const size_t row = (static_cast<size_t>(b) * Hkv + g) * pb.max_past;
-      if (out_scores) out_scores[row + p] = mine;
-      keys[row + p] = (static_cast<unsigned long long>(order_f32(mine)) << 32) |
-                      static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
-    }
-  }
-}
-
 // ---------------------------------------------------------------- select
-// One CTA per (group, problem): the K-th largest candidate key by 8-bit radix
-// passes from the top, each with a parallel suffix scan over the 256 bins;
-// stops early once the boundary bin is taken whole.  Then compacts kept ids in
-// ascending order.
-__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
-    const unsigned long long* __restrict__ keys_all, const int32_t* __restrict__ page_table,
-    const Problems pb, int top_k, int n_recent, int num_pool_pages,
-    int32_t* __restrict__ out_logical, int32_t* __restrict__ out_physical,
-    int32_t* __restrict__ out_count) {
+// The K-th largest candidate key of one (problem, group) by 8-bit radix passes
+// from the top, each with a parallel suffix scan over the 256 bins; stops
+// early once the boundary bin is taken whole.  Then compacts the kept ids in
+// ascending order.  Run by one CTA of NT threads (NT >= 256).
+template <int NT>
+__device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
+                                 const int32_t* __restrict__ page_table, int n_past, int top_k,
+                                 int n_recent, int num_pool_pages, int32_t* __restrict__ out_l,
+                                 int32_t* __restrict__ out_p, int32_t* __restrict__ out_count) {
   __shared__ unsigned int hist[256];
   __shared__ unsigned int warp_tot[8];
   __shared__ unsigned long long kth_sh;
   __shared__ int need_sh, done_sh;
-  __shared__ int warp_sum[kSelectThreads / 32];
+  __shared__ int warp_sum[NT / 32];
   __shared__ int running_sh;
-  const int g = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int n_past = problem_npast(pb, b);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int max_sel = top_k + n_recent;
   const int n_cand = max(0, n_past - n_recent);
   const int k_eff = min(top_k, n_cand);
-  const size_t row = static_cast<size_t>(b) * gridDim.x + g;
-  const unsigned long long* keys = keys_all + row * pb.max_past;
-  int32_t* out_l = out_logical + row * max_sel;
-  int32_t* out_p = out_physical ? out_physical + row * max_sel : nullptr;
 
   if (t == 0) {
     kth_sh = 0ull;  // with k_eff >= n_cand every candidate is kept
@@ -266,7 +184,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
     for (int shift = 56; shift >= 0; shift -= 8) {
       if (t < 256) hist[t] = 0u;
       __syncthreads();
-      for (int p = t; p < n_cand; p += kSelectThreads) {
+      for (int p = t; p < n_cand; p += NT) {
         const unsigned long long k = keys[p];
         if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255ull], 1u);
       }
@@ -309,7 +227,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
 
   if (t == 0) running_sh = 0;
   __syncthreads();
-  for (int base = 0; base < n_past; base += kSelectThreads) {
+  for (int base = 0; base < n_past; base += NT) {
     const int p = base + t;
     int keep = 0;
     if (p < n_cand) keep = (k_eff >= n_cand) || (k_eff > 0 && keys[p] >= kth);
@@ -330,16 +248,129 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
     __syncthreads();
     if (t == 0) {
       int tot = 0;
-      for (int w = 0; w < kSelectThreads / 32; ++w) tot += warp_sum[w];
+      for (int w = 0; w < NT / 32; ++w) tot += warp_sum[w];
       running_sh += tot;
     }
     __syncthreads();
   }
-  if (t == 0) out_count[row] = min(running_sh, max_sel);
+  if (t == 0) *out_count = min(running_sh, max_sel);
 }
 
-// Workspace: partials [problems][splits <= 128][Hkv][d] fp32, q_bar
-// [problems][Hkv][d] fp32, then keys [problems][Hkv][max(max_past, 1)] u64.
+// ---------------------------------------------------------------- scores + select
+// grid (max(1, ceil(max_past / 64)), Hkv, problems), kScoreThreads threads.
+// q_bar: thread t sums splits [64 (t / D), ...) of column t % D in a fixed order
+// (eight chains, sixteen loads in flight), the two halves are added in a
+// fixed order and divided by rows * G.  Key = (ordered score << 32) |
+// (~logical id), stored at [problem][group][max_past].  The CTA whose ticket
+// is the last of its (problem, group) then runs the select.
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
+    const float* __restrict__ partial, const float* __restrict__ summary,
+    const int32_t* __restrict__ page_table, const Problems pb, int G, int Hkv,
+    int num_pool_pages, unsigned long long* __restrict__ keys, float* __restrict__ out_scores,
+    unsigned int* __restrict__ tickets, int top_k, int n_recent,
+    int32_t* __restrict__ out_logical, int32_t* __restrict__ out_physical,
+    int32_t* __restrict__ out_count) {
+  static_assert(kScoreThreads == 2 * 128 && D <= 128, "q_bar reduction layout");
+  __shared__ float qs[2][D];
+  __shared__ int last_sh;
+  const int g = blockIdx.y, b = blockIdx.z, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int n_past = problem_npast(pb, b);
+  const int n_ctas = max(1, (n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta);
+  if (static_cast<int>(blockIdx.x) >= n_ctas) return;  // beyond this problem's pages
+
+  // q_bar of (problem b, group g) from the query-mean partials
+  {
+    const int dd = t % 128, half = t / 128;
+    if (dd < D) {
+      const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D + g * D + dd;
+      const int lo = min(pb.splits, half * 64), hi = min(pb.splits, lo + 64);
+      float s8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+      int i = lo;
+      for (; i + 16 <= hi; i += 16) {
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = __ldg(pp + static_cast<size_t>(i + e) * Hkv * D);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
+      }
+      for (; i < hi; ++i) s8[i & 7] += __ldg(pp + static_cast<size_t>(i) * Hkv * D);
+      qs[half][dd] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+    }
+  }
+  __syncthreads();
+  int r0, r1;
+  problem_rows(pb, b, r0, r1);
+  const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
+  const size_t row = (static_cast<size_t>(b) * Hkv + g);
+  constexpr int PW = kPagesPerScoreCta / (kScoreThreads / 32);  // pages per warp
+  constexpr int EPL = D / 32;                                   // elements per lane
+  float qv[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int dd = lane * EPL + e;
+    qv[e] = rows > 0.f ? (qs[0][dd] + qs[1][dd]) / rows : 0.f;
+  }
+  const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
+  float acc[PW];
+#pragma unroll
+  for (int i = 0; i < PW; ++i) {
+    const int p = p0 + i;
+    acc[i] = 0.f;
+    if (p < n_past) {
+      int phys = __ldg(page_table + p);
+      if (phys < 0 || phys >= num_pool_pages) {
+        if (lane == 0) atomicOr(pb.status, OOMB_DEV_BAD_PAGE);
+        phys = 0;
+      }
+      const float* srow = summary + (static_cast<size_t>(phys) * Hkv + g) * D + lane * EPL;
+      if (EPL == 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(srow));
+        acc[i] = a.x * qv[0] + a.y * qv[1] + a.z * qv[2] + a.w * qv[3];
+      } else {
+        const float2 a = __ldg(reinterpret_cast<const float2*>(srow));
+        acc[i] = a.x * qv[0] + a.y * qv[1];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < PW; ++i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+  }
+  if (lane < PW) {
+    float mine = 0.f;
+#pragma unroll
+    for (int i = 0; i < PW; ++i)
+      if (lane == i) mine = acc[i];
+    const int p = p0 + lane;
+    if (p < n_past) {
+      if (out_scores) out_scores[row * pb.max_past + p] = mine;
+      keys[row * pb.max_past + p] =
+          (static_cast<unsigned long long>(order_f32(mine)) << 32) |
+          static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
+    }
+  }
+  // the last CTA of this (problem, group) to get here selects (its keys and
+  // every other CTA's are visible once their fences precede the ticket)
+  __threadfence();
+  __syncthreads();
+  if (t == 0) last_sh = atomicAdd(&tickets[row], 1u) == static_cast<unsigned>(n_ctas - 1);
+  __syncthreads();
+  if (!last_sh) return;
+  __threadfence();
+  const int max_sel = top_k + n_recent;
+  select_pages_cta<kScoreThreads>(keys + row * pb.max_past, page_table, n_past, top_k, n_recent,
+                                  num_pool_pages, out_logical + row * max_sel,
+                                  out_physical ? out_physical + row * max_sel : nullptr,
+                                  out_count + row);
+}
+
+// Workspace: partials [problems][splits <= 128][Hkv][d] fp32, a region of
+// [problems][Hkv][d] fp32 whose first problems * Hkv words are the select
+// tickets, then keys [problems][Hkv][max(max_past, 1)] u64.
 size_t workspace_bytes_for(int64_t problems, int Hkv, int D, int max_past) {
   const size_t partial = static_cast<size_t>(problems) * kSplits * Hkv * D * 4;
   const size_t qbar = static_cast<size_t>(problems) * Hkv * D * 4;
@@ -347,7 +378,7 @@ size_t workspace_bytes_for(int64_t problems, int Hkv, int D, int max_past) {
   return align256(partial) + align256(qbar) + align256(keys);
 }
 
-// Launches the three kernels for `n_problems` problems on `s`.
+// Launches the two kernels for `n_problems` problems on `s`.
 oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
                         const Problems& pb_in, int n_problems, const int32_t* d_page_table,
                         int top_k, int n_recent, int32_t* d_out_logical, int32_t* d_out_physical,
@@ -360,32 +391,33 @@ oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
   const size_t partial_bytes = align256(static_cast<size_t>(n_problems) * kSplits * Hkv * D * 4);
   const size_t qbar_bytes = align256(static_cast<size_t>(n_problems) * Hkv * D * 4);
   float* partial = static_cast<float*>(scratch);
-  float* qbar = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + partial_bytes);
+  unsigned int* tickets =
+      reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(scratch) + partial_bytes);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(
       static_cast<uint8_t*>(scratch) + partial_bytes + qbar_bytes);
+  const int n_tickets = n_problems * Hkv;
   const auto* q = static_cast<const __nv_bfloat16*>(d_q);
   // one thread per 16-byte column of a token row, a multiple of 32, at most 1024
   const int ncol = num_q_heads * D / 8;
   const int mean_threads = ncol >= kMeanThreadsMax ? kMeanThreadsMax : ((ncol + 31) / 32) * 32;
   const size_t mean_smem = static_cast<size_t>(num_q_heads) * D * 4;
   dim3 g1(pb.splits, n_problems);
-  dim3 g2((pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta, Hkv, n_problems);
+  dim3 g2(std::max(1, (pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta), Hkv,
+          n_problems);
   if (D == 128)
-    qmean_partial_kernel<128><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G);
+    qmean_partial_kernel<128><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G,
+                                                                  tickets, n_tickets);
   else
-    qmean_partial_kernel<64><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G);
-  qbar_kernel<<<dim3(n_problems, Hkv), D, 0, s>>>(partial, qbar, pb, G, D);
-  if (pb.max_past > 0) {
-    if (D == 128)
-      page_score_kernel<128><<<g2, kScoreThreads, 0, s>>>(qbar, pool->summary, d_page_table, pb,
-                                                          Hkv, d.num_pages, keys, d_out_scores);
-    else
-      page_score_kernel<64><<<g2, kScoreThreads, 0, s>>>(qbar, pool->summary, d_page_table, pb,
-                                                         Hkv, d.num_pages, keys, d_out_scores);
-  }
-  topk_select_kernel<<<dim3(Hkv, n_problems), kSelectThreads, 0, s>>>(
-      keys, d_page_table, pb, top_k, n_recent, d.num_pages, d_out_logical, d_out_physical,
-      d_out_count);
+    qmean_partial_kernel<64><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G,
+                                                                 tickets, n_tickets);
+  if (D == 128)
+    page_score_select_kernel<128><<<g2, kScoreThreads, 0, s>>>(
+        partial, pool->summary, d_page_table, pb, G, Hkv, d.num_pages, keys, d_out_scores,
+        tickets, top_k, n_recent, d_out_logical, d_out_physical, d_out_count);
+  else
+    page_score_select_kernel<64><<<g2, kScoreThreads, 0, s>>>(
+        partial, pool->summary, d_page_table, pb, G, Hkv, d.num_pages, keys, d_out_scores,
+        tickets, top_k, n_recent, d_out_logical, d_out_physical, d_out_count);
   return oomb::check_launch();
 }
 
@@ -510,6 +542,91 @@ extern "C" oomb_status oomb_local_pages(const oomb_pool* pool, const int32_t* d_
   local_pages_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       d_page_table, n_past, window, Hkv, pool->desc.num_pages, d_out_pages, d_out_count,
       pool->d_status);
+  return oomb::check_launch();
+}
+
+// ---------------------------------------------------------------- per-query-page lists
+// One thread per (128-row query tile, group): merges the ascending logical
+// lists of the tile's query pages (at most 8) into one ascending union,
+// writing each union entry's physical id and the bit set of the query pages
+// that listed it.
+namespace {
+
+__global__ void qpage_lists_kernel(const int32_t* __restrict__ sel_logical,
+                                   const int32_t* __restrict__ sel_physical,
+                                   const int32_t* __restrict__ sel_count, int n_qpages,
+                                   int per_tile, int n_qtiles, int Hkv, int max_sel,
+                                   int32_t* __restrict__ out_pages, uint8_t* __restrict__ out_masks,
+                                   int32_t* __restrict__ out_count, int max_union,
+                                   uint32_t* status) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n_qtiles * Hkv) return;
+  const int t = e / Hkv, g = e % Hkv;
+  const int b0 = t * per_tile, nb = min(per_tile, n_qpages - b0);
+  int cur[8], cnt[8];
+  for (int b = 0; b < nb; ++b) {
+    int c = sel_count[static_cast<size_t>(b0 + b) * Hkv + g];
+    if (c < 0 || c > max_sel) {
+      atomicOr(status, OOMB_DEV_BAD_COUNT);
+      c = c < 0 ? 0 : max_sel;
+    }
+    cnt[b] = c;
+    cur[b] = 0;
+  }
+  const size_t out0 = static_cast<size_t>(e) * max_union;
+  int n = 0;
+  while (true) {
+    int lo = INT_MAX, phys = 0;
+    for (int b = 0; b < nb; ++b) {
+      if (cur[b] < cnt[b]) {
+        const size_t i = (static_cast<size_t>(b0 + b) * Hkv + g) * max_sel + cur[b];
+        const int l = sel_logical[i];
+        if (l < lo) {
+          lo = l;
+          phys = sel_physical[i];
+        }
+      }
+    }
+    if (lo == INT_MAX) break;
+    uint32_t m = 0;
+    for (int b = 0; b < nb; ++b) {
+      if (cur[b] < cnt[b] &&
+          sel_logical[(static_cast<size_t>(b0 + b) * Hkv + g) * max_sel + cur[b]] == lo) {
+        m |= 1u << b;
+        ++cur[b];
+      }
+    }
+    out_pages[out0 + n] = phys;
+    out_masks[out0 + n] = static_cast<uint8_t>(m);
+    ++n;
+  }
+  out_count[e] = n;
+}
+
+}  // namespace
+
+extern "C" oomb_status oomb_qpage_lists(oomb_pool* pool, const int32_t* d_sel_logical,
+                                        const int32_t* d_sel_physical, const int32_t* d_sel_count,
+                                        int32_t chunk_len, int32_t max_sel, int32_t* d_out_pages,
+                                        uint8_t* d_out_masks, int32_t* d_out_count,
+                                        int32_t max_union, void* stream) {
+  if (!pool || pool->desc.location == OOMB_LOC_HOST) return OOMB_ERR_INVALID_ARG;
+  const int P = pool->desc.page_size, Hkv = pool->desc.num_kv_heads;
+  if (chunk_len <= 0 || chunk_len % P != 0 || max_sel <= 0) return OOMB_ERR_INVALID_ARG;
+  if (!d_sel_logical || !d_sel_physical || !d_sel_count || !d_out_pages || !d_out_masks ||
+      !d_out_count)
+    return OOMB_ERR_INVALID_ARG;
+  const int per_tile = 128 / P;  // query pages per 128-row tile (1 .. 8)
+  const int n_qpages = chunk_len / P;
+  if (static_cast<int64_t>(max_union) < static_cast<int64_t>(std::min(per_tile, n_qpages)) *
+                                            max_sel)
+    return OOMB_ERR_INVALID_ARG;
+  const int n_qtiles = (chunk_len + 127) / 128;
+  oomb::DeviceGuard guard(pool->desc.device);
+  const int n = n_qtiles * Hkv;
+  qpage_lists_kernel<<<(n + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      d_sel_logical, d_sel_physical, d_sel_count, n_qpages, per_tile, n_qtiles, Hkv, max_sel,
+      d_out_pages, d_out_masks, d_out_count, max_union, pool->d_status);
   return oomb::check_launch();
 }
 

@@ -16,6 +16,8 @@ Workloads (one attention layer each):
                 plus the 2 most recent pages per chunk and KV-head group.
 * ``qwen1m_topk_offload``  as ``qwen256k_topk`` with 256 chunks (16384 pages),
                 past KV and gradients in pinned host memory.
+* ``qwen256k_topk_qpage``  as ``qwen256k_topk`` with one selection per 64-token
+                query page instead of per chunk.
 
 Every draw is fp32 ``torch.randn`` from a CPU generator seeded per (workload
 seed, chunk, tensor), then rounded to bf16 with round-to-nearest-even
@@ -48,6 +50,7 @@ class Workload:
     host_resident: bool = False   # past KV and grads in pinned host memory
     window: int = 0               # > 0: recent-only lists of this many past pages
     qtile_topk: bool = False      # Top-K per 128-row query tile instead of per chunk
+    qpage_topk: bool = False      # Top-K per query page (page_size rows) instead of per chunk
 
     @property
     def group_size(self) -> int:
@@ -89,6 +92,10 @@ WORKLOADS = {
     "qwen256k_topk_qtile": Workload("qwen256k_topk_qtile", 28, 4, 128, 64, 4096, 64, seed=1007,
                                     shuffle_pages=True, page_direction=0.5, top_k=64,
                                     n_recent=2, qtile_topk=True),
+    # one Top-K selection per 64-token query page (per-query-page sparsity)
+    "qwen256k_topk_qpage": Workload("qwen256k_topk_qpage", 28, 4, 128, 64, 4096, 64, seed=1008,
+                                    shuffle_pages=True, page_direction=0.5, top_k=64,
+                                    n_recent=2, qpage_topk=True),
     # recent-only page lists: the last 64 past pages (4096 tokens) + the chunk
     "qwen256k_local": Workload("qwen256k_local", 28, 4, 128, 64, 4096, 64, seed=1006,
                                shuffle_pages=True, window=64),

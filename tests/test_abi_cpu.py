@@ -158,6 +158,8 @@ def test_newer_entry_points_reject_host_pools_without_touching_cuda():
                                     None) == L.ERR_INVALID_ARG
         assert lib.oomb_block_copy(None, pool, None, None, 0, None) == L.ERR_INVALID_ARG
         assert lib.oomb_selftest_wait_limit(pool, None) == L.ERR_INVALID_ARG
+        assert lib.oomb_qpage_lists(pool, None, None, None, 64, 4, None, None, None, 8,
+                                    None) == L.ERR_INVALID_ARG
     finally:
         L.pool_destroy(pool)
 

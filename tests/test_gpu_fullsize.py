@@ -29,6 +29,10 @@ out of reach at these sizes, so the oracle is evaluated on samples:
 * Top-K page ids of every chunk bit for bit, except pages whose fp64 score
   lies within 1e-5 of the K-th score.
 
+The per-query-page Top-K workload (one selection per 64-token query page)
+is checked on its selections, sampled rows (each against its own query
+page's pages) and the gradient-pool sums.
+
 The 1M offloaded run (KV and gradients in pinned host memory, selected pages
 prefetched into a staging pool) is checked against the same workload with
 every page in HBM: identical selections, bit-equal forward outputs and dQ on
@@ -121,9 +125,11 @@ def _sample_rows(C, seed):
     return np.sort(np.concatenate([[0, C - 1], inner]))
 
 
-def _check_rows(w, run, cpu, kf, vf, c, selected=None):
+def _check_rows(w, run, cpu, kf, vf, c, selected=None, block_rows=None):
     """O, LSE, dQ of ROWS sampled rows of every head of chunk c against the
-    oracle over every key those rows see."""
+    oracle over every key those rows see.  `selected`: per group the kept
+    pages (None: dense); with `block_rows`, per block of that many rows a
+    per-group selection (the rows of block b see selected[b][g])."""
     C, Hq, Hkv = w.chunk_len, w.num_q_heads, w.num_kv_heads
     G = Hq // Hkv
     rows = _sample_rows(C, 9000 + c)
@@ -134,13 +140,20 @@ def _check_rows(w, run, cpu, kf, vf, c, selected=None):
     q = cpu[c]["q"][rows].double().numpy()
     do = cpu[c]["do"][rows].double().numpy()
     o_ref, lse_ref, dq_ref = np.zeros_like(o_gpu), np.zeros_like(lse_gpu), np.zeros_like(dq_gpu)
-    for g in range(Hkv):
-        tok = _tokens(w, c, None if selected is None else selected[g])
-        kk = kf[tok, g].astype(np.float64)
-        vv = vf[tok, g].astype(np.float64)
-        for h in range(g * G, (g + 1) * G):
-            o_ref[:, h], lse_ref[h], dq_ref[:, h] = chunk_rows_backward(
-                q[:, h], do[:, h], c * C + rows, kk, vv, tok, w.softmax_scale)
+    if block_rows is None:
+        groups = [(np.arange(len(rows)), selected)]
+    else:
+        blk = rows // block_rows
+        groups = [(np.nonzero(blk == b)[0], selected[b]) for b in np.unique(blk)]
+    for sel_rows, sel in groups:
+        for g in range(Hkv):
+            tok = _tokens(w, c, None if sel is None else sel[g])
+            kk = kf[tok, g].astype(np.float64)
+            vv = vf[tok, g].astype(np.float64)
+            for h in range(g * G, (g + 1) * G):
+                o_ref[sel_rows, h], lse_ref[h, sel_rows], dq_ref[sel_rows, h] = \
+                    chunk_rows_backward(q[sel_rows, h], do[sel_rows, h], c * C + rows[sel_rows],
+                                        kk, vv, tok, w.softmax_scale)
     assert rel_l2(o_gpu, o_ref) <= FWD_REL, (c, rel_l2(o_gpu, o_ref))
     assert np.max(np.abs(o_gpu - o_ref)) <= FWD_ABS, c
     assert rel_l2(lse_gpu, lse_ref) <= FWD_REL, c
@@ -289,6 +302,37 @@ def test_fullsize_qwen256k_topk():
         for c in (1, N // 2, N - 1):
             _check_rows(w, run, cpu, kf, vf, c, _selected(run, c))
         _check_single_chunk_grads(w, run, cpu, kf, vf, N - 1, _selected(run, N - 1))
+    finally:
+        _close(run)
+
+
+def test_fullsize_qwen256k_topk_per_query_page():
+    """256K Top-64 + 2 recent pages per 64-token query page and group: the
+    selections of chunks 1, N/2 and N-1 (every query page), sampled rows of
+    those chunks each against its own query page's pages, and the
+    gradient-pool sums."""
+    w = synth.WORKLOADS["qwen256k_topk_qpage"]
+    cpu = _draw(w)
+    kf, vf = _keys(cpu)
+    run = _run(w, True, cpu)
+    try:
+        N, P, Hkv = w.num_chunks, w.page_size, w.num_kv_heads
+        kbar_all = page_key_means(kf, P)
+        _check_sums(w, run)
+        for c in (1, N // 2, N - 1):
+            n_past = c * w.pages_per_chunk
+            cnt = run.sel_n[c].cpu().numpy()
+            lg = run.sel_l[c].cpu().numpy()
+            sel = [[lg[b, g, :cnt[b, g]].tolist() for g in range(Hkv)] for b in range(len(cnt))]
+            for b in range(len(cnt)):
+                ref = page_scores(group_query_means(cpu[c]["q"][b * P:(b + 1) * P], Hkv),
+                                  kbar_all[:n_past])
+                want = select_pages(ref, n_past, w.top_k, w.n_recent)
+                for g in range(Hkv):
+                    kth = kth_score(ref[g], n_past, w.top_k, w.n_recent)
+                    for p in set(sel[b][g]) ^ set(want[g]):
+                        assert kth is not None and abs(ref[g, p] - kth) <= TIE, (c, b, g, p)
+            _check_rows(w, run, cpu, kf, vf, c, sel, block_rows=P)
     finally:
         _close(run)
 
