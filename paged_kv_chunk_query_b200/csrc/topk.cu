@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
     int G, unsigned int* __restrict__ tickets, int n_tickets) {
   extern __shared__ float col_sum[];  // [Hq][D]
   constexpr int VPR = D / 8;          // 16-byte vectors per (token, head) row
-  constexpr int U = 4;                // rows in flight per thread
+  constexpr int U = 8;                // rows in flight per thread
   const int split = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
   // the next kernel on the stream counts finished CTAs from zero
   if (split == 0 && b == 0)
@@ -184,9 +184,20 @@ __device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
     for (int shift = 56; shift >= 0; shift -= 8) {
       if (t < 256) hist[t] = 0u;
       __syncthreads();
-      for (int p = t; p < n_cand; p += NT) {
-        const unsigned long long k = keys[p];
-        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255ull], 1u);
+      // eight keys per thread in flight before their histogram updates
+      for (int base = 0; base < n_cand; base += 8 * NT) {
+        unsigned long long kv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int p = base + u * NT + t;
+          kv[u] = p < n_cand ? keys[p] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int p = base + u * NT + t;
+          if (p < n_cand && (kv[u] & mask) == prefix)
+            atomicAdd(&hist[(kv[u] >> shift) & 255ull], 1u);
+        }
       }
       __syncthreads();
       // every thread reads the remaining count here, before the barrier that
