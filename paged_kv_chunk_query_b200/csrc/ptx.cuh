@@ -273,22 +273,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
-// Register budget of the executing warpgroup (all 128 threads execute it):
-// raise to / lower to N registers per thread.  The launch's registers
-// (threads x registers per thread at launch) bound the sum over warpgroups.
-template <uint32_t N>
-__device__ __forceinline__ void warpgroup_reg_raise() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void warpgroup_reg_lower() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
 
-// Warp-uniform bounded wait: lane 0 polls, the result is broadcast, and the
+// Warp-uniform bounded wait.  Every lane first tests the phase once (no
+// divergence when it has already completed, the common case inside a
+// pipelined loop); otherwise lane 0 polls, the result is broadcast, and the
 // warp re-converges before any warp-collective tcgen05 operation follows.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
                                           const volatile int* abort) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
