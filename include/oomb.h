@@ -138,9 +138,9 @@ typedef struct oomb_attn_args {
   const int32_t* cur_pages;   /* device int32 [chunk_len/page_size] physical ids      */
   float softmax_scale;        /* usually 1/sqrt(head_dim)                             */
   /* 0: one past list per group for the whole chunk (layouts above).
-   * 1: one past list per 128-row query tile and group ([pt] §2C: the pages
-   *    relevant to each query page; the query page is the kernels' 128-row
-   *    query tile): past_pages [n_qtiles][num_kv_heads][max_past] and
+   * 1: one past list per 128-row query tile and group (a coarser form of
+   *    mode 2 below, one list for two 64-token query pages):
+   *    past_pages [n_qtiles][num_kv_heads][max_past] and
    *    past_counts [n_qtiles][num_kv_heads], n_qtiles = ceil(chunk_len / 128);
    *    rows of query tile t attend to list t (plus the chunk, causally).  The
    *    outputs of oomb_page_topk_batched with one problem per query tile have

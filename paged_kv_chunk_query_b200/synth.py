@@ -88,7 +88,7 @@ WORKLOADS = {
     "qwen256k_topk": Workload("qwen256k_topk", 28, 4, 128, 64, 4096, 64, seed=1003,
                               shuffle_pages=True, page_direction=0.5, top_k=64,
                               n_recent=2),
-    # one Top-K selection per 128-row query tile (per-query-page sparsity)
+    # one Top-K selection per 128-row query tile (two 64-token query pages share one list)
     "qwen256k_topk_qtile": Workload("qwen256k_topk_qtile", 28, 4, 128, 64, 4096, 64, seed=1007,
                                     shuffle_pages=True, page_direction=0.5, top_k=64,
                                     n_recent=2, qtile_topk=True),

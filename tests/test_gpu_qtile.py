@@ -1,5 +1,6 @@
-"""GPU parity: one past-page list per 128-row query tile (per-query-page
-selection) vs the oracle's per-row-block attention.
+"""GPU parity: one past-page list per 128-row query tile (the coarser form
+of per-query-page selection: two 64-token query pages share a list) vs the
+oracle's per-row-block attention.
 
 Tolerances as for the chunk-wide lists: forward O/LSE relative L2 <= 5e-3 and
 max abs <= 1e-2, dQ/dK/dV relative L2 <= 1e-2.  Lists that are the same for
