@@ -282,8 +282,9 @@ oomb_status oomb_qpage_lists(oomb_pool* pool, const int32_t* d_sel_logical,
  * The first call on a device looks up the array's device address (with that
  * device current); make that first call before any stream capture.  All calls
  * share the one array: calls that overlap on the GPU (different streams) race
- * on it and must be ordered by the caller.  No scratch word needs clearing:
- * each call writes what it reads.  The looked-up address is kept per device
+ * on it and must be ordered by the caller.  The caller clears nothing: each
+ * call writes every scratch word it reads, and its first launch zeroes the
+ * counters its second launch counts on.  The looked-up address is kept per device
  * ordinal for the life of the process, so resetting a device
  * (cudaDeviceReset, or tearing down and re-creating its primary context)
  * while this library is loaded is not supported for this entry point. */

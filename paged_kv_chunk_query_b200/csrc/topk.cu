@@ -650,7 +650,8 @@ extern "C" oomb_status oomb_qpage_lists(oomb_pool* pool, const int32_t* d_sel_lo
 // taken from the file-scope device array below instead of a caller workspace.
 // Every GPU that loads the library holds this array until the process exits.
 // All calls share it and it keeps the last call's contents; the kernels write
-// every scratch word before reading it, so nothing needs clearing, but calls
+// every scratch word before reading it (the first launch zeroes the select
+// tickets the second counts on), so the caller clears nothing, but calls
 // that overlap on the GPU (on different streams) race on it.
 namespace {
 

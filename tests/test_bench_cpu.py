@@ -79,3 +79,19 @@ def test_flop_accounting_matches_the_published_workload_figures():
     w = W["qwen256k"]
     assert bench.step_pairs(synth.Workload("x", 28, 4, 128, 64, 4096, 64, seed=1,
                                            window=4096), False) == bench.step_pairs(w, False)
+
+
+def test_clock_scaled_peak_and_step_fractions():
+    """The burst tensor peak scales with the SM clock the run held; without a
+    clock record there is no scaled peak (and no scaled fraction)."""
+    import bench
+    assert bench.clock_scaled_peak(1654.6, 1965.0, 1965.0) == 1654.6
+    assert abs(bench.clock_scaled_peak(1654.6, 1710.0, 1965.0) - 1654.6 * 1710.0 / 1965.0) < 1e-9
+    assert bench.clock_scaled_peak(1654.6, None, 1965.0) is None
+    assert bench.clock_scaled_peak(1654.6, 1710.0, None) is None
+    peaks = {"bf16": 1654.6, "bf16_sustained": 1359.8, "sm_max_mhz": 1965.0}
+    f = bench.step_fractions(784.1, peaks, 1710.0)
+    assert abs(f["of_sustained"] - 784.1 / 1359.8) < 1e-12
+    assert abs(f["of_burst"] - 784.1 / 1654.6) < 1e-12
+    assert abs(f["of_clock_normalised"] - 784.1 / (1654.6 * 1710.0 / 1965.0)) < 1e-12
+    assert bench.step_fractions(784.1, peaks, None)["of_clock_normalised"] is None

@@ -31,7 +31,8 @@ out of reach at these sizes, so the oracle is evaluated on samples:
 
 The per-query-page Top-K workload (one selection per 64-token query page)
 is checked on its selections, sampled rows (each against its own query
-page's pages) and the gradient-pool sums.
+page's pages), the gradient-pool sums, and one chunk's dK / dV on sampled
+pages (each block of rows contributing through its own key set).
 
 The 1M offloaded run (KV and gradients in pinned host memory, selected pages
 prefetched into a staging pool) is checked against the same workload with
@@ -309,8 +310,8 @@ def test_fullsize_qwen256k_topk():
 def test_fullsize_qwen256k_topk_per_query_page():
     """256K Top-64 + 2 recent pages per 64-token query page and group: the
     selections of chunks 1, N/2 and N-1 (every query page), sampled rows of
-    those chunks each against its own query page's pages, and the
-    gradient-pool sums."""
+    those chunks each against its own query page's pages, the gradient-pool
+    sums, and the last chunk's dK / dV on sampled pages."""
     w = synth.WORKLOADS["qwen256k_topk_qpage"]
     cpu = _draw(w)
     kf, vf = _keys(cpu)
@@ -333,8 +334,66 @@ def test_fullsize_qwen256k_topk_per_query_page():
                     for p in set(sel[b][g]) ^ set(want[g]):
                         assert kth is not None and abs(ref[g, p] - kth) <= TIE, (c, b, g, p)
             _check_rows(w, run, cpu, kf, vf, c, sel, block_rows=P)
+        _check_single_chunk_grads_qpage(w, run, cpu, kf, vf, N - 1)
     finally:
         _close(run)
+
+
+def _check_single_chunk_grads_qpage(w, run, cpu, kf, vf, c):
+    """As _check_single_chunk_grads, for per-query-page lists: each block of
+    page_size rows has its own key set, so the oracle's contribution to a
+    sampled key is summed over the blocks whose set holds it."""
+    C, Hq, Hkv, P = w.chunk_len, w.num_q_heads, w.num_kv_heads, w.page_size
+    G = Hq // Hkv
+    _, grad, _ = pk.pool_views(run.pool)
+    grad.zero_()
+    x = run.inputs[c]
+    for step in (pk.BWD_PREPROCESS, pk.BWD_DKDV):
+        pk.chunk_attn_bwd(run.pool, x["q"], run.o[c], run.lse[c], x["do"], run.dq[c],
+                          run.deltas[c], run.u_pages[c], run.u_cnt[c], run.cur[c],
+                          w.softmax_scale, step=step, past_masks=run.masks[c])
+    torch.cuda.synchronize()
+    assert pk.get_device_status(run.pool) == 0
+    cnt = run.sel_n[c].cpu().numpy()
+    lg = run.sel_l[c].cpu().numpy()
+    nb = C // P
+    sel = [[lg[b, g, :cnt[b, g]].tolist() for g in range(Hkv)] for b in range(nb)]
+    q = cpu[c]["q"].double().numpy()
+    do = cpu[c]["do"].double().numpy()
+    rng = np.random.default_rng(9700 + c)
+    ppc = w.pages_per_chunk
+    for g in range(Hkv):
+        listed = sorted(set().union(*[set(sel[b][g]) for b in range(nb)]))
+        rest = [p for p in listed if p not in (listed[0], listed[-1])]
+        pick = sorted({listed[0], listed[-1], c * ppc, (c + 1) * ppc - 1} |
+                      set(rng.choice(rest, size=PAGES - 4, replace=False).tolist()))
+        ptok = {p: np.arange(p * P, (p + 1) * P) for p in pick}
+        dk_ref = {p: np.zeros((P, w.head_dim)) for p in pick}
+        dv_ref = {p: np.zeros((P, w.head_dim)) for p in pick}
+        for b in range(nb):
+            tok = _tokens(w, c, sel[b][g])
+            pos_in = {int(t): i for i, t in enumerate(tok)}
+            seen = [p for p in pick if int(ptok[p][0]) in pos_in]
+            if not seen:
+                continue
+            key_idx = np.array([pos_in[int(t)] for p in seen for t in ptok[p]])
+            rows = np.arange(b * P, (b + 1) * P)
+            dk_b, dv_b = chunk_keys_backward(
+                q[rows, g * G:(g + 1) * G], do[rows, g * G:(g + 1) * G], c * C + rows,
+                kf[tok, g].astype(np.float64), vf[tok, g].astype(np.float64), tok, key_idx,
+                w.softmax_scale)
+            for i, p in enumerate(seen):
+                dk_ref[p] += dk_b[i * P:(i + 1) * P]
+                dv_ref[p] += dv_b[i * P:(i + 1) * P]
+        phys = torch.tensor([run.page_table[p] for p in pick], dtype=torch.long,
+                            device=grad.device)
+        blk = to64(grad[phys, g])                      # [pages][2][P][d]
+        dk_gpu = blk[:, 0].reshape(-1, w.head_dim)
+        dv_gpu = blk[:, 1].reshape(-1, w.head_dim)
+        want_k = np.concatenate([dk_ref[p] for p in pick])
+        want_v = np.concatenate([dv_ref[p] for p in pick])
+        assert rel_l2(dk_gpu, want_k) <= BWD_REL, (g, rel_l2(dk_gpu, want_k))
+        assert rel_l2(dv_gpu, want_v) <= BWD_REL, (g, rel_l2(dv_gpu, want_v))
 
 
 def test_fullsize_qwen1m_offload_matches_device_resident():
