@@ -396,15 +396,45 @@ def _check_single_chunk_grads_qpage(w, run, cpu, kf, vf, c):
         assert rel_l2(dv_gpu, want_v) <= BWD_REL, (g, rel_l2(dv_gpu, want_v))
 
 
+class _TokenKeys:
+    """K or V of a long sequence kept as one bf16 CPU tensor [L][Hkv][d];
+    indexing [tokens, g] gives those rows of KV head g as fp32 numpy."""
+
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, idx):
+        tok, g = idx
+        return self.t[torch.as_tensor(tok, dtype=torch.long), g].float().numpy()
+
+
 def test_fullsize_qwen1m_offload_matches_device_resident():
     """1M tokens (16,384 pages, 256 chunks): the offloaded schedule (pinned
     host pools, staging prefetch, gradient write-back) against the same
-    workload with every page in HBM."""
+    workload with every page in HBM, and the last chunk against the oracle.
+
+    Every chunk's K and V, and the last chunk's Q and dO, come from the seeded
+    CPU generator (the other chunks' Q and dO are drawn on the device: they
+    do not enter the last chunk's selection or outputs), so the last chunk's
+    Top-K ids and 256 sampled rows of every head are checked against the
+    oracle over all 16,320 past pages.  The host gradient pool must also
+    hold the two softmax sums (sum over keys of dK_g = 0, of dV_g = sum of dO)."""
     from paged_kv_chunk_query_b200.offload import OffloadRun
     w = synth.WORKLOADS["qwen1m_topk_offload"]
     dev = _dev()
-    N, C, Hq, Hkv = w.num_chunks, w.chunk_len, w.num_q_heads, w.num_kv_heads
-    ins = [synth.device_chunk_inputs(w, c, dev) for c in range(N)]
+    N, C, Hq, Hkv, P, d = (w.num_chunks, w.chunk_len, w.num_q_heads, w.num_kv_heads,
+                           w.page_size, w.head_dim)
+    G = Hq // Hkv
+    with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+        kv_cpu = list(ex.map(lambda c: synth.chunk_inputs(w, c, which=("k", "v")), range(N)))
+    last_cpu = synth.chunk_inputs(w, N - 1, which=("q", "do"))
+    ins = []
+    for c in range(N):
+        x = synth.device_chunk_inputs(w, c, dev)
+        x["k"], x["v"] = kv_cpu[c]["k"].to(dev), kv_cpu[c]["v"].to(dev)
+        if c == N - 1:
+            x["q"], x["do"] = last_cpu["q"].to(dev), last_cpu["do"].to(dev)
+        ins.append(x)
     sample = (1, N // 2, N - 1)
     outs = {c: (torch.empty_like(ins[c]["q"]), torch.empty((Hq, C), dtype=torch.float32,
                                                            device=dev),
@@ -441,7 +471,41 @@ def test_fullsize_qwen1m_offload_matches_device_resident():
             assert (err / ref) ** 0.5 <= 1e-3, (err / ref) ** 0.5
         finally:
             run.close()
+        # the softmax sums on the host gradient pool the offloaded run built
+        dk_sum = torch.zeros((Hkv, d), dtype=torch.float64, device=dev)
+        dv_sum = torch.zeros_like(dk_sum)
+        dk_sq = torch.zeros(Hkv, dtype=torch.float64, device=dev)
+        for a in torch.tensor(off.table, dtype=torch.long).split(512):
+            gg = gh[a].to(dev).double()
+            dk_sum += gg[:, :, 0].sum(dim=(0, 2))
+            dv_sum += gg[:, :, 1].sum(dim=(0, 2))
+            dk_sq += gg[:, :, 0].pow(2).sum(dim=(0, 2, 3))
+        do_sum = torch.zeros_like(dk_sum)
+        for x in ins:
+            do_sum += x["do"].double().view(-1, Hkv, G, d).sum(dim=(0, 2))
+        for g in range(Hkv):
+            assert float(dk_sum[g].norm()) <= 1e-2 * float(dk_sq[g].sqrt()), g
+            assert float((dv_sum[g] - do_sum[g]).norm()) <= 1e-2 * float(do_sum[g].norm()), g
     finally:
         off.close()
-        del ins
-        torch.cuda.empty_cache()
+    # the last chunk against the oracle: its selection over 16,320 past pages
+    # and 256 sampled rows of every head on that selection
+    c = N - 1
+    kbar = np.concatenate([page_key_means(x["k"], P) for x in kv_cpu[:c]])
+    n_past = c * w.pages_per_chunk
+    ref = page_scores(group_query_means(last_cpu["q"], Hkv), kbar)
+    want = select_pages(ref, n_past, w.top_k, w.n_recent)
+    for g in range(Hkv):
+        got = sels[c][g]
+        assert len(got) == w.top_k + w.n_recent and got == sorted(got), g
+        kth = kth_score(ref[g], n_past, w.top_k, w.n_recent)
+        for pg in set(got) ^ set(want[g]):
+            assert kth is not None and abs(ref[g, pg] - kth) <= TIE, (g, pg)
+    kf = _TokenKeys(torch.cat([x["k"] for x in kv_cpu]))
+    vf = _TokenKeys(torch.cat([x["v"] for x in kv_cpu]))
+    cpu = {c: last_cpu}
+    fake = type("R", (), {})()
+    fake.o, fake.lse, fake.dq = ({c: outs[c][0]}, {c: outs[c][1]}, {c: outs[c][2]})
+    _check_rows(w, fake, cpu, kf, vf, c, sels[c])
+    del ins
+    torch.cuda.empty_cache()
