@@ -189,6 +189,9 @@ class Run:
         # delta while chunk c+1's preprocess runs
         self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(N)]
         self.side = torch.cuda.Stream(device=device)
+        # selections of the next chunk run here, beside the current chunk's attention
+        self.sel_stream = torch.cuda.Stream(device=device)
+        self.early_select = True
         self.fwd_stream = torch.cuda.Stream(device=device)
         self.concurrent_bwd = True
         self.fwd_overlap = False
@@ -346,7 +349,13 @@ class Run:
         """One pass over all chunks.  With concurrent_bwd, chunk c's dQ launch
         runs on a second stream next to its dK/dV launch (the two only read
         what the forward and preprocess wrote and write disjoint outputs), so
-        each fills the other's last partial wave of CTAs."""
+        each fills the other's last partial wave of CTAs.  With early_select,
+        chunk c+1's past lists (Top-K or recent pages) are made on a third
+        stream as soon as chunk c's pages are appended: they read only chunk
+        c+1's queries and the page means of chunks 0..c, which the backward
+        does not change, so they run beside chunk c's attention instead of
+        between chunk c's dK/dV and chunk c+1's forward.  All selections share
+        one workspace and so stay in order on that stream."""
         pk, w = self.pk, self.w
         stream = torch.cuda.current_stream()
         side = self.side if self.concurrent_bwd else stream
@@ -366,12 +375,37 @@ class Run:
         ppc = w.pages_per_chunk
         if side is not stream:
             side.wait_stream(stream)
+        early = self.early_select and (self.sparse or self.local)
+        sel = self.sel_stream
+        if early:
+            sel.wait_stream(stream)
+        lists = {}
+
+        def select_next(c):
+            # chunk c's lists on the selection stream, once chunks 0..c-1 are appended
+            appended = torch.cuda.Event()
+            appended.record(stream)
+            sel.wait_event(appended)
+            lists[c] = self.select(c, sel, timed)
+            done = torch.cuda.Event()
+            done.record(sel)
+            lists[c] = lists[c] + (done,)
+
         for c in range(w.num_chunks):
             x = self.inputs[c]
             if c == 0:
                 timed("append", lambda: pk.kv_append(self.pool, self.cur[0], x["k"], x["v"],
                                                      stream))
-            past, cnt, msk = self.select(c, stream, timed)
+            if early:
+                if c + 1 < w.num_chunks:
+                    select_next(c + 1)
+                if c == 0:
+                    past, cnt, msk = None, None, None
+                else:
+                    past, cnt, msk, done = lists.pop(c)
+                    stream.wait_event(done)
+            else:
+                past, cnt, msk = self.select(c, stream, timed)
             o, lse, dq = self.o[c], self.lse[c], self.dq[c]
             s = w.softmax_scale
             delta = self.deltas[c]
@@ -395,32 +429,63 @@ class Run:
                 step=pk.BWD_DKDV, past_masks=msk))
         if side is not stream:
             stream.wait_stream(side)
+        if early:
+            stream.wait_stream(sel)
 
     def time_topk_alone(self, reps=3):
         """Every chunk's Top-K selection back to back (no attention launches in
-        between), on the launching stream: ms for one pass over chunks 1..N-1.
-        The chunks' queries (1.8 GiB together) rotate, so L2 does not hold them."""
+        between): ms for one pass over chunks 1..N-1, (two-launch form from Q,
+        one-launch form from per-group Q sums).  Each pass is captured once in
+        a CUDA graph and replayed (a loop of microsecond launches is bound by
+        host launch cost otherwise).  The chunks' queries (1.8 GiB together)
+        rotate, so L2 does not hold them.  The Q sums are made beforehand, as
+        the projection's epilogue makes them in a full layer."""
         pk, w = self.pk, self.w
-        stream = torch.cuda.current_stream()
         ppc = w.pages_per_chunk
+        C, Hq, Hkv, d = w.chunk_len, w.num_q_heads, w.num_kv_heads, w.head_dim
+        qsums = [x["q"].float().reshape(C, Hkv, Hq // Hkv, d).sum(dim=(0, 2)).contiguous()
+                 for x in self.inputs]
+        ws_q = torch.zeros(pk.page_topk_qsum_workspace_size(Hkv, (w.num_chunks - 1) * ppc),
+                           dtype=torch.uint8, device=self.dev)
 
-        def one_pass():
+        def from_q(st):
             for c in range(1, w.num_chunks):
                 n_past = c * ppc
                 pk.page_topk(self.pool, self.inputs[c]["q"], self.page_table_dev[:n_past], n_past,
                              w.top_k, w.n_recent, self.sel_l[c], self.sel_p[c], self.sel_n[c],
-                             self.ws, stream=stream)
-        for _ in range(2):
-            one_pass()
-        torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            one_pass()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / reps
+                             self.ws, stream=st)
+
+        def from_qsum(st):
+            for c in range(1, w.num_chunks):
+                n_past = c * ppc
+                pk.page_topk_qsum(self.pool, qsums[c], C, Hq, self.page_table_dev[:n_past],
+                                  n_past, w.top_k, w.n_recent, self.sel_l[c], self.sel_p[c],
+                                  self.sel_n[c], ws_q, stream=st)
+
+        def graph_ms(one_pass):
+            s = torch.cuda.Stream(device=self.dev)
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                one_pass(s)
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                one_pass(torch.cuda.current_stream())
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            del g
+            return a.elapsed_time(b) / reps
+
+        return graph_ms(from_q), graph_ms(from_qsum)
 
     def close(self):
         self.pk.pool_destroy(self.pool)
@@ -1067,7 +1132,9 @@ def main():
             n_past = c * ws.pages_per_chunk
             topk_bytes += C * Hq * d * 2 + n_past * (Hkv * d * 4 + 4) + Hkv * (ws.top_k + ws.n_recent) * 8
         topk_in_step_ms = kt_s.get("topk", 0.0)
-        topk_ms = sp.time_topk_alone()
+        topk_ms, topk_qsum_ms = sp.time_topk_alone()
+        n_sel = ws.num_chunks - 1
+        topk_qsum_bytes = topk_bytes - n_sel * C * Hq * d * 2
         sparse_obj = {"workload": ws.name, "value": sp.step_flops * world / (ms_s / 1e3) / 1e12,
                       "gpu_launches": sp.launches_per_step * a.steps,
                       "unit": "TFLOP/s", "ms_per_step": ms_s,
@@ -1079,10 +1146,23 @@ def main():
                                    "frac": (topk_bytes / (topk_ms / 1e3) / 1e9) / peaks["hbm_gbs"]
                                    if topk_ms else None,
                                    "ms_per_step_alone": topk_ms,
+                                   "us_per_chunk_alone": topk_ms * 1e3 / n_sel,
                                    "ms_per_step_in_step": topk_in_step_ms,
-                                   "note": "all chunks' selections timed back to back, alone "
-                                   "(query mean, page scores, radix select per chunk); in the "
-                                   "step its launches wait for SMs the dQ stream holds"},
+                                   "from_qsum": {
+                                       "ms_per_step_alone": topk_qsum_ms,
+                                       "us_per_chunk_alone": topk_qsum_ms * 1e3 / n_sel,
+                                       "achieved": topk_qsum_bytes / (topk_qsum_ms / 1e3) / 1e9,
+                                       "frac": topk_qsum_bytes / (topk_qsum_ms / 1e3) / 1e9
+                                       / peaks["hbm_gbs"],
+                                       "note": "one launch per chunk (scores + select) from "
+                                       "per-group Q sums such as the projection's epilogue "
+                                       "writes; reads the page summaries only"},
+                                   "note": "all chunks' selections timed back to back, alone, "
+                                   "replayed from a CUDA graph (query mean, page scores, radix "
+                                   "select per chunk); in the "
+                                   "step chunk c+1's selection runs on its own stream beside "
+                                   "chunk c's attention, and ms_per_step_in_step is its event "
+                                   "time there (overlapped, off the critical path)"},
                       "device_status": sparse_status}
         sp.close()
         del sp

@@ -269,6 +269,34 @@ oomb_status oomb_qpage_lists(oomb_pool* pool, const int32_t* d_sel_logical,
                              uint8_t* d_out_masks, int32_t* d_out_count, int32_t max_union,
                              void* stream);
 
+/* oomb_page_topk from per-group sums of Q instead of Q: the query mean is
+ * left to the kernel that produces Q (oomb_qkv_project's d_qsum, written by
+ * its GEMM epilogue), so the selection is one launch that reads only the
+ * page summaries ([pt] §2D: the pages a chunk needs are known once its
+ * queries exist).
+ *   d_qsum           device fp32 [num_kv_heads][head_dim]: per group g the
+ *                    sum of Q over the chunk's chunk_len rows and the G =
+ *                    num_q_heads / num_kv_heads heads of g; q_bar_g =
+ *                    d_qsum[g] / (chunk_len G)
+ *   d_workspace      device memory of oomb_page_topk_qsum_workspace_size()
+ *                    bytes, 16-byte aligned.  Its first num_kv_heads words
+ *                    are counters that must be zero before the first call on
+ *                    a workspace (e.g. cudaMemsetAsync once); every completed
+ *                    call leaves them at zero, so later calls need no clear.
+ *                    Calls sharing a workspace must be ordered (one stream).
+ * Everything else (outputs, limits, tie rule, pool locations) as
+ * oomb_page_topk.  Scores use the fp32 q_bar of the given sums, so where
+ * those sums differ in rounding from oomb_page_topk's own query mean (a
+ * different summation order) pages whose scores tie within that rounding
+ * may be exchanged. */
+size_t oomb_page_topk_qsum_workspace_size(int32_t num_kv_heads, int32_t n_past);
+oomb_status oomb_page_topk_qsum(const oomb_pool* pool, const float* d_qsum, int32_t chunk_len,
+                                int32_t num_q_heads, const int32_t* d_page_table, int32_t n_past,
+                                int32_t top_k, int32_t n_recent, int32_t* d_out_logical,
+                                int32_t* d_out_physical, int32_t* d_out_count,
+                                float* d_out_scores, void* d_workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* Allocation-free variant of oomb_page_topk (this one has no counterpart in
  * the paper; it exists for callers that cannot allocate device memory, e.g.
  * code running under a host framework that owns every device allocation, or a
@@ -296,7 +324,7 @@ oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* d_q, int32_
                                   int32_t* d_out_count, float* d_out_scores, void* stream);
 
 /* Batched Top-K: n_problems independent selections in one set of launches
- * (three kernels for the whole batch).  Problem b takes the query rows
+ * (two kernels for the whole batch).  Problem b takes the query rows
  * [d_row_start[b], d_row_start[b+1]) of d_q ([num_rows][num_q_heads][d]
  * bf16) and the candidates among logical pages [0, d_n_past[b]) of the one
  * page table d_page_table (length >= max_past); each problem is exactly one

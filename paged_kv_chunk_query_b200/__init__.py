@@ -13,7 +13,7 @@ from ._lib import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, LOC_DEVICE, LOC_HOST, LOC_P
                    OombError, block_copy, chunk_attn_bwd, chunk_attn_fwd, get_device_status,
                    grad_block_add, grad_writeback, grad_writeback_sync, kv_append, local_pages, page_prefetch,
                    page_topk, page_topk_batched, page_topk_batched_workspace_size,
-                   page_topk_workspace_size, pool_alloc_page, pool_buffers, pool_create,
+                   page_topk_qsum, page_topk_qsum_workspace_size, page_topk_workspace_size, pool_alloc_page, pool_buffers, pool_create,
                    pool_destroy, pool_free_page, pool_get_desc, pool_num_free, pool_views,
                    prefetch_lists, qkv_project, qpage_lists, status_string, version, wait)
 from .synth import WORKLOADS, Workload
@@ -27,6 +27,6 @@ __all__ = [
     "get_device_status", "status_string", "version",
     "LOC_DEVICE", "LOC_PINNED_HOST", "LOC_HOST", "BWD_PREPROCESS", "BWD_DKDV", "BWD_DQ",
     "SEG_WHOLE", "SEG_FIRST", "SEG_NEXT", "SEG_LAST", "PROJ_Q", "PROJ_KV", "PROJ_QKV",
-    "qkv_project", "qpage_lists",
+    "qkv_project", "qpage_lists", "page_topk_qsum", "page_topk_qsum_workspace_size",
     "WORKLOADS", "Workload",
 ]

@@ -40,6 +40,7 @@ EXPORTS = (
     "oomb_selftest_wait_limit", "oomb_page_topk_batched_workspace_size", "oomb_page_topk_batched",
     "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists", "oomb_local_pages",
     "oomb_qkv_project", "oomb_selftest_writeback_copy", "oomb_qpage_lists",
+    "oomb_page_topk_qsum_workspace_size", "oomb_page_topk_qsum",
 )
 
 
@@ -95,6 +96,8 @@ def load() -> ctypes.CDLL:
         "oomb_page_topk": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp,
                            ctypes.c_size_t, vp],
         "oomb_page_topk_static": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp],
+        "oomb_page_topk_qsum": [vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp,
+                                ctypes.c_size_t, vp],
         "oomb_page_prefetch": [vp, vp, vp, vp, i32, vp, vp],
         "oomb_grad_writeback": [vp, vp, vp, vp, i32, vp],
         "oomb_grad_writeback_sync": [vp, ctypes.c_int64],
@@ -120,6 +123,9 @@ def load() -> ctypes.CDLL:
     if hasattr(lib, "oomb_page_topk_workspace_size"):
         lib.oomb_page_topk_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         lib.oomb_page_topk_workspace_size.restype = ctypes.c_size_t
+    if hasattr(lib, "oomb_page_topk_qsum_workspace_size"):
+        lib.oomb_page_topk_qsum_workspace_size.argtypes = [i32, i32]
+        lib.oomb_page_topk_qsum_workspace_size.restype = ctypes.c_size_t
     if hasattr(lib, "oomb_page_topk_batched_workspace_size"):
         lib.oomb_page_topk_batched_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.oomb_page_topk_batched_workspace_size.restype = ctypes.c_size_t
@@ -332,6 +338,26 @@ def page_topk(pool, q, page_table, n_past, top_k, n_recent, out_logical, out_phy
         _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
         _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "oomb_page_topk")
+
+
+def page_topk_qsum_workspace_size(num_kv_heads, n_past) -> int:
+    return load().oomb_page_topk_qsum_workspace_size(num_kv_heads, n_past)
+
+
+def page_topk_qsum(pool, qsum, chunk_len, num_q_heads, page_table, n_past, top_k, n_recent,
+                   out_logical, out_physical, out_count, workspace, out_scores=None, stream=None):
+    """oomb_page_topk_qsum: the selection from per-group sums of Q ([Hkv][d]
+    fp32, e.g. qkv_project's qsum).  The workspace's counters must be zero
+    before its first use (torch.zeros); each call leaves them at zero."""
+    _check(load().oomb_page_topk_qsum(
+        pool, _dev_tensor(qsum, torch.float32, "qsum"), chunk_len, num_q_heads,
+        _dev_tensor(page_table, torch.int32, "page_table") if n_past else None, n_past, top_k,
+        n_recent, _dev_tensor(out_logical, torch.int32, "out_logical"),
+        _dev_tensor(out_physical, torch.int32, "out_physical") if out_physical is not None
+        else None, _dev_tensor(out_count, torch.int32, "out_count"),
+        _dev_tensor(out_scores, torch.float32, "out_scores") if out_scores is not None else None,
+        _dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "oomb_page_topk_qsum")
 
 
 def page_topk_batched_workspace_size(n_problems, num_kv_heads, head_dim, max_past) -> int:

@@ -10,13 +10,14 @@
 // ties going to the lower logical id; pages [n_past - R, n_past) are always
 // kept; the output lists ascending logical ids.
 //
-// The kernels take a batch of independent problems (blockIdx.z / .y), each a
+// The kernels take a batch of independent problems (blockIdx.z), each a
 // range of query rows and its own number of past pages; the per-chunk entry
 // points run a batch of one.  Two launches:
-// Kernel 1 (qmean_partial): grid (slices, problems); each CTA streams whole
-//   token rows (all heads, contiguous) of a slice of its problem's rows, one
-//   thread per 16-byte column, and writes one fp32 partial per (group, d).
-//   It also zeroes the tickets kernel 2 counts on.
+// Kernel 1 (qmean_partial): grid (slices, Hkv, problems); each CTA streams the
+//   G heads of one group (contiguous in a token row) over a slice of its
+//   problem's rows, one thread per 16-byte column, 16 rows in flight, and
+//   writes one fp32 partial per d.  It also zeroes the tickets kernel 2
+//   counts on.
 // Kernel 2 (page_score_select): grid (pages / 64, Hkv, problems).  Each CTA
 //   sums the slice partials of its (problem, group) in one fixed order into
 //   q_bar (every CTA of a group gets the identical q_bar), then each warp
@@ -25,7 +26,9 @@
 //   waits) finds the K-th largest 64-bit key (ordered score, inverted id) by
 //   8-bit radix passes from the top with a parallel bin scan, stopping once
 //   the boundary bin is kept whole, and compacts the kept ids in ascending
-//   order.
+//   order.  Up to 4,096 past pages the keys stay in registers (16 contiguous
+//   pages per thread, warp-aggregated histogram updates, one scan for the
+//   compaction); beyond that they are re-read from L2 on every pass.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -37,9 +40,26 @@
 namespace {
 
 constexpr int kSplits = 128;         // max query-mean slices per (problem, group)
-constexpr int kMeanThreadsMax = 1024;  // query mean: one thread per 16-byte column of a token
+constexpr int kMeanThreads = 256;    // query mean: one thread per 16-byte column of a group's heads
 constexpr int kScoreThreads = 256;   // 8 warps x 8 pages per CTA
 constexpr int kPagesPerScoreCta = 64;
+constexpr int kKeysPerThread = 16;   // register-resident select: up to 4,096 past pages
+
+// Programmatic dependent launch (sm_90+): the query-mean kernel lets the
+// scores kernel launch once all of its CTAs have started; the scores kernel
+// does the work that does not read the query mean's output, then waits for
+// that grid to complete and its writes to be visible.  Without a dependent
+// launch the wait returns at once.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Row stride of the 64-bit key array: even, so that every row starts on a
+// 16-byte boundary and key pairs load as one vector.
+__host__ __device__ __forceinline__ int key_stride(int max_past) {
+  return ((max_past > 0 ? max_past : 1) + 1) & ~1;
+}
 
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -89,28 +109,32 @@ __device__ __forceinline__ int problem_npast(const Problems& pb, int b) {
 }
 
 // ---------------------------------------------------------------- query mean
-// grid (splits, problems): CTA (s, b) streams slice s of problem b's tokens,
-// whole token rows (every head: Hq * d * 2 contiguous bytes), one thread per
-// 16-byte column, 4 rows in flight per thread; then sums the G heads of each
-// group in shared memory (fixed order) and writes one fp32 partial per
-// (group, d).  Reading whole rows keeps every DRAM page opened once.
+// grid (splits, Hkv, problems): CTA (s, g, b) streams slice s of problem b's
+// tokens, the G heads of group g (G * d * 2 contiguous bytes of each token
+// row), one thread per 16-byte column, 16 rows in flight per thread; then sums
+// the G heads in shared memory (fixed order) and writes one fp32 partial per
+// d.  Each partial is the same sum, in the same order, for any grid shape:
+// rows in slice order per column, then heads in order.
 template <int D>
-__global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
+__global__ void __launch_bounds__(kMeanThreads, 1) qmean_partial_kernel(
     const __nv_bfloat16* __restrict__ q, float* __restrict__ partial, const Problems pb, int Hq,
     int G, unsigned int* __restrict__ tickets, int n_tickets) {
-  extern __shared__ float col_sum[];  // [Hq][D]
+  extern __shared__ float col_sum[];  // [G][D]
   constexpr int VPR = D / 8;          // 16-byte vectors per (token, head) row
-  constexpr int U = 8;                // rows in flight per thread
-  const int split = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  constexpr int U = 16;               // rows in flight per thread
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
+  const int Hkv = gridDim.y;
+  pdl_launch_dependents();
   // the next kernel on the stream counts finished CTAs from zero
-  if (split == 0 && b == 0)
+  if (split == 0 && g == 0 && b == 0)
     for (int i = t; i < n_tickets; i += blockDim.x) tickets[i] = 0u;
-  const int ncol = Hq * VPR;          // 16-byte vectors per token
+  const int ncol = G * VPR;           // 16-byte vectors of the group's heads in a token row
+  const size_t row_vecs = static_cast<size_t>(Hq) * VPR;
   int r0, r1;
   problem_rows(pb, b, r0, r1);
   const int per = (r1 - r0 + pb.splits - 1) / pb.splits;
   const int tok0 = r0 + split * per, tok1 = min(r1, tok0 + per);
-  const uint4* base = reinterpret_cast<const uint4*>(q);
+  const uint4* base = reinterpret_cast<const uint4*>(q) + static_cast<size_t>(g) * ncol;
   for (int col = t; col < ncol; col += blockDim.x) {
     float acc[8];
 #pragma unroll
@@ -119,7 +143,7 @@ __global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
     for (; tok + U <= tok1; tok += U) {
       uint4 v[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) v[u] = __ldg(base + static_cast<size_t>(tok + u) * ncol + col);
+      for (int u = 0; u < U; ++u) v[u] = __ldg(base + (tok + u) * row_vecs + col);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
@@ -128,20 +152,18 @@ __global__ void __launch_bounds__(kMeanThreadsMax, 1) qmean_partial_kernel(
       }
     }
     for (; tok < tok1; ++tok) {
-      const uint4 v = __ldg(base + static_cast<size_t>(tok) * ncol + col);
+      const uint4 v = __ldg(base + tok * row_vecs + col);
       const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(bv[e]);
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) col_sum[col * 8 + e] = acc[e];  // (head, d) = col * 8 + e
+    for (int e = 0; e < 8; ++e) col_sum[col * 8 + e] = acc[e];  // (head in group, d) = col * 8 + e
   }
   __syncthreads();
-  const int Hkv = Hq / G;
-  for (int i = t; i < Hkv * D; i += blockDim.x) {
-    const int g = i / D, dd = i % D;
+  for (int dd = t; dd < D; dd += blockDim.x) {
     float s = 0.f;
-    for (int hh = 0; hh < G; ++hh) s += col_sum[(g * G + hh) * D + dd];  // fixed order
+    for (int hh = 0; hh < G; ++hh) s += col_sum[hh * D + dd];  // fixed order
     partial[((static_cast<size_t>(b) * pb.splits + split) * Hkv + g) * D + dd] = s;
   }
 }
@@ -153,20 +175,65 @@ __device__ __forceinline__ uint32_t order_f32(float f) {
 }
 
 // ---------------------------------------------------------------- select
+// Shared state of one CTA's radix select (256 bins, 8 warps of bin scan).
+struct RadixShared {
+  unsigned int hist[256];
+  unsigned int warp_tot[8];
+  int warp_cnt[32];
+  unsigned long long kth;
+  int need, done;
+};
+
+// One radix step's bin search, once hist[] holds the counts, by the 8-bit
+// digit at `shift`, of the keys still in play (those equal to the K-th key's
+// prefix found so far): the bin, scanned from 255 down, that holds the
+// need-th largest of them.  Sets kth (prefix plus that digit), need (the rank
+// left inside the bin) and done (the bin is kept whole, so the lower digits
+// do not matter).  Thread t < 256 owns bin 255 - t.  Ends on a barrier.
+__device__ __forceinline__ void radix_pick_bin(RadixShared& sh, unsigned long long prefix,
+                                               int shift) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  // every thread reads the remaining count here, before the barrier that
+  // precedes its one update below (a read after the update could let a
+  // second bin match)
+  const int need = sh.need;
+  // inclusive suffix sum over bins 255..0
+  unsigned int incl = 0;
+  if (t < 256) {
+    incl = sh.hist[255 - t];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) sh.warp_tot[warp] = incl;
+  }
+  __syncthreads();
+  if (t < 256) {
+    for (int w = 0; w < warp; ++w) incl += sh.warp_tot[w];
+    const int bin = 255 - t;
+    const unsigned int v = sh.hist[bin];
+    const unsigned int excl = incl - v;
+    if (excl < static_cast<unsigned>(need) && static_cast<unsigned>(need) <= incl) {
+      sh.kth = prefix | (static_cast<unsigned long long>(bin) << shift);
+      sh.need = need - static_cast<int>(excl);
+      if (v == static_cast<unsigned>(need) - excl) sh.done = 1;  // bin taken whole
+    }
+  }
+  __syncthreads();
+}
+
 // The K-th largest candidate key of one (problem, group) by 8-bit radix passes
-// from the top, each with a parallel suffix scan over the 256 bins; stops
-// early once the boundary bin is taken whole.  Then compacts the kept ids in
-// ascending order.  Run by one CTA of NT threads (NT >= 256).
+// from the top, stopping early once the boundary bin is taken whole; then the
+// kept ids compacted in ascending order.  Keys are read from L2 on every pass
+// (coherent loads: other CTAs of this launch wrote them).  Any n_past.  Run
+// by one CTA of NT threads (NT >= 256).
 template <int NT>
-__device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
+__device__ void select_pages_cta(const unsigned long long* keys,
                                  const int32_t* __restrict__ page_table, int n_past, int top_k,
                                  int n_recent, int num_pool_pages, int32_t* __restrict__ out_l,
                                  int32_t* __restrict__ out_p, int32_t* __restrict__ out_count) {
-  __shared__ unsigned int hist[256];
-  __shared__ unsigned int warp_tot[8];
-  __shared__ unsigned long long kth_sh;
-  __shared__ int need_sh, done_sh;
-  __shared__ int warp_sum[NT / 32];
+  __shared__ RadixShared sh;
   __shared__ int running_sh;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int max_sel = top_k + n_recent;
@@ -174,15 +241,15 @@ __device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
   const int k_eff = min(top_k, n_cand);
 
   if (t == 0) {
-    kth_sh = 0ull;  // with k_eff >= n_cand every candidate is kept
-    need_sh = k_eff;
-    done_sh = 0;
+    sh.kth = 0ull;  // with k_eff >= n_cand every candidate is kept
+    sh.need = k_eff;
+    sh.done = 0;
   }
   __syncthreads();
   if (k_eff > 0 && k_eff < n_cand) {
     unsigned long long prefix = 0ull, mask = 0ull;
     for (int shift = 56; shift >= 0; shift -= 8) {
-      if (t < 256) hist[t] = 0u;
+      if (t < 256) sh.hist[t] = 0u;
       __syncthreads();
       // eight keys per thread in flight before their histogram updates
       for (int base = 0; base < n_cand; base += 8 * NT) {
@@ -190,64 +257,36 @@ __device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int p = base + u * NT + t;
-          kv[u] = p < n_cand ? keys[p] : 0ull;
+          kv[u] = p < n_cand ? __ldcg(keys + p) : 0ull;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int p = base + u * NT + t;
           if (p < n_cand && (kv[u] & mask) == prefix)
-            atomicAdd(&hist[(kv[u] >> shift) & 255ull], 1u);
+            atomicAdd(&sh.hist[(kv[u] >> shift) & 255ull], 1u);
         }
       }
       __syncthreads();
-      // every thread reads the remaining count here, before the barrier that
-      // precedes its one update below (a read after the update could let a
-      // second bin match)
-      const int need = need_sh;
-      // inclusive suffix sum over bins 255..0: thread t < 256 owns bin 255 - t
-      unsigned int incl = 0;
-      if (t < 256) {
-        const unsigned int v = hist[255 - t];
-        incl = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += y;
-        }
-        if (lane == 31) warp_tot[warp] = incl;
-      }
-      __syncthreads();
-      if (t < 256) {
-        for (int w = 0; w < warp; ++w) incl += warp_tot[w];
-        const int bin = 255 - t;
-        const unsigned int v = hist[bin];
-        const unsigned int excl = incl - v;
-        if (excl < static_cast<unsigned>(need) && static_cast<unsigned>(need) <= incl) {
-          kth_sh = prefix | (static_cast<unsigned long long>(bin) << shift);
-          need_sh = need - static_cast<int>(excl);
-          if (v == static_cast<unsigned>(need) - excl) done_sh = 1;  // bin taken whole
-        }
-      }
-      __syncthreads();
-      prefix = kth_sh;
+      radix_pick_bin(sh, prefix, shift);
+      prefix = sh.kth;
       mask |= 255ull << shift;
-      if (done_sh) break;
+      if (sh.done) break;
     }
   }
-  const unsigned long long kth = kth_sh;
+  const unsigned long long kth = sh.kth;
 
   if (t == 0) running_sh = 0;
   __syncthreads();
   for (int base = 0; base < n_past; base += NT) {
     const int p = base + t;
     int keep = 0;
-    if (p < n_cand) keep = (k_eff >= n_cand) || (k_eff > 0 && keys[p] >= kth);
+    if (p < n_cand) keep = (k_eff >= n_cand) || (k_eff > 0 && __ldcg(keys + p) >= kth);
     else if (p < n_past) keep = 1;
     const unsigned ballot = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) warp_sum[warp] = __popc(ballot);
+    if (lane == 0) sh.warp_cnt[warp] = __popc(ballot);
     __syncthreads();
     int before = running_sh;
-    for (int w = 0; w < warp; ++w) before += warp_sum[w];
+    for (int w = 0; w < warp; ++w) before += sh.warp_cnt[w];
     before += __popc(ballot & ((1u << lane) - 1u));
     if (keep && before < max_sel) {
       out_l[before] = p;
@@ -259,7 +298,7 @@ __device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
     __syncthreads();
     if (t == 0) {
       int tot = 0;
-      for (int w = 0; w < NT / 32; ++w) tot += warp_sum[w];
+      for (int w = 0; w < NT / 32; ++w) tot += sh.warp_cnt[w];
       running_sh += tot;
     }
     __syncthreads();
@@ -267,22 +306,225 @@ __device__ void select_pages_cta(const unsigned long long* __restrict__ keys,
   if (t == 0) *out_count = min(running_sh, max_sel);
 }
 
+// Score of a key: the inverse of order_f32 on its upper 32 bits.
+__device__ __forceinline__ float key_score(unsigned long long k) {
+  const uint32_t u = static_cast<uint32_t>(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+// Bucket of a score on a linear scale from smin (bucket 0) over 256 buckets.
+// Non-decreasing in s: a key in a higher bucket has a strictly higher score.
+__device__ __forceinline__ int score_bucket(float s, float smin, float scale) {
+  const float x = (s - smin) * scale;
+  return x >= 255.f ? 255 : (x > 0.f ? static_cast<int>(x) : 0);
+}
+
+// The same selection with the keys held in registers, for n_past <= NT * KPT:
+// thread t owns logical pages [t * KPT, (t + 1) * KPT), loaded once together
+// with their physical ids (key rows start 16-byte aligned, so pairs load as
+// one vector).  The first digit is not a byte of the key (whose top bytes,
+// sign and exponent, most scores share, so that nearly every key would land
+// in one or two bins) but a bucket of the score on a linear scale between
+// the candidates' minimum and maximum: the bucket holding the K-th largest
+// key is found from its histogram; the keys above it are kept, and only the
+// keys inside it go through exact radix passes over the 64-bit key, starting
+// at the highest bit in which they differ.  The kept ids come out ascending
+// from one CTA-wide scan of the per-thread counts.
+template <int NT, int KPT>
+__device__ void select_pages_regs(const unsigned long long* keys,
+                                  const int32_t* __restrict__ page_table, int n_past, int top_k,
+                                  int n_recent, int num_pool_pages, int32_t* __restrict__ out_l,
+                                  int32_t* __restrict__ out_p, int32_t* __restrict__ out_count) {
+  static_assert(NT == 256 && KPT % 2 == 0 && KPT <= 32, "select layout");
+  constexpr int NW = NT / 32;
+  __shared__ RadixShared sh;
+  __shared__ float wmin[NW], wmax[NW];
+  __shared__ unsigned long long wlo[NW], whi[NW];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int max_sel = top_k + n_recent;
+  const int n_cand = max(0, n_past - n_recent);
+  const int k_eff = min(top_k, n_cand);
+  const int p0 = t * KPT;
+
+  unsigned long long kv[KPT];
+  int phys[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) phys[j] = p0 + j < n_past && out_p ? page_table[p0 + j] : 0;
+#pragma unroll
+  for (int j = 0; j < KPT; j += 2) {
+    if (p0 + j + 1 < n_cand) {
+      const ulonglong2 v = __ldcg(reinterpret_cast<const ulonglong2*>(keys + p0 + j));
+      kv[j] = v.x;
+      kv[j + 1] = v.y;
+    } else {
+      kv[j] = p0 + j < n_cand ? __ldcg(keys + p0 + j) : 0ull;
+      kv[j + 1] = 0ull;
+    }
+  }
+  const bool keep_all = k_eff >= n_cand;
+  const bool run = k_eff > 0 && !keep_all;  // uniform over the CTA
+  unsigned int above_bits = 0u, member_bits = 0u;
+  bool bucket_whole = false;
+  unsigned long long kth = 0ull;
+  if (run) {
+    // score range of the candidates
+    float lo = __int_as_float(0x7f800000), hi = -lo;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (p0 + j < n_cand) {
+        const float sc = key_score(kv[j]);
+        lo = fminf(lo, sc);
+        hi = fmaxf(hi, sc);
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+      wmin[warp] = lo;
+      wmax[warp] = hi;
+    }
+    if (t == 0) {
+      sh.need = k_eff;
+      sh.done = 0;
+    }
+    sh.hist[t] = 0u;
+    __syncthreads();
+    float smin = wmin[0], smax = wmax[0];
+    for (int w = 1; w < NW; ++w) {
+      smin = fminf(smin, wmin[w]);
+      smax = fmaxf(smax, wmax[w]);
+    }
+    const float range = smax - smin;
+    const float scale = range > 0.f && range < __int_as_float(0x7f800000) ? 256.f / range : 0.f;
+    // histogram of the score buckets, then the bucket of the K-th largest key
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (p0 + j < n_cand) atomicAdd(&sh.hist[score_bucket(key_score(kv[j]), smin, scale)], 1u);
+    __syncthreads();
+    radix_pick_bin(sh, 0ull, 0);
+    const int B = static_cast<int>(sh.kth);
+    bucket_whole = sh.done != 0;
+    unsigned long long klo = ~0ull, khi = 0ull;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (p0 + j < n_cand) {
+        const int bj = score_bucket(key_score(kv[j]), smin, scale);
+        above_bits |= static_cast<unsigned int>(bj > B) << j;
+        if (bj == B) {
+          member_bits |= 1u << j;
+          klo = min(klo, kv[j]);
+          khi = max(khi, kv[j]);
+        }
+      }
+    if (!bucket_whole) {
+      // exact K-th key among the boundary bucket's keys (at least two of
+      // them, all distinct): 8-bit digits from the highest differing bit
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        klo = min(klo, __shfl_xor_sync(0xffffffffu, klo, off));
+        khi = max(khi, __shfl_xor_sync(0xffffffffu, khi, off));
+      }
+      if (lane == 0) {
+        wlo[warp] = klo;
+        whi[warp] = khi;
+      }
+      __syncthreads();
+      klo = wlo[0];
+      khi = whi[0];
+      for (int w = 1; w < NW; ++w) {
+        klo = min(klo, wlo[w]);
+        khi = max(khi, whi[w]);
+      }
+      const int top = 63 - __clzll(static_cast<long long>(klo ^ khi));
+      unsigned long long mask = ~((2ull << top) - 1ull);  // the bits above `top`, common
+      unsigned long long prefix = klo & mask;
+      for (int s = top - 7; s > -8; s -= 8) {
+        const int shift = s > 0 ? s : 0;
+        const unsigned long long dmask = (1ull << (s >= 0 ? 8 : 8 + s)) - 1ull;
+        sh.hist[t] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+          if (((member_bits >> j) & 1u) && (kv[j] & mask) == prefix)
+            atomicAdd(&sh.hist[(kv[j] >> shift) & dmask], 1u);
+        __syncthreads();
+        radix_pick_bin(sh, prefix, shift);
+        prefix = sh.kth;
+        mask |= dmask << shift;
+        if (sh.done) break;
+      }
+      kth = sh.kth;
+    }
+  }
+
+  unsigned int keep_bits = 0u;
+  int cnt = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int p = p0 + j;
+    bool keep;
+    if (p < n_cand) {
+      const bool member = (member_bits >> j) & 1u;
+      keep = keep_all || ((above_bits >> j) & 1u) || (member && (bucket_whole || kv[j] >= kth));
+    } else {
+      keep = p < n_past;
+    }
+    keep_bits |= static_cast<unsigned int>(keep) << j;
+    cnt += keep;
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) sh.warp_cnt[warp] = incl;
+  __syncthreads();
+  int before = incl - cnt, total = 0;
+  for (int w = 0; w < NW; ++w) {
+    const int c = sh.warp_cnt[w];
+    if (w < warp) before += c;
+    total += c;
+  }
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if ((keep_bits >> j) & 1u) {
+      if (before < max_sel) {
+        out_l[before] = p0 + j;
+        if (out_p) out_p[before] = (phys[j] >= 0 && phys[j] < num_pool_pages) ? phys[j] : 0;
+      }
+      ++before;
+    }
+  }
+  if (t == 0) *out_count = min(total, max_sel);
+}
+
 // ---------------------------------------------------------------- scores + select
 // grid (max(1, ceil(max_past / 64)), Hkv, problems), kScoreThreads threads.
-// q_bar: thread t sums splits [64 (t / D), ...) of column t % D in a fixed order
-// (eight chains, sixteen loads in flight), the two halves are added in a
-// fixed order and divided by rows * G.  Key = (ordered score << 32) |
-// (~logical id), stored at [problem][group][max_past].  The CTA whose ticket
-// is the last of its (problem, group) then runs the select.
-template <int D>
+// Each warp first loads the summaries of its 8 pages (they do not depend on
+// q_bar, so these loads overlap its reduction).  q_bar, FROM_QSUM false:
+// thread t sums splits [64 (t / D), ...) of column t % D of the query-mean
+// partials in a fixed order (eight chains, sixteen loads in flight), the two
+// halves are added in a fixed order and divided by rows * G.  FROM_QSUM true:
+// q_bar = qsum[problem][group] / (rows * G), qsum being the group's sum of Q
+// over the rows and G heads made elsewhere (the projection's epilogue).
+// Key = (ordered score << 32) | (~logical id), stored at
+// [problem][group][key_stride(max_past)].  The CTA whose ticket is the last
+// of its (problem, group) then runs the select and sets the ticket back to
+// zero, so a completed call leaves every ticket at zero.
+template <int D, bool FROM_QSUM>
 __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
-    const float* __restrict__ partial, const float* __restrict__ summary,
-    const int32_t* __restrict__ page_table, const Problems pb, int G, int Hkv,
-    int num_pool_pages, unsigned long long* __restrict__ keys, float* __restrict__ out_scores,
-    unsigned int* __restrict__ tickets, int top_k, int n_recent,
+    const float* __restrict__ partial, const float* __restrict__ qsum,
+    const float* __restrict__ summary, const int32_t* __restrict__ page_table, const Problems pb,
+    int G, int Hkv, int num_pool_pages, unsigned long long* __restrict__ keys,
+    float* __restrict__ out_scores, unsigned int* __restrict__ tickets, int top_k, int n_recent,
     int32_t* __restrict__ out_logical, int32_t* __restrict__ out_physical,
     int32_t* __restrict__ out_count) {
   static_assert(kScoreThreads == 2 * 128 && D <= 128, "q_bar reduction layout");
+  constexpr int PW = kPagesPerScoreCta / (kScoreThreads / 32);  // pages per warp
+  constexpr int EPL = D / 32;                                   // elements per lane
   __shared__ float qs[2][D];
   __shared__ int last_sh;
   const int g = blockIdx.y, b = blockIdx.z, t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -290,8 +532,41 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
   const int n_ctas = max(1, (n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta);
   if (static_cast<int>(blockIdx.x) >= n_ctas) return;  // beyond this problem's pages
 
-  // q_bar of (problem b, group g) from the query-mean partials
+  // this warp's page summaries (EPL fp32 per lane and page)
+  const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
+  float sv[PW][EPL];
   {
+    int phys[PW];
+#pragma unroll
+    for (int i = 0; i < PW; ++i) phys[i] = p0 + i < n_past ? __ldg(page_table + p0 + i) : 0;
+#pragma unroll
+    for (int i = 0; i < PW; ++i) {
+      if (phys[i] < 0 || phys[i] >= num_pool_pages) {
+        if (lane == 0) atomicOr(pb.status, OOMB_DEV_BAD_PAGE);
+        phys[i] = 0;
+      }
+      const float* srow = summary + (static_cast<size_t>(phys[i]) * Hkv + g) * D + lane * EPL;
+      if (EPL == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(srow));
+        sv[i][0] = v.x;
+        sv[i][1] = v.y;
+        sv[i][2] = v.z;
+        sv[i][3] = v.w;
+      } else {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(srow));
+        sv[i][0] = v.x;
+        sv[i][1] = v.y;
+      }
+    }
+  }
+
+  // the query-mean partials and the tickets it zeroed are read from here on
+  pdl_wait();
+  // q_bar of (problem b, group g)
+  if (FROM_QSUM) {
+    if (t < D) qs[0][t] = __ldg(qsum + (static_cast<size_t>(b) * Hkv + g) * D + t);
+    else if (t >= 128 && t - 128 < D) qs[1][t - 128] = 0.f;
+  } else {
     const int dd = t % 128, half = t / 128;
     if (dd < D) {
       const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D + g * D + dd;
@@ -307,7 +582,14 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
 #pragma unroll
         for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
       }
-      for (; i < hi; ++i) s8[i & 7] += __ldg(pp + static_cast<size_t>(i) * Hkv * D);
+      if (i < hi) {  // the tail, as one more block of 16 with zeros past hi (x + 0 = x)
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          v[e] = i + e < hi ? __ldg(pp + static_cast<size_t>(i + e) * Hkv * D) : 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
+      }
       qs[half][dd] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
     }
   }
@@ -316,34 +598,22 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
   problem_rows(pb, b, r0, r1);
   const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
   const size_t row = (static_cast<size_t>(b) * Hkv + g);
-  constexpr int PW = kPagesPerScoreCta / (kScoreThreads / 32);  // pages per warp
-  constexpr int EPL = D / 32;                                   // elements per lane
+  unsigned long long* key_row = keys + row * key_stride(pb.max_past);
   float qv[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
     const int dd = lane * EPL + e;
     qv[e] = rows > 0.f ? (qs[0][dd] + qs[1][dd]) / rows : 0.f;
   }
-  const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
   float acc[PW];
 #pragma unroll
   for (int i = 0; i < PW; ++i) {
-    const int p = p0 + i;
     acc[i] = 0.f;
-    if (p < n_past) {
-      int phys = __ldg(page_table + p);
-      if (phys < 0 || phys >= num_pool_pages) {
-        if (lane == 0) atomicOr(pb.status, OOMB_DEV_BAD_PAGE);
-        phys = 0;
-      }
-      const float* srow = summary + (static_cast<size_t>(phys) * Hkv + g) * D + lane * EPL;
-      if (EPL == 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(srow));
-        acc[i] = a.x * qv[0] + a.y * qv[1] + a.z * qv[2] + a.w * qv[3];
-      } else {
-        const float2 a = __ldg(reinterpret_cast<const float2*>(srow));
-        acc[i] = a.x * qv[0] + a.y * qv[1];
-      }
+    if (p0 + i < n_past) {
+      if (EPL == 4)
+        acc[i] = sv[i][0] * qv[0] + sv[i][1] * qv[1] + sv[i][2] * qv[2] + sv[i][3] * qv[3];
+      else
+        acc[i] = sv[i][0] * qv[0] + sv[i][1] * qv[1];
     }
   }
 #pragma unroll
@@ -359,7 +629,7 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
     const int p = p0 + lane;
     if (p < n_past) {
       if (out_scores) out_scores[row * pb.max_past + p] = mine;
-      keys[row * pb.max_past + p] =
+      key_row[p] =
           (static_cast<unsigned long long>(order_f32(mine)) << 32) |
           static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
     }
@@ -373,20 +643,74 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
   if (!last_sh) return;
   __threadfence();
   const int max_sel = top_k + n_recent;
-  select_pages_cta<kScoreThreads>(keys + row * pb.max_past, page_table, n_past, top_k, n_recent,
-                                  num_pool_pages, out_logical + row * max_sel,
-                                  out_physical ? out_physical + row * max_sel : nullptr,
-                                  out_count + row);
+  int32_t* out_p = out_physical ? out_physical + row * max_sel : nullptr;
+  if (n_past <= kScoreThreads * kKeysPerThread)
+    select_pages_regs<kScoreThreads, kKeysPerThread>(key_row, page_table, n_past, top_k, n_recent,
+                                                     num_pool_pages, out_logical + row * max_sel,
+                                                     out_p, out_count + row);
+  else
+    select_pages_cta<kScoreThreads>(key_row, page_table, n_past, top_k, n_recent, num_pool_pages,
+                                    out_logical + row * max_sel, out_p, out_count + row);
+  if (t == 0) tickets[row] = 0u;  // every CTA of this (problem, group) has counted
 }
 
 // Workspace: partials [problems][splits <= 128][Hkv][d] fp32, a region of
 // [problems][Hkv][d] fp32 whose first problems * Hkv words are the select
-// tickets, then keys [problems][Hkv][max(max_past, 1)] u64.
+// tickets, then keys [problems][Hkv][key_stride(max_past)] u64.
 size_t workspace_bytes_for(int64_t problems, int Hkv, int D, int max_past) {
   const size_t partial = static_cast<size_t>(problems) * kSplits * Hkv * D * 4;
   const size_t qbar = static_cast<size_t>(problems) * Hkv * D * 4;
-  const size_t keys = static_cast<size_t>(problems) * Hkv * (max_past > 0 ? max_past : 1) * 8;
+  const size_t keys = static_cast<size_t>(problems) * Hkv * key_stride(max_past) * 8;
   return align256(partial) + align256(qbar) + align256(keys);
+}
+
+// Launches the scores + select kernel; q_bar from the query-mean partials
+// (qsum null) or from per-group sums of Q (partial null).
+oomb_status launch_score_select(const oomb_pool* pool, const float* partial, const float* qsum,
+                                const Problems& pb, int n_problems, int G,
+                                const int32_t* d_page_table, int top_k, int n_recent,
+                                int32_t* d_out_logical, int32_t* d_out_physical,
+                                int32_t* d_out_count, float* d_out_scores, unsigned int* tickets,
+                                unsigned long long* keys, cudaStream_t s) {
+  const oomb_pool_desc& d = pool->desc;
+  const int Hkv = d.num_kv_heads;
+  dim3 g2(std::max(1, (pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta), Hkv,
+          n_problems);
+  // after the query-mean kernel: a dependent launch (see pdl_wait); from
+  // sums made by an earlier kernel: an ordinary launch
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = g2;
+  cfg.blockDim = dim3(kScoreThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = qsum ? 0 : 1;
+  const float* summary = pool->summary;
+  const int num_pages = d.num_pages;
+  cudaError_t e;
+#define OOMB_SCORE_ARGS                                                                    \
+  partial, qsum, summary, d_page_table, pb, G, Hkv, num_pages, keys, d_out_scores, tickets, \
+      top_k, n_recent, d_out_logical, d_out_physical, d_out_count
+  if (d.head_dim == 128) {
+    if (qsum)
+      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<128, true>, OOMB_SCORE_ARGS);
+    else
+      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<128, false>, OOMB_SCORE_ARGS);
+  } else {
+    if (qsum)
+      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<64, true>, OOMB_SCORE_ARGS);
+    else
+      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<64, false>, OOMB_SCORE_ARGS);
+  }
+#undef OOMB_SCORE_ARGS
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return OOMB_ERR_CUDA;
+  }
+  return oomb::check_launch();
 }
 
 // Launches the two kernels for `n_problems` problems on `s`.
@@ -408,28 +732,20 @@ oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
       static_cast<uint8_t*>(scratch) + partial_bytes + qbar_bytes);
   const int n_tickets = n_problems * Hkv;
   const auto* q = static_cast<const __nv_bfloat16*>(d_q);
-  // one thread per 16-byte column of a token row, a multiple of 32, at most 1024
-  const int ncol = num_q_heads * D / 8;
-  const int mean_threads = ncol >= kMeanThreadsMax ? kMeanThreadsMax : ((ncol + 31) / 32) * 32;
-  const size_t mean_smem = static_cast<size_t>(num_q_heads) * D * 4;
-  dim3 g1(pb.splits, n_problems);
-  dim3 g2(std::max(1, (pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta), Hkv,
-          n_problems);
+  // one thread per 16-byte column of a group's heads, a multiple of 32, at most 256
+  const int ncol = G * D / 8;
+  const int mean_threads = ncol >= kMeanThreads ? kMeanThreads : ((ncol + 31) / 32) * 32;
+  const size_t mean_smem = static_cast<size_t>(G) * D * 4;
+  dim3 g1(pb.splits, Hkv, n_problems);
   if (D == 128)
     qmean_partial_kernel<128><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G,
                                                                   tickets, n_tickets);
   else
     qmean_partial_kernel<64><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G,
                                                                  tickets, n_tickets);
-  if (D == 128)
-    page_score_select_kernel<128><<<g2, kScoreThreads, 0, s>>>(
-        partial, pool->summary, d_page_table, pb, G, Hkv, d.num_pages, keys, d_out_scores,
-        tickets, top_k, n_recent, d_out_logical, d_out_physical, d_out_count);
-  else
-    page_score_select_kernel<64><<<g2, kScoreThreads, 0, s>>>(
-        partial, pool->summary, d_page_table, pb, G, Hkv, d.num_pages, keys, d_out_scores,
-        tickets, top_k, n_recent, d_out_logical, d_out_physical, d_out_count);
-  return oomb::check_launch();
+  return launch_score_select(pool, partial, nullptr, pb, n_problems, G, d_page_table, top_k,
+                             n_recent, d_out_logical, d_out_physical, d_out_count, d_out_scores,
+                             tickets, keys, s);
 }
 
 // Host-side checks shared by the entry points.
@@ -481,6 +797,49 @@ extern "C" oomb_status oomb_page_topk(const oomb_pool* pool, const void* d_q, in
   return launch_topk(pool, d_q, num_q_heads, pb, 1, d_page_table, top_k, n_recent, d_out_logical,
                      d_out_physical, d_out_count, d_out_scores, d_workspace,
                      static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+// Selection from per-group sums of Q made by the producer of Q (the
+// projection's epilogue): the scores + select kernel alone, one launch.  Its
+// workspace holds the Hkv tickets (zero before the first call; every
+// completed call leaves them at zero) and the keys.
+size_t qsum_workspace_bytes(int Hkv, int n_past) {
+  return align256(static_cast<size_t>(Hkv) * 4) +
+         align256(static_cast<size_t>(Hkv) * key_stride(n_past) * 8);
+}
+
+}  // namespace
+
+extern "C" size_t oomb_page_topk_qsum_workspace_size(int32_t num_kv_heads, int32_t n_past) {
+  if (num_kv_heads <= 0 || n_past < 0) return 0;
+  return qsum_workspace_bytes(num_kv_heads, n_past);
+}
+
+extern "C" oomb_status oomb_page_topk_qsum(const oomb_pool* pool, const float* d_qsum,
+                                           int32_t chunk_len, int32_t num_q_heads,
+                                           const int32_t* d_page_table, int32_t n_past,
+                                           int32_t top_k, int32_t n_recent,
+                                           int32_t* d_out_logical, int32_t* d_out_physical,
+                                           int32_t* d_out_count, float* d_out_scores,
+                                           void* d_workspace, size_t workspace_bytes,
+                                           void* stream) {
+  oomb_status st = check_topk_args(pool, d_qsum, num_q_heads, d_page_table, n_past, top_k,
+                                   n_recent, d_out_logical, d_out_count);
+  if (st != OOMB_OK) return st;
+  if (chunk_len <= 0 || !d_workspace || !oomb::aligned16(d_workspace)) return OOMB_ERR_INVALID_ARG;
+  const oomb_pool_desc& d = pool->desc;
+  if (workspace_bytes < qsum_workspace_bytes(d.num_kv_heads, n_past)) return OOMB_ERR_INVALID_ARG;
+  oomb::DeviceGuard guard(d.device);
+  const Problems pb{nullptr, nullptr, chunk_len, n_past, n_past, chunk_len, 1, pool->d_status};
+  auto* tickets = static_cast<unsigned int*>(d_workspace);
+  auto* keys = reinterpret_cast<unsigned long long*>(
+      static_cast<uint8_t*>(d_workspace) + align256(static_cast<size_t>(d.num_kv_heads) * 4));
+  return launch_score_select(pool, nullptr, d_qsum, pb, 1, num_q_heads / d.num_kv_heads,
+                             d_page_table, top_k, n_recent, d_out_logical, d_out_physical,
+                             d_out_count, d_out_scores, tickets, keys,
+                             static_cast<cudaStream_t>(stream));
 }
 
 extern "C" size_t oomb_page_topk_batched_workspace_size(int32_t n_problems, int32_t num_kv_heads,

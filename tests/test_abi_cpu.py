@@ -136,6 +136,20 @@ def test_topk_workspace_size_formula():
     # query-mean partials (128 slices), q_bar, then the 64-bit page keys
     assert ws == 128 * 4 * 128 * 4 + 4 * 128 * 4 + ((4 * 4094 * 8 + 255) // 256) * 256
     assert L.page_topk_workspace_size(0, 28, 4, 128, 10) == 0
+    # key rows have an even stride (16-byte aligned rows): 4095 pages take 4096 slots
+    assert L.page_topk_workspace_size(4096, 28, 4, 128, 4095) == \
+        128 * 4 * 128 * 4 + 4 * 128 * 4 + 4 * 4096 * 8
+
+
+def test_qsum_topk_workspace_size_formula():
+    """The one-launch selection needs only the counters and the keys."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+    assert L.page_topk_qsum_workspace_size(4, 4032) == a256(4 * 4) + a256(4 * 4032 * 8)
+    assert L.page_topk_qsum_workspace_size(4, 4031) == a256(4 * 4) + a256(4 * 4032 * 8)
+    assert L.page_topk_qsum_workspace_size(2, 0) == a256(2 * 4) + a256(2 * 2 * 8)
+    assert L.page_topk_qsum_workspace_size(0, 10) == 0
+    assert L.page_topk_qsum_workspace_size(4, -1) == 0
 
 
 def test_newer_entry_points_reject_host_pools_without_touching_cuda():
@@ -160,6 +174,8 @@ def test_newer_entry_points_reject_host_pools_without_touching_cuda():
         assert lib.oomb_selftest_wait_limit(pool, None) == L.ERR_INVALID_ARG
         assert lib.oomb_qpage_lists(pool, None, None, None, 64, 4, None, None, None, 8,
                                     None) == L.ERR_INVALID_ARG
+        assert lib.oomb_page_topk_qsum(pool, None, 64, 4, None, 0, 4, 2, None, None, None,
+                                       None, None, 0, None) == L.ERR_INVALID_ARG
     finally:
         L.pool_destroy(pool)
 

@@ -54,6 +54,25 @@ def _check_selection(gpu_lists, ref_scores, n_past, K, R):
             assert kth is not None and abs(ref_scores[g, p] - kth) <= TIE, (g, p)
 
 
+def _topk_qsum(run, qsum, C, Hq, n_past, K, R, ws):
+    """oomb_page_topk_qsum on a caller's workspace (counters zero at first use)."""
+    Hkv = run.w.num_kv_heads
+    dev = run.dev
+    ms = K + R
+    out_l = torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev)
+    out_p = torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(Hkv, dtype=torch.int32, device=dev)
+    sc = torch.zeros((Hkv, max(n_past, 1)), dtype=torch.float32, device=dev)
+    pt = torch.tensor(run.page_table[:n_past] or [0], dtype=torch.int32, device=dev)
+    pk.page_topk_qsum(run.pool, qsum, C, Hq, pt, n_past, K, R, out_l, out_p, cnt, ws,
+                      out_scores=sc)
+    torch.cuda.synchronize()
+    c = cnt.cpu().tolist()
+    lists = [out_l[g, :c[g]].cpu().tolist() for g in range(Hkv)]
+    phys = [out_p[g, :c[g]].cpu().tolist() for g in range(Hkv)]
+    return lists, phys, sc[:, :n_past].double().cpu().numpy()
+
+
 def test_summaries_are_page_means():
     w = synth.Workload("sum", 8, 2, 128, 64, 256, 2, seed=21, page_direction=0.5)
     with PagedRun(w) as r:
@@ -153,3 +172,108 @@ def test_sparse_chunks_match_oracle_on_gpu_selection():
     assert rel_l2(dv, ref["dv"]) <= 1e-2
     # unselected pages of a chunk got nothing from it: compare per-token grad mass
     assert np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
+
+
+@pytest.mark.parametrize("K,R", [(3, 2), (0, 2), (50, 2), (1, 0)])
+def test_topk_from_qsum_matches_oracle(K, R):
+    """Selection from per-group Q sums (one launch).  The sums are formed in
+    fp32 by torch from the chunk's bf16 Q (another summation order than the
+    library's own query mean), so scores match the oracle to fp32 rounding and
+    the kept set matches outside the tie band; the same holds against the
+    two-launch path.  One workspace serves every chunk (growing n_past), so
+    each call must leave its counters at zero for the next."""
+    w = synth.Workload("tq", 14, 2, 128, 64, 256, 6, seed=33, page_direction=0.5)
+    Hq, Hkv, d, C = w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_len
+    G = Hq // Hkv
+    inp = synth.sequence_inputs(w)
+    with PagedRun(w) as r:
+        max_past = (w.num_chunks - 1) * w.pages_per_chunk
+        ws = torch.zeros(pk.page_topk_qsum_workspace_size(Hkv, max_past), dtype=torch.uint8,
+                         device=r.dev)
+        for c in range(w.num_chunks):
+            ch = synth.chunk_inputs(w, c)
+            if c:
+                n_past = c * w.pages_per_chunk
+                qsum = ch["q"].to(r.dev).float().reshape(C, Hkv, G, d).sum(dim=(0, 2))
+                lists, phys, sc = _topk_qsum(r, qsum.contiguous(), C, Hq, n_past, K, R, ws)
+                ref = page_scores(group_query_means(ch["q"], Hkv),
+                                  page_key_means(inp["k"][: c * C], w.page_size))
+                assert np.max(np.abs(sc - ref)) <= 1e-6 + 1e-5 * np.max(np.abs(ref))
+                _check_selection(lists, ref, n_past, K, R)
+                for g in range(Hkv):
+                    assert phys[g] == [r.page_table[p] for p in lists[g]]
+                lists2, _, _ = _topk(r, ch["q"], n_past, K, R, scores=False)
+                for g in range(Hkv):
+                    kth = kth_score(ref[g], n_past, K, R)
+                    for p in set(lists[g]) ^ set(lists2[g]):
+                        assert kth is not None and abs(ref[g, p] - kth) <= TIE, (c, g, p)
+            r.append(ch["k"], ch["v"])
+        assert r.status() == 0
+        assert int(ws[:4 * Hkv].view(torch.int32).abs().sum()) == 0  # counters back at zero
+
+
+def test_topk_from_qsum_many_candidates():
+    """4,096 past pages (radix select from registers at its largest) and then
+    4,100 (the select that re-reads the keys), from Q sums."""
+    Hq, Hkv, d, P = 8, 2, 128, 16
+    for n_pages in (4096, 4100):
+        w = synth.Workload("bigq", Hq, Hkv, d, P, P * n_pages, 1, seed=43, page_direction=0.5,
+                           shuffle_pages=True)
+        gen = torch.Generator().manual_seed(n_pages)
+        k = torch.randn(n_pages * P, Hkv, d, generator=gen)
+        k += 0.5 * torch.randn(n_pages, 1, Hkv, d, generator=gen).expand(
+            n_pages, P, Hkv, d).reshape(-1, Hkv, d)
+        k = k.to(torch.bfloat16)
+        v = torch.randn(n_pages * P, Hkv, d, generator=gen).to(torch.bfloat16)
+        q = torch.randn(192, Hq, d, generator=gen).to(torch.bfloat16)
+        ref = page_scores(group_query_means(q, Hkv), page_key_means(k, P))
+        with PagedRun(w, num_pages=n_pages) as r:
+            r.append(k, v)
+            ws = torch.zeros(pk.page_topk_qsum_workspace_size(Hkv, n_pages), dtype=torch.uint8,
+                             device=r.dev)
+            qsum = q.to(r.dev).float().reshape(192, Hkv, Hq // Hkv, d).sum(dim=(0, 2))
+            for K in (64, 1000):
+                lists, _, _ = _topk_qsum(r, qsum.contiguous(), 192, Hq, n_pages, K, 2, ws)
+                _check_selection(lists, ref, n_pages, K, 2)
+            assert r.status() == 0
+
+
+def test_topk_from_projection_qsum():
+    """Q and its per-group sums from the projection GEMM's epilogue feed the
+    one-launch selection; the oracle selects from its own bf16-rounded
+    projection of the same X and W.  X and W are small integers (W scaled by
+    2^-5), so every fp32 partial sum of the GEMM is exact (|sum| <= 64 in
+    steps of 2^-5) and both sides round the same exact value: the GPU's Q
+    equals the oracle's bit for bit, and the per-group sums (|sum| <= 2^17 in
+    steps of 2^-5) are exact in any order.  What remains is the fp32 scoring,
+    inside the tie band."""
+    from oracle.projection import qkv_projection
+    C, hidden, Hq, Hkv, d, P, n_past = 256, 512, 14, 2, 128, 64, 48
+    gen = torch.Generator().manual_seed(77)
+    x = torch.randint(-2, 3, (C, hidden), generator=gen).to(torch.bfloat16)
+    wt = (torch.randint(-2, 3, ((Hq + 2 * Hkv) * d, hidden), generator=gen) / 32.0).to(
+        torch.bfloat16)
+    k = (torch.randn(n_past * P, Hkv, d, generator=gen)
+         + 0.5 * torch.randn(n_past, 1, Hkv, d, generator=gen).expand(
+             n_past, P, Hkv, d).reshape(-1, Hkv, d)).to(torch.bfloat16)
+    v = torch.randn(n_past * P, Hkv, d, generator=gen).to(torch.bfloat16)
+    q_ref = qkv_projection(x.float().numpy(), wt.float().numpy(), Hq, Hkv, d)[0]
+    q_ref = torch.tensor(q_ref).to(torch.bfloat16).double().numpy()
+    ref = page_scores(group_query_means(q_ref, Hkv), page_key_means(k, P))
+    w = synth.Workload("pq", Hq, Hkv, d, P, n_past * P, 1, seed=78, shuffle_pages=True)
+    with PagedRun(w, num_pages=n_past) as r:
+        r.append(k, v)
+        q = torch.zeros((C, Hq, d), dtype=torch.bfloat16, device=r.dev)
+        qsum = torch.zeros((Hkv, d), dtype=torch.float32, device=r.dev)
+        pk.qkv_project(r.pool, x.to(r.dev), wt.to(r.dev), Hq, pk.PROJ_Q, q=q, qsum=qsum)
+        torch.cuda.synchronize()
+        assert np.array_equal(q.double().cpu().numpy(), q_ref)
+        ws = torch.zeros(pk.page_topk_qsum_workspace_size(Hkv, n_past), dtype=torch.uint8,
+                         device=r.dev)
+        for K, R in ((8, 2), (20, 0)):
+            lists, phys, sc = _topk_qsum(r, qsum, C, Hq, n_past, K, R, ws)
+            assert np.max(np.abs(sc - ref)) <= 1e-5 * max(1.0, np.max(np.abs(ref)))
+            _check_selection(lists, ref, n_past, K, R)
+            for g in range(Hkv):
+                assert phys[g] == [r.page_table[p] for p in lists[g]]
+        assert r.status() == 0
