@@ -501,6 +501,58 @@ __device__ void select_pages_regs(const unsigned long long* keys,
   if (t == 0) *out_count = min(total, max_sel);
 }
 
+// ---------------------------------------------------------------- q_bar sums
+// The query-mean partials of (problem b, group g) summed in one fixed order:
+// thread t of 256 sums splits [64 (t / 128), ...) of column t % 128 in eight
+// chains (sixteen loads in flight, the tail as one more block of sixteen with
+// zeros, x + 0 = x), the chains in a fixed tree; qs[half][d] = that half's
+// sum.  The caller adds the halves (qs[0] + qs[1]).
+template <int D>
+__device__ __forceinline__ void reduce_partials(const float* __restrict__ partial, int splits,
+                                                int Hkv, int b, int g, float (*qs)[D]) {
+  const int t = threadIdx.x, dd = t % 128, half = t / 128;
+  if (dd >= D) return;
+  const float* pp = partial + static_cast<size_t>(b) * splits * Hkv * D + g * D + dd;
+  const int lo = min(splits, half * 64), hi = min(splits, lo + 64);
+  float s8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+  int i = lo;
+  for (; i + 16 <= hi; i += 16) {
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = __ldg(pp + static_cast<size_t>(i + e) * Hkv * D);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
+  }
+  if (i < hi) {
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      v[e] = i + e < hi ? __ldg(pp + static_cast<size_t>(i + e) * Hkv * D) : 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
+  }
+  qs[half][dd] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+}
+
+// A batch's Q sums, once per (group, problem): grid (Hkv, problems), 256
+// threads, a dependent launch after the query mean.  Writes qs[0] + qs[1]
+// into qsum [problems][Hkv][d]; the scores kernel then reads them as Q sums
+// (adding 0 for the second half), so every problem gets bit for bit the q_bar
+// of the one-problem path, whose CTAs each reduce the partials themselves.
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) qsum_reduce_kernel(
+    const float* __restrict__ partial, int splits, float* __restrict__ qsum) {
+  __shared__ float qs[2][D];
+  const int g = blockIdx.x, b = blockIdx.y, Hkv = gridDim.x, t = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  reduce_partials<D>(partial, splits, Hkv, b, g, qs);
+  __syncthreads();
+  if (t < D) qsum[(static_cast<size_t>(b) * Hkv + g) * D + t] = qs[0][t] + qs[1][t];
+}
+
 // ---------------------------------------------------------------- scores + select
 // grid (max(1, ceil(max_past / 64)), Hkv, problems), kScoreThreads threads.
 // Each warp first loads the summaries of its 8 pages (they do not depend on
@@ -514,8 +566,8 @@ __device__ void select_pages_regs(const unsigned long long* keys,
 // [problem][group][key_stride(max_past)].  The CTA whose ticket is the last
 // of its (problem, group) then runs the select and sets the ticket back to
 // zero, so a completed call leaves every ticket at zero.
-template <int D, bool FROM_QSUM>
-__global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
+template <int D, bool FROM_QSUM, bool FUSED_SELECT>
+__global__ void __launch_bounds__(kScoreThreads, FUSED_SELECT ? 3 : 5) page_score_select_kernel(
     const float* __restrict__ partial, const float* __restrict__ qsum,
     const float* __restrict__ summary, const int32_t* __restrict__ page_table, const Problems pb,
     int G, int Hkv, int num_pool_pages, unsigned long long* __restrict__ keys,
@@ -530,12 +582,16 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
   const int g = blockIdx.y, b = blockIdx.z, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int n_past = problem_npast(pb, b);
   const int n_ctas = max(1, (n_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta);
+  if (!FUSED_SELECT) pdl_launch_dependents();
   if (static_cast<int>(blockIdx.x) >= n_ctas) return;  // beyond this problem's pages
 
-  // this warp's page summaries (EPL fp32 per lane and page)
+  // this warp's page summaries (EPL fp32 per lane and page).  One problem:
+  // loaded first, so that the loads overlap the q_bar reduction (and the
+  // query-mean kernel's tail); a batch: loaded after q_bar, which keeps the
+  // registers, and so the occupancy of its many short CTAs, low.
   const int p0 = blockIdx.x * kPagesPerScoreCta + warp * PW;
   float sv[PW][EPL];
-  {
+  auto load_summaries = [&]() {
     int phys[PW];
 #pragma unroll
     for (int i = 0; i < PW; ++i) phys[i] = p0 + i < n_past ? __ldg(page_table + p0 + i) : 0;
@@ -558,7 +614,8 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
         sv[i][1] = v.y;
       }
     }
-  }
+  };
+  if (FUSED_SELECT) load_summaries();
 
   // the query-mean partials and the tickets it zeroed are read from here on
   pdl_wait();
@@ -567,33 +624,10 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
     if (t < D) qs[0][t] = __ldg(qsum + (static_cast<size_t>(b) * Hkv + g) * D + t);
     else if (t >= 128 && t - 128 < D) qs[1][t - 128] = 0.f;
   } else {
-    const int dd = t % 128, half = t / 128;
-    if (dd < D) {
-      const float* pp = partial + static_cast<size_t>(b) * pb.splits * Hkv * D + g * D + dd;
-      const int lo = min(pb.splits, half * 64), hi = min(pb.splits, lo + 64);
-      float s8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s8[e] = 0.f;
-      int i = lo;
-      for (; i + 16 <= hi; i += 16) {
-        float v[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = __ldg(pp + static_cast<size_t>(i + e) * Hkv * D);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
-      }
-      if (i < hi) {  // the tail, as one more block of 16 with zeros past hi (x + 0 = x)
-        float v[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          v[e] = i + e < hi ? __ldg(pp + static_cast<size_t>(i + e) * Hkv * D) : 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
-      }
-      qs[half][dd] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-    }
+    reduce_partials<D>(partial, pb.splits, Hkv, b, g, qs);
   }
   __syncthreads();
+  if (!FUSED_SELECT) load_summaries();
   int r0, r1;
   problem_rows(pb, b, r0, r1);
   const float rows = static_cast<float>(r1 - r0) * static_cast<float>(G);
@@ -634,6 +668,7 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
           static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(p));
     }
   }
+  if (!FUSED_SELECT) return;  // topk_select_kernel selects after this grid
   // the last CTA of this (problem, group) to get here selects (its keys and
   // every other CTA's are visible once their fences precede the ticket)
   __threadfence();
@@ -654,6 +689,29 @@ __global__ void __launch_bounds__(kScoreThreads) page_score_select_kernel(
   if (t == 0) tickets[row] = 0u;  // every CTA of this (problem, group) has counted
 }
 
+// The select alone, one CTA per (group, problem): grid (Hkv, problems), a
+// dependent launch after the scores kernel (of a batch of problems, whose
+// scoring CTAs then carry no select code and run at full occupancy).
+__global__ void __launch_bounds__(kScoreThreads) topk_select_kernel(
+    const unsigned long long* keys, const int32_t* __restrict__ page_table, const Problems pb,
+    int num_pool_pages, int top_k, int n_recent, int32_t* __restrict__ out_logical,
+    int32_t* __restrict__ out_physical, int32_t* __restrict__ out_count) {
+  const int g = blockIdx.x, b = blockIdx.y, Hkv = gridDim.x;
+  const int n_past = problem_npast(pb, b);
+  const size_t row = static_cast<size_t>(b) * Hkv + g;
+  const unsigned long long* key_row = keys + row * key_stride(pb.max_past);
+  const int max_sel = top_k + n_recent;
+  int32_t* out_p = out_physical ? out_physical + row * max_sel : nullptr;
+  pdl_wait();  // the keys of the scores kernel
+  if (n_past <= kScoreThreads * kKeysPerThread)
+    select_pages_regs<kScoreThreads, kKeysPerThread>(key_row, page_table, n_past, top_k, n_recent,
+                                                     num_pool_pages, out_logical + row * max_sel,
+                                                     out_p, out_count + row);
+  else
+    select_pages_cta<kScoreThreads>(key_row, page_table, n_past, top_k, n_recent, num_pool_pages,
+                                    out_logical + row * max_sel, out_p, out_count + row);
+}
+
 // Workspace: partials [problems][splits <= 128][Hkv][d] fp32, a region of
 // [problems][Hkv][d] fp32 whose first problems * Hkv words are the select
 // tickets, then keys [problems][Hkv][key_stride(max_past)] u64.
@@ -664,22 +722,21 @@ size_t workspace_bytes_for(int64_t problems, int Hkv, int D, int max_past) {
   return align256(partial) + align256(qbar) + align256(keys);
 }
 
-// Launches the scores + select kernel; q_bar from the query-mean partials
-// (qsum null) or from per-group sums of Q (partial null).
+// Launches the scores kernel (q_bar from the query-mean partials, or from Q
+// sums when qsum is set) and, for a batch, the select kernel after it.
+// dependent: the scores kernel is a programmatic dependent launch of the
+// kernel before it on the stream (which made its partials or sums).
 oomb_status launch_score_select(const oomb_pool* pool, const float* partial, const float* qsum,
-                                const Problems& pb, int n_problems, int G,
+                                bool dependent, const Problems& pb, int n_problems, int G,
                                 const int32_t* d_page_table, int top_k, int n_recent,
                                 int32_t* d_out_logical, int32_t* d_out_physical,
                                 int32_t* d_out_count, float* d_out_scores, unsigned int* tickets,
                                 unsigned long long* keys, cudaStream_t s) {
   const oomb_pool_desc& d = pool->desc;
   const int Hkv = d.num_kv_heads;
-  dim3 g2(std::max(1, (pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta), Hkv,
-          n_problems);
-  // after the query-mean kernel: a dependent launch (see pdl_wait); from
-  // sums made by an earlier kernel: an ordinary launch
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = g2;
+  cfg.gridDim = dim3(std::max(1, (pb.max_past + kPagesPerScoreCta - 1) / kPagesPerScoreCta),
+                     Hkv, n_problems);
   cfg.blockDim = dim3(kScoreThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -687,25 +744,33 @@ oomb_status launch_score_select(const oomb_pool* pool, const float* partial, con
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = qsum ? 0 : 1;
+  cfg.numAttrs = dependent ? 1 : 0;
   const float* summary = pool->summary;
   const int num_pages = d.num_pages;
+  // one problem: the last scoring CTA of a group selects; a batch: the
+  // scoring CTAs only score and a select kernel follows
+  const bool fused = n_problems == 1;
   cudaError_t e;
 #define OOMB_SCORE_ARGS                                                                    \
   partial, qsum, summary, d_page_table, pb, G, Hkv, num_pages, keys, d_out_scores, tickets, \
       top_k, n_recent, d_out_logical, d_out_physical, d_out_count
-  if (d.head_dim == 128) {
-    if (qsum)
-      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<128, true>, OOMB_SCORE_ARGS);
-    else
-      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<128, false>, OOMB_SCORE_ARGS);
-  } else {
-    if (qsum)
-      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<64, true>, OOMB_SCORE_ARGS);
-    else
-      e = cudaLaunchKernelEx(&cfg, page_score_select_kernel<64, false>, OOMB_SCORE_ARGS);
-  }
+  // (a batch always scores from Q sums: launch_topk reduces its partials once)
+#define OOMB_SCORE_LAUNCH(DD)                                                                   \
+  (!qsum   ? cudaLaunchKernelEx(&cfg, page_score_select_kernel<DD, false, true>, OOMB_SCORE_ARGS) \
+   : fused ? cudaLaunchKernelEx(&cfg, page_score_select_kernel<DD, true, true>, OOMB_SCORE_ARGS)  \
+           : cudaLaunchKernelEx(&cfg, page_score_select_kernel<DD, true, false>, OOMB_SCORE_ARGS))
+  if (!qsum && !fused) return OOMB_ERR_INVALID_ARG;
+  e = d.head_dim == 128 ? OOMB_SCORE_LAUNCH(128) : OOMB_SCORE_LAUNCH(64);
+#undef OOMB_SCORE_LAUNCH
 #undef OOMB_SCORE_ARGS
+  if (e == cudaSuccess && !fused) {
+    cudaLaunchConfig_t sel = cfg;
+    sel.gridDim = dim3(Hkv, n_problems, 1);
+    sel.numAttrs = 1;  // dependent of the scores kernel
+    const unsigned long long* ckeys = keys;
+    e = cudaLaunchKernelEx(&sel, topk_select_kernel, ckeys, d_page_table, pb, num_pages, top_k,
+                           n_recent, d_out_logical, d_out_physical, d_out_count);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return OOMB_ERR_CUDA;
@@ -713,7 +778,9 @@ oomb_status launch_score_select(const oomb_pool* pool, const float* partial, con
   return oomb::check_launch();
 }
 
-// Launches the two kernels for `n_problems` problems on `s`.
+// Launches the selection of `n_problems` problems from Q on `s`: the query
+// mean, then for one problem the fused scores + select kernel, for a batch
+// the Q-sum reduction, the scores kernel and the select kernel.
 oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
                         const Problems& pb_in, int n_problems, const int32_t* d_page_table,
                         int top_k, int n_recent, int32_t* d_out_logical, int32_t* d_out_physical,
@@ -726,8 +793,11 @@ oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
   const size_t partial_bytes = align256(static_cast<size_t>(n_problems) * kSplits * Hkv * D * 4);
   const size_t qbar_bytes = align256(static_cast<size_t>(n_problems) * Hkv * D * 4);
   float* partial = static_cast<float*>(scratch);
+  // the region after the partials: the tickets of the one-problem path, or a
+  // batch's Q sums
   unsigned int* tickets =
       reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(scratch) + partial_bytes);
+  float* batch_qsum = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + partial_bytes);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(
       static_cast<uint8_t*>(scratch) + partial_bytes + qbar_bytes);
   const int n_tickets = n_problems * Hkv;
@@ -743,9 +813,32 @@ oomb_status launch_topk(const oomb_pool* pool, const void* d_q, int num_q_heads,
   else
     qmean_partial_kernel<64><<<g1, mean_threads, mean_smem, s>>>(q, partial, pb, num_q_heads, G,
                                                                  tickets, n_tickets);
-  return launch_score_select(pool, partial, nullptr, pb, n_problems, G, d_page_table, top_k,
-                             n_recent, d_out_logical, d_out_physical, d_out_count, d_out_scores,
-                             tickets, keys, s);
+  if (n_problems == 1)
+    return launch_score_select(pool, partial, nullptr, true, pb, 1, G, d_page_table, top_k,
+                               n_recent, d_out_logical, d_out_physical, d_out_count,
+                               d_out_scores, tickets, keys, s);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(Hkv, n_problems, 1);
+  cfg.blockDim = dim3(kScoreThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* cpartial = partial;
+  const int splits = pb.splits;
+  const cudaError_t e =
+      D == 128 ? cudaLaunchKernelEx(&cfg, qsum_reduce_kernel<128>, cpartial, splits, batch_qsum)
+               : cudaLaunchKernelEx(&cfg, qsum_reduce_kernel<64>, cpartial, splits, batch_qsum);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return OOMB_ERR_CUDA;
+  }
+  return launch_score_select(pool, nullptr, batch_qsum, true, pb, n_problems, G, d_page_table,
+                             top_k, n_recent, d_out_logical, d_out_physical, d_out_count,
+                             d_out_scores, tickets, keys, s);
 }
 
 // Host-side checks shared by the entry points.
@@ -836,7 +929,7 @@ extern "C" oomb_status oomb_page_topk_qsum(const oomb_pool* pool, const float* d
   auto* tickets = static_cast<unsigned int*>(d_workspace);
   auto* keys = reinterpret_cast<unsigned long long*>(
       static_cast<uint8_t*>(d_workspace) + align256(static_cast<size_t>(d.num_kv_heads) * 4));
-  return launch_score_select(pool, nullptr, d_qsum, pb, 1, num_q_heads / d.num_kv_heads,
+  return launch_score_select(pool, nullptr, d_qsum, false, pb, 1, num_q_heads / d.num_kv_heads,
                              d_page_table, top_k, n_recent, d_out_logical, d_out_physical,
                              d_out_count, d_out_scores, tickets, keys,
                              static_cast<cudaStream_t>(stream));
