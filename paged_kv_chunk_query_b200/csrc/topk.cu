@@ -55,6 +55,18 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Ticket of a CTA that has written its keys: one acquire-release atomic add
+// at GPU scope by one thread, between two CTA barriers.  The release covers
+// the whole CTA's earlier writes (the first barrier orders them before it,
+// and release is cumulative); the CTA that draws the last ticket acquires
+// every earlier CTA's release, and its second barrier orders all of its
+// threads' later loads after that acquire.
+__device__ __forceinline__ unsigned int ticket_acq_rel(unsigned int* p) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
 // Row stride of the 64-bit key array: even, so that every row starts on a
 // 16-byte boundary and key pairs load as one vector.
 __host__ __device__ __forceinline__ int key_stride(int max_past) {
@@ -504,12 +516,15 @@ __device__ void select_pages_regs(const unsigned long long* keys,
 // ---------------------------------------------------------------- q_bar sums
 // The query-mean partials of (problem b, group g) summed in one fixed order:
 // thread t of 256 sums splits [64 (t / 128), ...) of column t % 128 in eight
-// chains (sixteen loads in flight, the tail as one more block of sixteen with
-// zeros, x + 0 = x), the chains in a fixed tree; qs[half][d] = that half's
-// sum.  The caller adds the halves (qs[0] + qs[1]).
-template <int D>
+// chains (split i goes to chain i mod 8, in increasing i; blocks of B loads
+// in flight, the tail as one more block with zeros, x + 0 = x), the chains
+// in a fixed tree; qs[half][d] = that half's sum.  The caller adds the halves
+// (qs[0] + qs[1]).  B (loads in flight, a multiple of 8) changes only the
+// registers used, not the result.
+template <int D, int B>
 __device__ __forceinline__ void reduce_partials(const float* __restrict__ partial, int splits,
                                                 int Hkv, int b, int g, float (*qs)[D]) {
+  static_assert(B % 8 == 0, "chains");
   const int t = threadIdx.x, dd = t % 128, half = t / 128;
   if (dd >= D) return;
   const float* pp = partial + static_cast<size_t>(b) * splits * Hkv * D + g * D + dd;
@@ -518,20 +533,20 @@ __device__ __forceinline__ void reduce_partials(const float* __restrict__ partia
 #pragma unroll
   for (int e = 0; e < 8; ++e) s8[e] = 0.f;
   int i = lo;
-  for (; i + 16 <= hi; i += 16) {
-    float v[16];
+  for (; i + B <= hi; i += B) {
+    float v[B];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) v[e] = __ldg(pp + static_cast<size_t>(i + e) * Hkv * D);
+    for (int e = 0; e < B; ++e) v[e] = __ldg(pp + static_cast<size_t>(i + e) * Hkv * D);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
+    for (int e = 0; e < B; ++e) s8[e & 7] += v[e];
   }
   if (i < hi) {
-    float v[16];
+    float v[B];
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
+    for (int e = 0; e < B; ++e)
       v[e] = i + e < hi ? __ldg(pp + static_cast<size_t>(i + e) * Hkv * D) : 0.f;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) s8[e & 7] += v[e];
+    for (int e = 0; e < B; ++e) s8[e & 7] += v[e];
   }
   qs[half][dd] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
 }
@@ -548,7 +563,7 @@ __global__ void __launch_bounds__(kScoreThreads) qsum_reduce_kernel(
   const int g = blockIdx.x, b = blockIdx.y, Hkv = gridDim.x, t = threadIdx.x;
   pdl_launch_dependents();
   pdl_wait();
-  reduce_partials<D>(partial, splits, Hkv, b, g, qs);
+  reduce_partials<D, 32>(partial, splits, Hkv, b, g, qs);
   __syncthreads();
   if (t < D) qsum[(static_cast<size_t>(b) * Hkv + g) * D + t] = qs[0][t] + qs[1][t];
 }
@@ -567,7 +582,7 @@ __global__ void __launch_bounds__(kScoreThreads) qsum_reduce_kernel(
 // of its (problem, group) then runs the select and sets the ticket back to
 // zero, so a completed call leaves every ticket at zero.
 template <int D, bool FROM_QSUM, bool FUSED_SELECT>
-__global__ void __launch_bounds__(kScoreThreads, FUSED_SELECT ? 3 : 5) page_score_select_kernel(
+__global__ void __launch_bounds__(kScoreThreads, FUSED_SELECT ? 2 : 5) page_score_select_kernel(
     const float* __restrict__ partial, const float* __restrict__ qsum,
     const float* __restrict__ summary, const int32_t* __restrict__ page_table, const Problems pb,
     int G, int Hkv, int num_pool_pages, unsigned long long* __restrict__ keys,
@@ -624,7 +639,7 @@ __global__ void __launch_bounds__(kScoreThreads, FUSED_SELECT ? 3 : 5) page_scor
     if (t < D) qs[0][t] = __ldg(qsum + (static_cast<size_t>(b) * Hkv + g) * D + t);
     else if (t >= 128 && t - 128 < D) qs[1][t - 128] = 0.f;
   } else {
-    reduce_partials<D>(partial, pb.splits, Hkv, b, g, qs);
+    reduce_partials<D, 32>(partial, pb.splits, Hkv, b, g, qs);
   }
   __syncthreads();
   if (!FUSED_SELECT) load_summaries();
@@ -669,14 +684,12 @@ __global__ void __launch_bounds__(kScoreThreads, FUSED_SELECT ? 3 : 5) page_scor
     }
   }
   if (!FUSED_SELECT) return;  // topk_select_kernel selects after this grid
-  // the last CTA of this (problem, group) to get here selects (its keys and
-  // every other CTA's are visible once their fences precede the ticket)
-  __threadfence();
+  // the last CTA of this (problem, group) to get here selects; its ticket
+  // makes every other CTA's keys visible to it (see ticket_acq_rel)
   __syncthreads();
-  if (t == 0) last_sh = atomicAdd(&tickets[row], 1u) == static_cast<unsigned>(n_ctas - 1);
+  if (t == 0) last_sh = ticket_acq_rel(&tickets[row]) == static_cast<unsigned>(n_ctas - 1);
   __syncthreads();
   if (!last_sh) return;
-  __threadfence();
   const int max_sel = top_k + n_recent;
   int32_t* out_p = out_physical ? out_physical + row * max_sel : nullptr;
   if (n_past <= kScoreThreads * kKeysPerThread)
