@@ -26,10 +26,15 @@ c % 3):
   S: store those pages and summaries into the host pool
   S: Top-K for chunk c+1 against the host pool's summaries, its block lists,
      and the prefetch of its blocks into part (c+1) % 3
-  C: forward + backward of chunk c on the staging part
+  C: forward, backward preprocess and dK/dV of chunk c on the staging part;
+     its dQ on a third stream D beside the dK/dV launch (each fills the
+     other's last partial wave of CTAs, as in the device-resident step)
   S: once chunk c-1 has computed, add its gradient blocks into the host pool
      and zero them on the device
-Part (c+1) % 3 was last used by chunk c-2, whose write-back came earlier on S.
+Part (c+1) % 3 was last used by chunk c-2, whose write-back came earlier on S
+and whose dQ C waits for before chunk c's append (after which S starts
+overwriting that part).  Delta, O, LSE and dQ scratch are per part, since
+chunk c's dQ may still read its LSE and delta while chunk c+1 runs on C.
 """
 from __future__ import annotations
 
@@ -62,6 +67,7 @@ class OffloadRun:
         # a higher-priority copy stream: its short kernels take SMs as soon as
         # an attention CTA retires
         self.copy = torch.cuda.Stream(device=device, priority=-1)
+        self.side = torch.cuda.Stream(device=device)   # each chunk's dQ
         C, Hq = w.chunk_len, w.num_q_heads
         heads = np.arange(Hkv, dtype=np.int64)
 
@@ -83,7 +89,8 @@ class OffloadRun:
         self.pf_dst = [torch.full((self.sel_max * Hkv,), -1, **i32) for _ in range(n)]
         ws = L.page_topk_workspace_size(C, Hq, Hkv, d, max(1, (N - 1) * self.ppc))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
-        self.delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device)
+                       for _ in range(n)]
         # every chunk's selection, copied back for inspection (not on the schedule's path)
         self.sel_hist = torch.zeros((N, Hkv, self.sel_max), dtype=torch.int32).pin_memory()
         self.cnt_hist = torch.zeros((N, Hkv), dtype=torch.int32).pin_memory()
@@ -101,24 +108,29 @@ class OffloadRun:
         w = self.w
         N = w.num_chunks
         comp = torch.cuda.current_stream(self.dev)
-        S = self.copy
-        scratch = None
+        S, D = self.copy, self.side
+        scratch = [None] * self.parts
+        dq_done = [None] * self.parts   # event: the dQ of the part's last chunk has finished
         prefetched = None       # event: chunk c's blocks are in its staging part
         prev_computed = None    # event: chunk c-1's backward has finished
         self.copy.wait_stream(comp)
+        D.wait_stream(comp)
         for c in range(N):
             b = c % self.parts
             x = chunks(c)
             if outputs is not None:
                 o, lse, dq = outputs(c)
             else:
-                if scratch is None:
-                    scratch = (torch.empty_like(x["q"]),
-                               torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32,
-                                           device=self.dev), torch.empty_like(x["q"]))
-                o, lse, dq = scratch
+                if scratch[b] is None:
+                    scratch[b] = (torch.empty_like(x["q"]),
+                                  torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32,
+                                              device=self.dev), torch.empty_like(x["q"]))
+                o, lse, dq = scratch[b]
             if prefetched is not None:
                 comp.wait_event(prefetched)
+            b2 = (c + 1) % self.parts   # the part chunk c+1's prefetch overwrites (chunk c-2's)
+            if dq_done[b2] is not None:
+                comp.wait_event(dq_done[b2])
             L.kv_append(self.stage, self.cur_dev[b], x["k"], x["v"], comp)
             appended = torch.cuda.Event()
             appended.record(comp)
@@ -146,8 +158,16 @@ class OffloadRun:
             L.chunk_attn_fwd(self.stage, x["q"], o, lse, past, cnt, self.cur_dev[b],
                              w.softmax_scale, comp)
             if backward:
-                L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, self.delta, past, cnt,
-                                 self.cur_dev[b], w.softmax_scale, comp)
+                delta = self.deltas[b]
+                L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta, past, cnt,
+                                 self.cur_dev[b], w.softmax_scale, comp, step=L.BWD_PREPROCESS)
+                D.wait_stream(comp)
+                L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta, past, cnt,
+                                 self.cur_dev[b], w.softmax_scale, D, step=L.BWD_DQ)
+                dq_done[b] = torch.cuda.Event()
+                dq_done[b].record(D)
+                L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta, past, cnt,
+                                 self.cur_dev[b], w.softmax_scale, comp, step=L.BWD_DKDV)
                 computed = torch.cuda.Event()
                 computed.record(comp)
                 if prev_computed is not None:
@@ -156,6 +176,7 @@ class OffloadRun:
         if backward and prev_computed is not None:
             self._writeback(N - 1, prev_computed)
         comp.wait_stream(S)
+        comp.wait_stream(D)
 
     def _writeback(self, c, computed):
         """Chunk c's gradient blocks (its prefetched blocks and its own pages)
@@ -278,7 +299,11 @@ class DenseOffloadRun:
         self.copy = torch.cuda.Stream(device=device, priority=-1)
         self.o_acc = torch.empty((C, Hq, d), dtype=torch.float32, device=device)
         self.dq_acc = torch.empty_like(self.o_acc)
-        self.delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        # dQ of each backward segment runs on its own stream beside that
+        # segment's dK/dV; chunk c's dQ may still read its delta (and LSE)
+        # while chunk c+1 runs, so these alternate by chunk parity
+        self.side = torch.cuda.Stream(device=device)
+        self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(2)]
         self.h2d_bytes = self.d2h_bytes = 0
 
     def close(self):
@@ -301,25 +326,30 @@ class DenseOffloadRun:
         w = self.w
         Hkv = w.num_kv_heads
         comp = torch.cuda.current_stream(self.dev)
-        X = self.copy
+        X, D = self.copy, self.side
         kv_blk, g_blk = 2 * w.page_size * w.head_dim * 2, 2 * w.page_size * w.head_dim * 4
-        slot_used = [None, None]   # event: last compute on the slot has finished
+        slot_used = [(), ()]       # events: the last compute on the slot has finished
         use = 0                    # slots alternate over every segment call
         cur_free = [None, None]    # event: a chunk-page set's store and write-back are done
+        dq_chunk = [None, None]    # event: the last dQ of the parity's previous chunk is done
         next_first = None          # chunk c+1's first fetch, issued during chunk c
         X.wait_stream(comp)
-        scratch = None
+        D.wait_stream(comp)
+        scratch = [None, None]
         for c in range(w.num_chunks):
             x = chunks(c)
+            cb = c % 2
             if outputs is not None:
                 o, lse, dq = outputs(c)
             else:
-                if scratch is None:
-                    scratch = (torch.empty_like(x["q"]),
-                               torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32,
-                                           device=self.dev), torch.empty_like(x["q"]))
-                o, lse, dq = scratch
-            cb = c % 2
+                if scratch[cb] is None:
+                    scratch[cb] = (torch.empty_like(x["q"]),
+                                   torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32,
+                                               device=self.dev), torch.empty_like(x["q"]))
+                o, lse, dq = scratch[cb]
+            delta = self.deltas[cb]
+            if dq_chunk[cb] is not None:
+                comp.wait_event(dq_chunk[cb])   # chunk c-2's dQ read this delta / scratch
             cur = self.cur_dev[cb]
             if cur_free[cb] is not None:
                 comp.wait_event(cur_free[cb])
@@ -342,8 +372,8 @@ class DenseOffloadRun:
                 nonlocal use
                 slot = use % 2
                 use += 1
-                if slot_used[slot] is not None:
-                    X.wait_event(slot_used[slot])
+                for ev_used in slot_used[slot]:
+                    X.wait_event(ev_used)
                 if n:
                     s = a // self.window
                     L.page_prefetch(self.host, self.stage, self.seg_blocks_host[s][:n * Hkv],
@@ -372,17 +402,26 @@ class DenseOffloadRun:
                                      w.softmax_scale, comp, segment=mode, o_acc=self.o_acc)
                 else:
                     if calls[i - 1][0] == "fwd":
-                        L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, self.delta,
+                        L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta,
                                          None, None, cur, w.softmax_scale, comp,
                                          step=L.BWD_PREPROCESS)
-                    for st in (L.BWD_DKDV, L.BWD_DQ):
-                        L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, self.delta,
-                                         past, cnt, cur, w.softmax_scale, comp,
-                                         step=st, segment=mode, o_acc=self.o_acc,
-                                         dq_acc=self.dq_acc)
+                    # dQ beside dK/dV: D after the slot's fetch and the preprocess
+                    D.wait_stream(comp)
+                    L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta,
+                                     past, cnt, cur, w.softmax_scale, D,
+                                     step=L.BWD_DQ, segment=mode, o_acc=self.o_acc,
+                                     dq_acc=self.dq_acc)
+                    L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta,
+                                     past, cnt, cur, w.softmax_scale, comp,
+                                     step=L.BWD_DKDV, segment=mode, o_acc=self.o_acc,
+                                     dq_acc=self.dq_acc)
                 done = torch.cuda.Event()
                 done.record(comp)
-                slot_used[slot] = done
+                slot_used[slot] = (done,)
+                if kind == "bwd":
+                    done_dq = torch.cuda.Event()
+                    done_dq.record(D)
+                    slot_used[slot] = (done, done_dq)
                 if kind == "bwd" and n:
                     # the segment's gradients into the host pool, zeroed here
                     X.wait_event(done)
@@ -400,7 +439,9 @@ class DenseOffloadRun:
                 _, a1, n1 = self._segments(c + 1)[0]
                 next_first = fetch(a1, n1)
             if backward:
-                X.wait_event(slot_used[last_slot])
+                for ev_used in slot_used[last_slot]:
+                    X.wait_event(ev_used)
+                dq_chunk[cb] = slot_used[last_slot][-1]
                 self._grads_back(self.cur_blocks[cb], self.own_blocks[c], self.cur_blocks_host[cb],
                                  self.own_blocks_host[c], X)
                 if self.grad_path == "gpu":
@@ -409,6 +450,7 @@ class DenseOffloadRun:
             cur_free[cb] = torch.cuda.Event()
             cur_free[cb].record(X)
         comp.wait_stream(X)
+        comp.wait_stream(D)
 
     def sync(self):
         """Waits for the device and, on the host path, every queued addition."""
