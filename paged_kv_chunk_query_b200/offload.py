@@ -19,8 +19,8 @@ stays on the device, oomb_prefetch_lists turns it into block lists, and
 oomb_block_copy / oomb_grad_block_add move the blocks by reading and writing
 the pinned pages in place (one launch per list).  The host only enqueues.
 
-Per chunk c (compute stream C, copy stream S with higher priority; part =
-c % 3):
+Per chunk c (compute stream C, copy stream S and write-back stream W with
+higher priority; part = c % 3):
   C: wait for prefetch(c); append K_c, V_c into the part's current pages
      (page summaries, zeroed gradient blocks)
   S: store those pages and summaries into the host pool
@@ -29,12 +29,17 @@ c % 3):
   C: forward, backward preprocess and dK/dV of chunk c on the staging part;
      its dQ on a third stream D beside the dK/dV launch (each fills the
      other's last partial wave of CTAs, as in the device-resident step)
-  S: once chunk c-1 has computed, add its gradient blocks into the host pool
+  W: once chunk c-1 has computed, add its gradient blocks into the host pool
      and zero them on the device
-Part (c+1) % 3 was last used by chunk c-2, whose write-back came earlier on S
-and whose dQ C waits for before chunk c's append (after which S starts
-overwriting that part).  Delta, O, LSE and dQ scratch are per part, since
-chunk c's dQ may still read its LSE and delta while chunk c+1 runs on C.
+The write-backs have their own stream so that the prefetch chain of the next
+chunk (store, Top-K, lists, gather on S) does not queue behind a write-back:
+on one copy stream the compute stream waited about 0.3 ms per chunk for its
+prefetch.  Part (c+1) % 3 was last used by chunk c-2: S waits for that
+chunk's write-back (which reads the part's block lists and zeroes its
+gradient blocks) before rebuilding the lists, and C waits for its dQ before
+chunk c's append (after which S starts overwriting the part).  Delta, O, LSE
+and dQ scratch are per part, since chunk c's dQ may still read its LSE and
+delta while chunk c+1 runs on C.
 """
 from __future__ import annotations
 
@@ -67,6 +72,7 @@ class OffloadRun:
         # a higher-priority copy stream: its short kernels take SMs as soon as
         # an attention CTA retires
         self.copy = torch.cuda.Stream(device=device, priority=-1)
+        self.wb = torch.cuda.Stream(device=device, priority=-1)   # gradient write-backs
         self.side = torch.cuda.Stream(device=device)   # each chunk's dQ
         C, Hq = w.chunk_len, w.num_q_heads
         heads = np.arange(Hkv, dtype=np.int64)
@@ -108,13 +114,15 @@ class OffloadRun:
         w = self.w
         N = w.num_chunks
         comp = torch.cuda.current_stream(self.dev)
-        S, D = self.copy, self.side
+        S, D, W = self.copy, self.side, self.wb
         scratch = [None] * self.parts
         dq_done = [None] * self.parts   # event: the dQ of the part's last chunk has finished
+        self.wb_done = [None] * self.parts  # event: the part's last write-back has finished
         prefetched = None       # event: chunk c's blocks are in its staging part
         prev_computed = None    # event: chunk c-1's backward has finished
         self.copy.wait_stream(comp)
         D.wait_stream(comp)
+        W.wait_stream(comp)
         for c in range(N):
             b = c % self.parts
             x = chunks(c)
@@ -144,6 +152,8 @@ class OffloadRun:
                 L.page_topk(self.host, chunks(c + 1)["q"], self.table_dev[:n_past], n_past,
                             w.top_k, w.n_recent, self.sel_l[b1], None, self.cnt_dev[b1], self.ws,
                             stream=S)
+                if self.wb_done[b1] is not None:   # chunk c-2's write-back read these lists
+                    S.wait_event(self.wb_done[b1])
                 L.prefetch_lists(self.host, self.stage, self.sel_l[b1], self.cnt_dev[b1],
                                  self.table_dev[:n_past], self.slots_dev[b1], self.pf_src[b1],
                                  self.pf_dst[b1], self.past_dev[b1], stream=S)
@@ -177,17 +187,21 @@ class OffloadRun:
             self._writeback(N - 1, prev_computed)
         comp.wait_stream(S)
         comp.wait_stream(D)
+        comp.wait_stream(W)
 
     def _writeback(self, c, computed):
         """Chunk c's gradient blocks (its prefetched blocks and its own pages)
-        added into the host pool on the copy stream, zeroed on the device."""
+        added into the host pool on the write-back stream, zeroed on the
+        device."""
         b = c % self.parts
-        S = self.copy
-        S.wait_event(computed)
+        W = self.wb
+        W.wait_event(computed)
         if c > 0:
-            L.grad_block_add(self.stage, self.host, self.pf_dst[b], self.pf_src[b], True, stream=S)
+            L.grad_block_add(self.stage, self.host, self.pf_dst[b], self.pf_src[b], True, stream=W)
         L.grad_block_add(self.stage, self.host, self.cur_blocks[b], self.own_host_blocks[c], True,
-                         stream=S)
+                         stream=W)
+        self.wb_done[b] = torch.cuda.Event()
+        self.wb_done[b].record(W)
 
     def sync(self):
         """Waits for the device (every copy and gradient addition is stream-ordered)."""
