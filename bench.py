@@ -670,7 +670,7 @@ def offload_run(w, steps, device, dist_on):
 
 def dense_offload_run(w, window, device, dist_on, grad_path="host"):
     """Dense 256K with KV and gradients in pinned host memory and a window of
-    `window` past pages (two slots) on the device; one step = all chunks,
+    `window` past pages per slot (three slots) on the device; one step = all chunks,
     timed with CUDA events on the compute stream (1 warm-up step)."""
     from paged_kv_chunk_query_b200 import synth
     from paged_kv_chunk_query_b200.offload import DenseOffloadRun
@@ -692,14 +692,15 @@ def dense_offload_run(w, window, device, dist_on, grad_path="host"):
         import paged_kv_chunk_query_b200 as pk
         status = pk.get_device_status(run.stage) | pk.get_device_status(run.host)
         P, Hkv, d = w.page_size, w.num_kv_heads, w.head_dim
-        dev_bytes = (2 * window + w.pages_per_chunk) * Hkv * 2 * P * d * (2 + 4)
+        dev_bytes = (run.slots * window + 2 * w.pages_per_chunk) * Hkv * 2 * P * d * (2 + 4)
         full_bytes = w.num_pages * Hkv * 2 * P * d * (2 + 4)
         h2d, d2h = run.h2d_bytes, run.d2h_bytes
     finally:
         run.close()
         del ins
         torch.cuda.empty_cache()
-    return {"workload": w.name, "window_pages": window, "grad_path": grad_path,
+    return {"workload": w.name, "window_pages": window, "slots": run.slots,
+            "grad_path": grad_path,
             "ms_per_step": ms,
             "tokens_per_s": w.context / (ms / 1e3),
             "device_window_bytes": dev_bytes, "full_pool_bytes": full_bytes,

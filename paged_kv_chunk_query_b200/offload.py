@@ -248,39 +248,51 @@ class DenseOffloadRun:
     bounded device window ([pt] §2D: pages move between host and GPU on
     dedicated streams while computation runs; the pages' dense-model case).
 
-    The device holds two slots of ``window`` pages each plus the chunk's own
-    pages.  A chunk's past is taken in segments of ``window`` pages: the
-    forward merges them into an fp32 running output (oomb segment modes,
-    FIRST / NEXT / LAST, the last with the chunk itself), then the backward
-    streams the same segments again, and each segment's gradient blocks are
-    added into the host pool (and zeroed) as soon as its backward is done.
-    While one slot computes, the copy stream (higher priority) fills the
-    other; the chunk's own pages are appended on the device, stored to the
-    host pool, and their gradients added back after the chunk's backward.
+    The device holds ``slots`` slots of ``window`` pages each plus two sets
+    of the chunk's own pages.  A chunk's past is taken in segments of
+    ``window`` pages: the forward merges them into an fp32 running output
+    (oomb segment modes, FIRST / NEXT / LAST, the last with the chunk itself),
+    then the backward streams the same segments again, and each segment's
+    gradient blocks are added into the host pool (and zeroed) as soon as its
+    backward is done.  Calls take the slots in turn, and each call's pages
+    are fetched ``slots - 1`` calls ahead on a fetch stream (higher priority),
+    while a write-back stream stores the chunk's own pages and returns the
+    gradients, so the link's two directions run at once and a fetch never
+    queues behind a gradient copy.  The chunk's own pages are appended on the
+    device, stored to the host pool, and their gradients added back after the
+    chunk's backward.
 
     Host pages are taken in logical order (and the slots' pages in order), so
     a segment is one contiguous range in both pools: its K/V travel as one
     copy-engine transfer (oomb_page_prefetch merges consecutive blocks), which
     takes no SM from the attention kernels; only the gradient additions run
     as (small) kernels over the host link.
+
+    Ordering (events): a slot's next fetch waits for the slot's last compute
+    (both streams of a backward call) and its gradient write-back; the
+    fetches of chunk c+1 wait for chunk c's pages to be stored; chunk c+2's
+    append waits for chunk c's own pages to be stored and written back.
     """
 
-    def __init__(self, w, device, window, grad_path="host"):
+    def __init__(self, w, device, window, grad_path="host", slots=3):
         """grad_path "gpu": a kernel adds each segment's gradient blocks into the
         pinned host pages over the host link; "host": they are copied
         device -> host (copy engine) and a library worker thread adds them with
         CPU threads (oomb_grad_writeback), leaving the link's host -> device
-        direction to the K/V."""
-        self.w, self.dev, self.window = w, device, window
+        direction to the K/V.  slots >= 2: device slots of `window` pages (the
+        fetch lead is slots - 1 calls)."""
+        if slots < 2:
+            raise ValueError("slots must be at least 2")
+        self.w, self.dev, self.window, self.slots = w, device, window, slots
         self.grad_path = grad_path
         P, Hkv, d, N = w.page_size, w.num_kv_heads, w.head_dim, w.num_chunks
         C, Hq = w.chunk_len, w.num_q_heads
         self.ppc = w.pages_per_chunk
         self.host = L.pool_create(w.num_pages, P, Hkv, d, L.LOC_PINNED_HOST, True, 0,
                                   device.index or 0)
-        # two slots of `window` pages and two sets of the chunk's own pages (used
-        # by chunks in turn, so chunk c+1 appends while chunk c's drain)
-        n_stage = 2 * window + 2 * self.ppc
+        # `slots` slots of `window` pages and two sets of the chunk's own pages
+        # (used by chunks in turn, so chunk c+1 appends while chunk c's drain)
+        n_stage = slots * window + 2 * self.ppc
         self.stage = L.pool_create(n_stage, P, Hkv, d, L.LOC_DEVICE, True, 0, device.index or 0)
         sp = np.array([L.pool_alloc_page(self.stage) for _ in range(n_stage)], dtype=np.int64)
         self.table = np.array([L.pool_alloc_page(self.host) for _ in range(N * self.ppc)],
@@ -291,12 +303,13 @@ class DenseOffloadRun:
         def blocks(pages):
             return (np.asarray(pages, dtype=np.int64)[:, None] * Hkv + heads[None, :]).reshape(-1)
 
-        slots = [sp[:window], sp[window:2 * window]]
-        curs = [sp[2 * window:2 * window + self.ppc], sp[2 * window + self.ppc:]]
-        self.slot_blocks = [torch.tensor(blocks(x), **i32) for x in slots]
-        self.slot_blocks_host = [blocks(x) for x in slots]
+        slot_pages = [sp[i * window:(i + 1) * window] for i in range(slots)]
+        base = slots * window
+        curs = [sp[base:base + self.ppc], sp[base + self.ppc:]]
+        self.slot_blocks = [torch.tensor(blocks(x), **i32) for x in slot_pages]
+        self.slot_blocks_host = [blocks(x) for x in slot_pages]
         # the past list of a slot: its pages, the same for every group
-        self.slot_lists = [torch.tensor(np.tile(x, (Hkv, 1)), **i32) for x in slots]
+        self.slot_lists = [torch.tensor(np.tile(x, (Hkv, 1)), **i32) for x in slot_pages]
         self.counts = torch.tensor(np.repeat(np.arange(window + 1)[:, None], Hkv, 1), **i32)
         self.cur_dev = [torch.tensor(x, **i32) for x in curs]
         self.cur_blocks = [torch.tensor(blocks(x), **i32) for x in curs]
@@ -310,7 +323,8 @@ class DenseOffloadRun:
             self.seg_blocks_host.append(blocks(pages))
         self.own_blocks = torch.tensor(blocks(self.table).reshape(N, -1), **i32)
         self.own_blocks_host = blocks(self.table).reshape(N, -1)
-        self.copy = torch.cuda.Stream(device=device, priority=-1)
+        self.copy = torch.cuda.Stream(device=device, priority=-1)   # fetches (host -> device)
+        self.wb = torch.cuda.Stream(device=device, priority=-1)     # stores and gradients back
         self.o_acc = torch.empty((C, Hq, d), dtype=torch.float32, device=device)
         self.dq_acc = torch.empty_like(self.o_acc)
         # dQ of each backward segment runs on its own stream beside that
@@ -338,19 +352,56 @@ class DenseOffloadRun:
 
     def run(self, chunks, outputs=None, backward=True):
         w = self.w
-        Hkv = w.num_kv_heads
+        Hkv, N = w.num_kv_heads, w.num_chunks
         comp = torch.cuda.current_stream(self.dev)
-        X, D = self.copy, self.side
+        F, B, D = self.copy, self.wb, self.side
         kv_blk, g_blk = 2 * w.page_size * w.head_dim * 2, 2 * w.page_size * w.head_dim * 4
-        slot_used = [(), ()]       # events: the last compute on the slot has finished
-        use = 0                    # slots alternate over every segment call
+        lead = self.slots - 1
+        slot_used = [() for _ in range(self.slots)]  # events a slot's next fetch waits for
         cur_free = [None, None]    # event: a chunk-page set's store and write-back are done
         dq_chunk = [None, None]    # event: the last dQ of the parity's previous chunk is done
-        next_first = None          # chunk c+1's first fetch, issued during chunk c
-        X.wait_stream(comp)
-        D.wait_stream(comp)
+        stored = [None] * N        # event: chunk c's own pages are in the host pool
+        for st in (F, B, D):
+            st.wait_stream(comp)
         scratch = [None, None]
-        for c in range(w.num_chunks):
+
+        def calls_of(c):
+            segs = self._segments(c)
+            return [(c, "fwd") + sg for sg in segs] + \
+                ([(c, "bwd") + sg for sg in segs] if backward else [])
+
+        # every call of the run in order: (chunk, kind, segment mode, first page, pages)
+        seq = [call for c in range(N) for call in calls_of(c)]
+        fetched = {}               # call index -> (slot, event after its fetch)
+        nxt = 0                    # the next call to fetch
+        use = 0                    # calls take the slots in turn
+
+        def fetch_upto(j_max, cur_chunk):
+            """Fetches the calls up to j_max, stopping before any call of a chunk
+            beyond cur_chunk + 1 (its past would hold pages not stored yet)."""
+            nonlocal nxt, use
+            while nxt <= min(j_max, len(seq) - 1):
+                c2, _, _, a, n = seq[nxt]
+                if c2 > cur_chunk + 1:
+                    break
+                slot = use % self.slots
+                use += 1
+                for ev_used in slot_used[slot]:
+                    F.wait_event(ev_used)
+                if c2 >= 1:
+                    F.wait_event(stored[c2 - 1])
+                if n:
+                    sgi = a // self.window
+                    L.page_prefetch(self.host, self.stage, self.seg_blocks_host[sgi][:n * Hkv],
+                                    self.slot_blocks_host[slot][:n * Hkv], stream=F)
+                    self.h2d_bytes += n * Hkv * kv_blk
+                e = torch.cuda.Event()
+                e.record(F)
+                fetched[nxt] = (slot, e)
+                nxt += 1
+
+        i = 0
+        for c in range(N):
             x = chunks(c)
             cb = c % 2
             if outputs is not None:
@@ -370,55 +421,32 @@ class DenseOffloadRun:
             L.kv_append(self.stage, cur, x["k"], x["v"], comp)
             ev = torch.cuda.Event()
             ev.record(comp)
-            X.wait_event(ev)
+            B.wait_event(ev)
             L.page_prefetch(self.stage, self.host, self.cur_blocks_host[cb], self.own_blocks_host[c],
-                            stream=X)
+                            stream=B)
             self.d2h_bytes += self.ppc * Hkv * kv_blk
-            segs = self._segments(c)
-            # every call of the chunk in order: the forward segments, then the
-            # backward ones; each needs its segment's pages in a slot
-            calls = [("fwd",) + sg for sg in segs] + \
-                ([("bwd",) + sg for sg in segs] if backward else [])
-
-            def fetch(a, n):
-                """Segment pages into the next slot on the copy stream; returns
-                (slot, event after the copy)."""
-                nonlocal use
-                slot = use % 2
-                use += 1
-                for ev_used in slot_used[slot]:
-                    X.wait_event(ev_used)
-                if n:
-                    s = a // self.window
-                    L.page_prefetch(self.host, self.stage, self.seg_blocks_host[s][:n * Hkv],
-                                    self.slot_blocks_host[slot][:n * Hkv], stream=X)
-                    self.h2d_bytes += n * Hkv * kv_blk
-                e = torch.cuda.Event()
-                e.record(X)
-                return slot, e
-
-            def lists(slot, n):
-                return (self.slot_lists[slot], self.counts[n]) if n else (None, None)
-
-            # prefetch one call ahead: call i+1's pages are queued on the copy
-            # stream before call i's gradient write-back, so they arrive while
-            # call i computes
-            fetched = {0: next_first if next_first is not None else fetch(calls[0][2], calls[0][3])}
-            next_first = None
-            for i, (kind, mode, a, n) in enumerate(calls):
-                if i + 1 < len(calls):
-                    fetched[i + 1] = fetch(calls[i + 1][2], calls[i + 1][3])
+            stored[c] = torch.cuda.Event()
+            stored[c].record(B)
+            first_bwd = True
+            last = ()
+            while i < len(seq) and seq[i][0] == c:
+                fetch_upto(i + lead, c)
+                _, kind, mode, a, n = seq[i]
                 slot, e = fetched.pop(i)
                 comp.wait_event(e)
-                past, cnt = lists(slot, n)
+                past, cnt = (self.slot_lists[slot], self.counts[n]) if n else (None, None)
                 if kind == "fwd":
                     L.chunk_attn_fwd(self.stage, x["q"], o, lse, past, cnt, cur,
                                      w.softmax_scale, comp, segment=mode, o_acc=self.o_acc)
+                    done = torch.cuda.Event()
+                    done.record(comp)
+                    slot_used[slot] = (done,)
                 else:
-                    if calls[i - 1][0] == "fwd":
+                    if first_bwd:
                         L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta,
                                          None, None, cur, w.softmax_scale, comp,
                                          step=L.BWD_PREPROCESS)
+                        first_bwd = False
                     # dQ beside dK/dV: D after the slot's fetch and the preprocess
                     D.wait_stream(comp)
                     L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta,
@@ -429,41 +457,40 @@ class DenseOffloadRun:
                                      past, cnt, cur, w.softmax_scale, comp,
                                      step=L.BWD_DKDV, segment=mode, o_acc=self.o_acc,
                                      dq_acc=self.dq_acc)
-                done = torch.cuda.Event()
-                done.record(comp)
-                slot_used[slot] = (done,)
-                if kind == "bwd":
+                    done = torch.cuda.Event()
+                    done.record(comp)
                     done_dq = torch.cuda.Event()
                     done_dq.record(D)
-                    slot_used[slot] = (done, done_dq)
-                if kind == "bwd" and n:
-                    # the segment's gradients into the host pool, zeroed here
-                    X.wait_event(done)
-                    s = a // self.window
-                    self._grads_back(self.slot_blocks[slot][:n * Hkv],
-                                     self.seg_blocks[s][:n * Hkv],
-                                     self.slot_blocks_host[slot][:n * Hkv],
-                                     self.seg_blocks_host[s][:n * Hkv], X)
-                    if self.grad_path == "gpu":
-                        self.h2d_bytes += n * Hkv * g_blk
-                    self.d2h_bytes += n * Hkv * g_blk
-            last_slot = (use - 1) % 2
-            if c + 1 < w.num_chunks:
-                # the next chunk's first segment comes in while this one drains
-                _, a1, n1 = self._segments(c + 1)[0]
-                next_first = fetch(a1, n1)
+                    last = (done, done_dq)
+                    slot_used[slot] = last
+                    if n:
+                        # the segment's gradients into the host pool, zeroed here
+                        B.wait_event(done)
+                        sgi = a // self.window
+                        self._grads_back(self.slot_blocks[slot][:n * Hkv],
+                                         self.seg_blocks[sgi][:n * Hkv],
+                                         self.slot_blocks_host[slot][:n * Hkv],
+                                         self.seg_blocks_host[sgi][:n * Hkv], B)
+                        gb = torch.cuda.Event()
+                        gb.record(B)
+                        slot_used[slot] = last + (gb,)
+                        if self.grad_path == "gpu":
+                            self.h2d_bytes += n * Hkv * g_blk
+                        self.d2h_bytes += n * Hkv * g_blk
+                i += 1
             if backward:
-                for ev_used in slot_used[last_slot]:
-                    X.wait_event(ev_used)
-                dq_chunk[cb] = slot_used[last_slot][-1]
+                # the chunk's own gradients (final after its last dK/dV)
+                B.wait_event(last[0])
                 self._grads_back(self.cur_blocks[cb], self.own_blocks[c], self.cur_blocks_host[cb],
-                                 self.own_blocks_host[c], X)
+                                 self.own_blocks_host[c], B)
                 if self.grad_path == "gpu":
                     self.h2d_bytes += self.ppc * Hkv * g_blk
                 self.d2h_bytes += self.ppc * Hkv * g_blk
+                dq_chunk[cb] = last[1]   # its dQ read the chunk's pages, delta and LSE
             cur_free[cb] = torch.cuda.Event()
-            cur_free[cb].record(X)
-        comp.wait_stream(X)
+            cur_free[cb].record(B)
+        comp.wait_stream(F)
+        comp.wait_stream(B)
         comp.wait_stream(D)
 
     def sync(self):

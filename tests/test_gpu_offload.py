@@ -147,11 +147,14 @@ def _check_outputs_against_oracle(outs, orc):
     assert rel_l2(dq, orc["dq"]) <= 1e-2
 
 
-@pytest.mark.parametrize("window,grad_path", [(3, "gpu"), (20, "gpu"), (3, "host")])
-def test_dense_offload_matches_device_resident_run(window, grad_path):
-    """Dense attention with KV and gradients in pinned host memory and a
-    window of `window` past pages on the device (segments merged in fp32)
-    against the device-resident dense run and the oracle."""
+@pytest.mark.parametrize("window,grad_path,slots", [(3, "gpu", 3), (20, "gpu", 3),
+                                                    (3, "host", 3), (3, "gpu", 2),
+                                                    (2, "host", 2), (3, "host", 4)])
+def test_dense_offload_matches_device_resident_run(window, grad_path, slots):
+    """Dense attention with KV and gradients in pinned host memory and
+    `slots` slots of `window` past pages on the device (segments merged in
+    fp32; fetches slots - 1 calls ahead) against the device-resident dense
+    run and the oracle."""
     from paged_kv_chunk_query_b200.offload import DenseOffloadRun
     dev = torch.device("cuda", 0)
     w = synth.Workload("doff", 14, 2, 128, 64, 256, 5, seed=67, shuffle_pages=True)
@@ -159,7 +162,7 @@ def test_dense_offload_matches_device_resident_run(window, grad_path):
     C, Hq = w.chunk_len, w.num_q_heads
     outs = [(torch.empty_like(x["q"]), torch.empty((Hq, C), dtype=torch.float32, device=dev),
              torch.empty_like(x["q"])) for x in ins]
-    run = DenseOffloadRun(w, dev, window, grad_path)
+    run = DenseOffloadRun(w, dev, window, grad_path, slots)
     try:
         run.run(lambda c: ins[c], lambda c: outs[c])
         run.sync()
