@@ -12,23 +12,30 @@
 //
 // The kernels take a batch of independent problems (blockIdx.z), each a
 // range of query rows and its own number of past pages; the per-chunk entry
-// points run a batch of one.  Two launches:
+// points run a batch of one.
 // Kernel 1 (qmean_partial): grid (slices, Hkv, problems); each CTA streams the
 //   G heads of one group (contiguous in a token row) over a slice of its
 //   problem's rows, one thread per 16-byte column, 16 rows in flight, and
-//   writes one fp32 partial per d.  It also zeroes the tickets kernel 2
-//   counts on.
-// Kernel 2 (page_score_select): grid (pages / 64, Hkv, problems).  Each CTA
-//   sums the slice partials of its (problem, group) in one fixed order into
-//   q_bar (every CTA of a group gets the identical q_bar), then each warp
-//   scores 8 pages (float4 loads of the summaries, shuffle reduction).  The
-//   last CTA of a (problem, group) to finish (a ticket counter; nothing
-//   waits) finds the K-th largest 64-bit key (ordered score, inverted id) by
-//   8-bit radix passes from the top with a parallel bin scan, stopping once
-//   the boundary bin is kept whole, and compacts the kept ids in ascending
-//   order.  Up to 4,096 past pages the keys stay in registers (16 contiguous
-//   pages per thread, warp-aggregated histogram updates, one scan for the
-//   compaction); beyond that they are re-read from L2 on every pass.
+//   writes one fp32 partial per d.  It also zeroes the select tickets.
+// One problem (oomb_page_topk, two launches): kernel 2 (page_score_select,
+//   fused select) is a programmatic dependent launch: grid (pages / 64, Hkv),
+//   each warp loads the summaries of its 8 pages while kernel 1 finishes,
+//   then every CTA sums the slice partials of its group in one fixed order
+//   into q_bar (so all CTAs of a group score against the identical q_bar),
+//   scores its pages into 64-bit keys (ordered score, inverted id), and the
+//   last CTA of the group to take a ticket runs the select.
+// A batch (oomb_page_topk_batched, four dependent launches): a Q-sum kernel
+//   reduces each (problem, group)'s partials once, in the same order; the
+//   scores kernel without the select (few registers, full occupancy); then
+//   one select CTA per (problem, group).
+// From Q sums made by the producer of Q (oomb_page_topk_qsum): the fused
+//   scores + select kernel alone, one launch.
+// The select (up to 4,096 past pages: keys in registers, 16 contiguous pages
+//   per thread): a 256-bucket histogram of the fp32 score on a linear scale
+//   between the candidates' minimum and maximum finds the bucket of the K-th
+//   largest key, exact 8-bit radix passes over the 64-bit keys of that bucket
+//   finish it, and one CTA-wide scan compacts the kept ids in ascending
+//   order; beyond 4,096 pages, 8-bit passes over the keys re-read from L2.
 #include <cuda_bf16.h>
 
 #include <algorithm>
