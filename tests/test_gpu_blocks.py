@@ -229,9 +229,12 @@ def _batched(pool, q, row_start, n_past, max_rows, max_past, table, K, R, Hkv):
     return out_l.cpu(), out_p.cpu(), cnt.cpu(), sc.cpu()
 
 
-def test_batched_topk_equals_per_chunk_calls():
-    """All chunks' selections in one batch == one oomb_page_topk per chunk."""
-    w = synth.Workload("bt", 14, 2, 128, 64, 512, 8, seed=71, page_direction=0.5,
+@pytest.mark.parametrize("d", [128, 64])
+def test_batched_topk_equals_per_chunk_calls(d):
+    """All chunks' selections in one batch == one oomb_page_topk per chunk
+    (the batch reduces its query means once per problem and selects in a
+    kernel of its own; the bits must not change)."""
+    w = synth.Workload("bt", 14, 2, d, 64, 512, 8, seed=71, page_direction=0.5,
                        shuffle_pages=True)
     K, R = 3, 2
     Hkv, ppc, C = w.num_kv_heads, w.pages_per_chunk, w.chunk_len

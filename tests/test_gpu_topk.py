@@ -174,15 +174,16 @@ def test_sparse_chunks_match_oracle_on_gpu_selection():
     assert np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
 
 
-@pytest.mark.parametrize("K,R", [(3, 2), (0, 2), (50, 2), (1, 0)])
-def test_topk_from_qsum_matches_oracle(K, R):
+@pytest.mark.parametrize("K,R,d", [(3, 2, 128), (0, 2, 128), (50, 2, 128), (1, 0, 128),
+                                   (3, 2, 64), (20, 2, 64)])
+def test_topk_from_qsum_matches_oracle(K, R, d):
     """Selection from per-group Q sums (one launch).  The sums are formed in
     fp32 by torch from the chunk's bf16 Q (another summation order than the
     library's own query mean), so scores match the oracle to fp32 rounding and
     the kept set matches outside the tie band; the same holds against the
     two-launch path.  One workspace serves every chunk (growing n_past), so
     each call must leave its counters at zero for the next."""
-    w = synth.Workload("tq", 14, 2, 128, 64, 256, 6, seed=33, page_direction=0.5)
+    w = synth.Workload("tq", 14, 2, d, 64, 256, 6, seed=33, page_direction=0.5)
     Hq, Hkv, d, C = w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_len
     G = Hq // Hkv
     inp = synth.sequence_inputs(w)
