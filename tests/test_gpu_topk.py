@@ -278,3 +278,81 @@ def test_topk_from_projection_qsum():
             for g in range(Hkv):
                 assert phys[g] == [r.page_table[p] for p in lists[g]]
         assert r.status() == 0
+
+
+def test_topk_replayed_from_cuda_graph_equals_eager():
+    """The selections are dependent launches (the scores kernel after the
+    query mean, the batch's kernels after one another): captured in a CUDA
+    graph and replayed, the per-chunk, batched and Q-sum forms give the same
+    lists, counts and scores as eager calls, bit for bit."""
+    w = synth.Workload("tg", 14, 2, 128, 64, 256, 6, seed=35, page_direction=0.5,
+                       shuffle_pages=True)
+    Hq, Hkv, d, C, ppc = w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_len, w.pages_per_chunk
+    K, R = 5, 2
+    ms = K + R
+    dev = torch.device("cuda", 0)
+    with PagedRun(w) as r:
+        qs = []
+        for c in range(w.num_chunks):
+            ch = synth.chunk_inputs(w, c)
+            r.append(ch["k"], ch["v"])
+            qs.append(ch["q"].to(dev).contiguous())
+        n_past = (w.num_chunks - 1) * ppc
+        pt = torch.tensor(r.page_table[:n_past], dtype=torch.int32, device=dev)
+        q_all = torch.cat(qs[1:]).contiguous()
+        nb = w.num_chunks - 1
+        rs = torch.arange(0, (nb + 1) * C, C, dtype=torch.int32, device=dev)
+        npast_b = torch.tensor([c * ppc for c in range(1, w.num_chunks)], dtype=torch.int32,
+                               device=dev)
+        qsum = qs[-1].float().reshape(C, Hkv, Hq // Hkv, d).sum(dim=(0, 2)).contiguous()
+
+        def buffers():
+            return {"l": torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev),
+                    "p": torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev),
+                    "n": torch.zeros(Hkv, dtype=torch.int32, device=dev),
+                    "s": torch.zeros((Hkv, n_past), dtype=torch.float32, device=dev),
+                    "bl": torch.full((nb, Hkv, ms), -1, dtype=torch.int32, device=dev),
+                    "bp": torch.full((nb, Hkv, ms), -1, dtype=torch.int32, device=dev),
+                    "bn": torch.zeros((nb, Hkv), dtype=torch.int32, device=dev),
+                    "ql": torch.full((Hkv, ms), -1, dtype=torch.int32, device=dev),
+                    "qn": torch.zeros(Hkv, dtype=torch.int32, device=dev)}
+
+        ws = torch.empty(pk.page_topk_workspace_size(C, Hq, Hkv, d, n_past), dtype=torch.uint8,
+                         device=dev)
+        wsb = torch.empty(pk.page_topk_batched_workspace_size(nb, Hkv, d, n_past),
+                          dtype=torch.uint8, device=dev)
+        wsq = torch.zeros(pk.page_topk_qsum_workspace_size(Hkv, n_past), dtype=torch.uint8,
+                          device=dev)
+
+        def run(b, st):
+            pk.page_topk(r.pool, qs[-1], pt, n_past, K, R, b["l"], b["p"], b["n"], ws,
+                         out_scores=b["s"], stream=st)
+            pk.page_topk_batched(r.pool, q_all, rs, C, npast_b, n_past, pt, K, R, b["bl"],
+                                 b["bp"], b["bn"], wsb, stream=st)
+            pk.page_topk_qsum(r.pool, qsum, C, Hq, pt, n_past, K, R, b["ql"], None, b["qn"],
+                              wsq, stream=st)
+
+        eager = buffers()
+        for v in eager.values():
+            v.fill_(-7)               # the sentinel the graphed buffers get too
+        run(eager, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        graphed = buffers()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run(graphed, s)           # warm-up outside the capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        for v in graphed.values():
+            v.fill_(-7)               # whatever the replays do not write stays -7, as in eager
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run(graphed, torch.cuda.current_stream())
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        assert r.status() == 0
+        for key in eager:
+            assert torch.equal(eager[key], graphed[key]), key
+        del g
