@@ -1272,7 +1272,9 @@ def main():
 
     e2e = None
     if not a.no_e2e:
+        _barrier(dist_on)
         ms_e, h2d, d2h = e2e_dense(w, max(1, min(a.steps, 2)), device)
+        ms_e = _max_over_ranks(ms_e, dist_on, device)   # every rank runs this line
         e2e = {"value": step_flops * world / (ms_e / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
 
