@@ -324,7 +324,8 @@ oomb_status oomb_page_topk_static(const oomb_pool* pool, const void* d_q, int32_
                                   int32_t* d_out_count, float* d_out_scores, void* stream);
 
 /* Batched Top-K: n_problems independent selections in one set of launches
- * (two kernels for the whole batch).  Problem b takes the query rows
+ * (four dependent kernels for the whole batch: query means, their per-problem
+ * sums, scores, select).  Problem b takes the query rows
  * [d_row_start[b], d_row_start[b+1]) of d_q ([num_rows][num_q_heads][d]
  * bf16) and the candidates among logical pages [0, d_n_past[b]) of the one
  * page table d_page_table (length >= max_past); each problem is exactly one
