@@ -188,6 +188,9 @@ class Run:
         # one delta workspace per chunk: chunk c's dQ launch may still read its
         # delta while chunk c+1's preprocess runs
         self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(N)]
+        # forward workspace (partial O/LSE of a split last wave); every forward
+        # of a step runs on one stream, so one workspace serves them all
+        self.fwd_ws = pk.fwd_workspace(d, device)
         self.side = torch.cuda.Stream(device=device)
         # selections of the next chunk run here, beside the current chunk's attention
         self.sel_stream = torch.cuda.Stream(device=device)
@@ -245,11 +248,16 @@ class Run:
             self.flops["dkdv"].append(8.0 * pairs * d)
             self.flops["dq"].append(2.0 * pairs * d)
         self.step_flops = sum(sum(v) for v in self.flops.values())
-        # per chunk: append, forward, preprocess, dK/dV, dQ; Top-K adds its two
+        # per chunk: append, forward (+ merge), preprocess, dK/dV, dQ; Top-K adds its two
         # launches (query mean; scores with the select) per chunk with a past
         # (per-query-tile lists: and a second dK/dV launch; per-query-page
         # lists: that and the union-list launch); local lists one
-        self.launches_per_step = N * 5 + ((N - 1) * 2 if sparse else 0) + \
+        # the forward's merge launch when its last wave of (query tile, head)
+        # units is split over the free SMs (the launcher's rule)
+        ns = torch.cuda.get_device_properties(device).multi_processor_count
+        tail = ((C + 127) // 128 * Hq) % ns
+        self.fwd_merge = tail > 0 and min(ns // tail, 256 // tail) >= 2
+        self.launches_per_step = N * (5 + int(self.fwd_merge)) + ((N - 1) * 2 if sparse else 0) + \
             ((N - 1) if self.local else 0) + ((N - 1) if self.qtile else 0) + \
             ((N - 1) * 2 if self.qpage else 0)
 
@@ -324,7 +332,8 @@ class Run:
             sc = w.softmax_scale
             delta = self.deltas[c]
             timed("fwd", lambda: pk.chunk_attn_fwd(self.pool, x["q"], o, lse, past, cnt,
-                                                   self.cur[c], sc, F, past_masks=msk), F)
+                                                   self.cur[c], sc, F, past_masks=msk,
+                                                   fwd_ws=self.fwd_ws), F)
             timed("preprocess", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], sc, F,
                 step=pk.BWD_PREPROCESS, past_masks=msk), F)
@@ -410,7 +419,8 @@ class Run:
             s = w.softmax_scale
             delta = self.deltas[c]
             timed("fwd", lambda: pk.chunk_attn_fwd(self.pool, x["q"], o, lse, past, cnt,
-                                                   self.cur[c], s, stream, past_masks=msk))
+                                                   self.cur[c], s, stream, past_masks=msk,
+                                                   fwd_ws=self.fwd_ws))
             timed("preprocess", lambda: pk.chunk_attn_bwd(
                 self.pool, x["q"], o, lse, x["do"], dq, delta, past, cnt, self.cur[c], s, stream,
                 step=pk.BWD_PREPROCESS, past_masks=msk))
@@ -566,6 +576,7 @@ def e2e_dense(w, steps, device):
                     torch.empty((Hq, C), dtype=torch.float32, device=device),
                     torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device)) for _ in range(2)]
         delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        fwd_ws = pk.fwd_workspace(d, device)
         past = [None] + [pt[:c * ppc].repeat(Hkv, 1).contiguous() for c in range(1, N)]
         cnt = [None] + [torch.full((Hkv,), c * ppc, dtype=torch.int32, device=device)
                         for c in range(1, N)]
@@ -599,7 +610,8 @@ def e2e_dense(w, steps, device):
                 o, lse, dq = dev_out[buf]
                 cur = pt[c * ppc:(c + 1) * ppc]
                 pk.kv_append(pool, cur, x["k"], x["v"], comp)
-                pk.chunk_attn_fwd(pool, x["q"], o, lse, past[c], cnt[c], cur, w.softmax_scale, comp)
+                pk.chunk_attn_fwd(pool, x["q"], o, lse, past[c], cnt[c], cur, w.softmax_scale, comp,
+                                  fwd_ws=fwd_ws)
                 pk.chunk_attn_bwd(pool, x["q"], o, lse, x["do"], dq, delta, past[c], cnt[c], cur,
                                   w.softmax_scale, comp)
                 out_ready[c].record(comp)

@@ -176,12 +176,25 @@ typedef struct oomb_attn_args {
   float* o_acc;   /* device fp32 [chunk_len][num_q_heads][head_dim]: running O  */
   float* dq_acc;  /* device fp32, layout of o_acc: running dQ (backward)         */
   const uint8_t* past_masks;  /* lists_per_qtile == 2 only (else ignored), see above */
+  /* Optional forward workspace (device fp32, oomb_chunk_attn_fwd_workspace_size()
+   * bytes, 16-byte aligned; NULL: none).  The forward runs one CTA per (128-row
+   * query tile, query head) and one CTA per SM; when the number of such units is
+   * not a multiple of the SM count, the units of the last, partial wave are split
+   * along their key tiles over the free SMs (whole-key-set calls only), each part
+   * writes a normalised partial O and its LSE here, and a second launch merges
+   * them (LSE = ln sum_k e^LSE_k, O = sum_k e^(LSE_k - LSE) O_k).  Without it the
+   * last wave runs its few units alone.  The backward ignores it.  Calls sharing
+   * a workspace must be ordered (one stream). */
+  float* fwd_ws;
 } oomb_attn_args;
 
 enum { OOMB_SEG_WHOLE = 0, OOMB_SEG_FIRST = 1, OOMB_SEG_NEXT = 2, OOMB_SEG_LAST = 3 };
 
-/* Forward with online softmax; writes o and lse. */
+/* Forward with online softmax; writes o and lse (one launch, or two with a
+ * split last wave, see fwd_ws). */
 oomb_status oomb_chunk_attn_fwd(oomb_pool* pool, const oomb_attn_args* args, void* stream);
+/* Bytes of the optional forward workspace for head_dim (64 or 128); 0 otherwise. */
+size_t oomb_chunk_attn_fwd_workspace_size(int32_t head_dim);
 
 /* Backward of sum(O * dO): writes dq and ADDS dK, dV into the pool's gradient
  * blocks of every page read (fp32 atomic adds, in place; [it] §2B).  Needs o

@@ -10,7 +10,8 @@ compute runs in hand-written CUDA kernels inside ``liboomb.so`` (C ABI in
 from . import _lib
 from ._lib import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, LOC_DEVICE, LOC_HOST, LOC_PINNED_HOST,
                    PROJ_KV, PROJ_Q, PROJ_QKV, SEG_FIRST, SEG_LAST, SEG_NEXT, SEG_WHOLE,
-                   OombError, block_copy, chunk_attn_bwd, chunk_attn_fwd, get_device_status,
+                   OombError, block_copy, chunk_attn_bwd, chunk_attn_fwd, chunk_attn_fwd_workspace_size,
+                   fwd_workspace, get_device_status,
                    grad_block_add, grad_writeback, grad_writeback_sync, kv_append, local_pages, page_prefetch,
                    page_topk, page_topk_batched, page_topk_batched_workspace_size,
                    page_topk_qsum, page_topk_qsum_workspace_size, page_topk_workspace_size, pool_alloc_page, pool_buffers, pool_create,
@@ -28,5 +29,6 @@ __all__ = [
     "LOC_DEVICE", "LOC_PINNED_HOST", "LOC_HOST", "BWD_PREPROCESS", "BWD_DKDV", "BWD_DQ",
     "SEG_WHOLE", "SEG_FIRST", "SEG_NEXT", "SEG_LAST", "PROJ_Q", "PROJ_KV", "PROJ_QKV",
     "qkv_project", "qpage_lists", "page_topk_qsum", "page_topk_qsum_workspace_size",
+    "chunk_attn_fwd_workspace_size", "fwd_workspace",
     "WORKLOADS", "Workload",
 ]

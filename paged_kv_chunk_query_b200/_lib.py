@@ -41,6 +41,7 @@ EXPORTS = (
     "oomb_block_copy", "oomb_grad_block_add", "oomb_prefetch_lists", "oomb_local_pages",
     "oomb_qkv_project", "oomb_selftest_writeback_copy", "oomb_qpage_lists",
     "oomb_page_topk_qsum_workspace_size", "oomb_page_topk_qsum",
+    "oomb_chunk_attn_fwd_workspace_size",
 )
 
 
@@ -66,7 +67,7 @@ class AttnArgs(ctypes.Structure):
                 ("cur_pages", ctypes.c_void_p), ("softmax_scale", ctypes.c_float),
                 ("lists_per_qtile", ctypes.c_int32), ("segment", ctypes.c_int32),
                 ("o_acc", ctypes.c_void_p), ("dq_acc", ctypes.c_void_p),
-                ("past_masks", ctypes.c_void_p)]
+                ("past_masks", ctypes.c_void_p), ("fwd_ws", ctypes.c_void_p)]
 
 
 _lib = None
@@ -126,6 +127,9 @@ def load() -> ctypes.CDLL:
     if hasattr(lib, "oomb_page_topk_qsum_workspace_size"):
         lib.oomb_page_topk_qsum_workspace_size.argtypes = [i32, i32]
         lib.oomb_page_topk_qsum_workspace_size.restype = ctypes.c_size_t
+    if hasattr(lib, "oomb_chunk_attn_fwd_workspace_size"):
+        lib.oomb_chunk_attn_fwd_workspace_size.argtypes = [i32]
+        lib.oomb_chunk_attn_fwd_workspace_size.restype = ctypes.c_size_t
     if hasattr(lib, "oomb_page_topk_batched_workspace_size"):
         lib.oomb_page_topk_batched_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.oomb_page_topk_batched_workspace_size.restype = ctypes.c_size_t
@@ -264,7 +268,8 @@ def kv_append(pool: int, page_ids: torch.Tensor, k: torch.Tensor, v: torch.Tenso
 
 
 def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o=None, dq=None,
-               delta_ws=None, segment=SEG_WHOLE, o_acc=None, dq_acc=None, past_masks=None):
+               delta_ws=None, segment=SEG_WHOLE, o_acc=None, dq_acc=None, past_masks=None,
+               fwd_ws=None):
     """past_pages [Hkv][max_past] (one list per group) or [n_qtiles][Hkv][max_past]
     (one list per 128-row query tile and group; counts [n_qtiles][Hkv]); with
     past_masks (uint8, layout of past_pages) the per-tile lists are unions of
@@ -297,15 +302,31 @@ def _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale, d_o
         _dev_tensor(o_acc, torch.float32, "o_acc") if o_acc is not None else None,
         _dev_tensor(dq_acc, torch.float32, "dq_acc") if dq_acc is not None else None,
         _dev_tensor(past_masks, torch.uint8, "past_masks") if past_masks is not None and max_past
-        else None)
+        else None,
+        _dev_tensor(fwd_ws, torch.float32, "fwd_ws") if fwd_ws is not None else None)
 
 
 def chunk_attn_fwd(pool, q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
-                   stream=None, segment=SEG_WHOLE, o_acc=None, past_masks=None):
+                   stream=None, segment=SEG_WHOLE, o_acc=None, past_masks=None, fwd_ws=None):
+    """fwd_ws: optional fp32 device workspace of chunk_attn_fwd_workspace_size(d) bytes
+    (see fwd_workspace); with it the last partial wave of units is split along its key
+    tiles and merged by a second launch."""
     a = _attn_args(q, o, lse, past_pages, past_counts, cur_pages, softmax_scale,
-                   segment=segment, o_acc=o_acc, past_masks=past_masks)
+                   segment=segment, o_acc=o_acc, past_masks=past_masks, fwd_ws=fwd_ws)
     _check(load().oomb_chunk_attn_fwd(pool, ctypes.byref(a), _stream(stream)),
            "oomb_chunk_attn_fwd")
+
+
+def chunk_attn_fwd_workspace_size(head_dim) -> int:
+    return load().oomb_chunk_attn_fwd_workspace_size(head_dim)
+
+
+def fwd_workspace(head_dim, device) -> torch.Tensor:
+    """A forward workspace (fp32, zero-initialised) for chunk_attn_fwd's fwd_ws."""
+    n = chunk_attn_fwd_workspace_size(head_dim)
+    if n == 0:
+        raise ValueError(f"no forward workspace for head_dim {head_dim}")
+    return torch.zeros(n // 4, dtype=torch.float32, device=device)
 
 
 def chunk_attn_bwd(pool, q, o, lse, d_o, dq, delta_ws, past_pages, past_counts, cur_pages,

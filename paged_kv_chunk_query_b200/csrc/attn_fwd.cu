@@ -24,6 +24,8 @@
 // only moved when a tile's maximum exceeds it by more than 8 (a factor 256),
 // so O is rescaled rarely; the final O / l and LSE = ln2 * (m + log2 l) are
 // exact whichever maximum was used.
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 #include "tiles.cuh"
@@ -51,7 +53,19 @@ struct FwdParams {
   const uint8_t* masks;  // lpq 2: query-page membership bits of each list entry
   int lg_p;              // log2(P)
   float scale_log2;
+  // units (query tile, head) u = h * n_qtiles + qt.  CTAs [0, n_full) take unit
+  // = blockIdx.x whole; with n_split > 0 the remaining units (the last wave's)
+  // are split: CTA n_full + k takes part k % n_split of the key tiles of unit
+  // n_full + k / n_split and writes its normalised O and LSE to part_o /
+  // part_lse [k][128 rows] for fwd_merge_kernel.
+  int n_qtiles, n_full, n_split;
+  float* part_o;
+  float* part_lse;
 };
+
+// Partial-result capacity of the forward workspace: parts of at most this many
+// CTAs (a wave on 148 SMs fits).
+constexpr int kMaxFwdParts = 256;
 
 template <int D>
 struct FwdCfg {
@@ -85,7 +99,14 @@ __global__ void __launch_bounds__(224, 1)
   __shared__ int k_issued_sh, v_issued_sh, k_used_sh, v_used_sh;
 
   const int warp = warp_id(), lane = lane_id();
-  const int qt = blockIdx.x, h = blockIdx.y, g = h / p.G;
+  // this CTA's unit, and its part of the unit's key tiles (part < 0: all)
+  const int cid = blockIdx.x;
+  int unit = cid, part = -1;
+  if (p.n_split > 0 && cid >= p.n_full) {
+    unit = p.n_full + (cid - p.n_full) / p.n_split;
+    part = (cid - p.n_full) % p.n_split;
+  }
+  const int qt = unit % p.n_qtiles, h = unit / p.n_qtiles, g = h / p.G;
   // list of (query tile, group) or of the group
   const int li = (p.lpq ? qt * (p.Hq / p.G) : 0) + g;
   const KvSchedule sch = kv_schedule(p.past_counts ? p.past_counts + (li - g) : nullptr, g,
@@ -93,7 +114,11 @@ __global__ void __launch_bounds__(224, 1)
   // past tiles + (unless this call is a past-only segment) the chunk's tiles up
   // to the diagonal; a past-only segment with an empty list has no tile
   const bool with_cur = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
-  const int T = sch.n_past_tiles + (with_cur ? qt + 1 : 0);
+  const int T_all = sch.n_past_tiles + (with_cur ? qt + 1 : 0);
+  // key tiles [j0, j0 + T) in the unit's order (past, then the chunk's own);
+  // loops count j from 0 and tile j is the unit's tile j0 + j
+  const int j0 = part < 0 ? 0 : part * T_all / p.n_split;
+  const int T = part < 0 ? T_all : (part + 1) * T_all / p.n_split - j0;
   const int n_cur_pages = p.C / p.P;
 
   if (threadIdx.x == 0) {
@@ -151,7 +176,7 @@ __global__ void __launch_bounds__(224, 1)
       for (int j = 0; j < T; ++j) {
         int pg[8];
         for (int s = 0; s < per; ++s)
-          pg[s] = tile_page(j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
+          pg[s] = tile_page(j0 + j, s, sch, past_list, p.cur_pages, n_cur_pages, p.P,
                             p.num_pool_pages, is_k ? p.status : nullptr);
         const int st = j % nst;
         if (!mbar_wait(&empty[st], ((j / nst) & 1) ^ 1, abort_flag)) break;
@@ -258,28 +283,29 @@ __global__ void __launch_bounds__(224, 1)
       for (int c = 0; c < kTile / 32; ++c)
         tmem_ld32(tmem + lane_off + b * 128 + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
       tmem_ld_wait();
+      const int jt = j0 + j;  // the unit's tile
       int lim;
-      if (j < sch.n_past_tiles) {
-        lim = n_past_keys - j * kTile;
+      if (jt < sch.n_past_tiles) {
+        lim = n_past_keys - jt * kTile;
       } else {
-        const int key0 = (j - sch.n_past_tiles) * kTile;
+        const int key0 = (jt - sch.n_past_tiles) * kTile;
         lim = min(p.C, q_local + 1) - key0;
       }
       if (lim < kTile) {  // diagonal or ragged tile: keys at and past `lim` are masked
 #pragma unroll
         for (int c = 0; c < kTile; ++c) s[c] = c < lim ? s[c] : -INFINITY;
       }
-      if (p.masks && j < sch.n_past_tiles) {
+      if (p.masks && jt < sch.n_past_tiles) {
         // per-query-page lists: a listed page this row's query page did not
         // select is masked (its bit in the entry's membership mask is clear)
         const int per = kTile >> p.lg_p;
-        const uint8_t* mrow = p.masks + static_cast<size_t>(li) * p.max_past + j * per;
+        const uint8_t* mrow = p.masks + static_cast<size_t>(li) * p.max_past + jt * per;
         const int qb = r >> p.lg_p;
         // bit k: columns [16k, 16k + 16) (one page: P >= 16) are kept
         uint32_t keep = 0;
         for (int k = 0; k < kTile / 16; ++k) {
           const int sl = (16 * k) >> p.lg_p;
-          if (j * per + sl < sch.n_past_pages && ((mrow[sl] >> qb) & 1u)) keep |= 1u << k;
+          if (jt * per + sl < sch.n_past_pages && ((mrow[sl] >> qb) & 1u)) keep |= 1u << k;
         }
         if (keep != 0xFFu) {
 #pragma unroll
@@ -368,6 +394,10 @@ __global__ void __launch_bounds__(224, 1)
       const float scale_s = (T > 0 && l > 0.f) ? w_s / l : 0.f;
       const size_t ridx = (static_cast<size_t>(q_local) * p.Hq + h) * D;
       const bool write_bf16 = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
+      // a part of a split unit: its normalised O and LSE into the workspace
+      // (every row; the merge writes the valid ones)
+      const bool as_part = part >= 0;
+      const size_t prow = as_part ? static_cast<size_t>(cid - p.n_full) * kTile + r : 0;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -375,7 +405,17 @@ __global__ void __launch_bounds__(224, 1)
           tmem_ld32(tmem + lane_off + Cfg::kColO + c * 32, o);
           tmem_ld_wait();
         }
-        if (valid) {
+        if (as_part) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x0 = T > 0 ? __uint_as_float(o[4 * e]) * scale_s : 0.f;
+            const float x1 = T > 0 ? __uint_as_float(o[4 * e + 1]) * scale_s : 0.f;
+            const float x2 = T > 0 ? __uint_as_float(o[4 * e + 2]) * scale_s : 0.f;
+            const float x3 = T > 0 ? __uint_as_float(o[4 * e + 3]) * scale_s : 0.f;
+            dst[e] = make_float4(x0, x1, x2, x3);
+          }
+        } else if (valid) {
           float x[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[e] = T > 0 ? __uint_as_float(o[e]) * scale_s : 0.f;
@@ -406,7 +446,8 @@ __global__ void __launch_bounds__(224, 1)
           }
         }
       }
-      if (valid) *lse_ptr = merge ? lse_new : lse_s;
+      if (as_part) p.part_lse[prow] = lse_s;
+      else if (valid) *lse_ptr = merge ? lse_new : lse_s;
     }
   }
 
@@ -424,6 +465,64 @@ __global__ void __launch_bounds__(224, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }
+}
+
+// The parts of the split units merged: grid (n_tail, kTile / rows per CTA),
+// 128 threads, a thread 8 consecutive d of one row.  For each row
+//   LSE = ln sum_k e^LSE_k,  O = sum_k e^(LSE_k - LSE) O_k
+// over the unit's n_split parts in part order (a part whose keys were all
+// masked for the row has LSE_k = -inf and weight 0); writes o (bf16) and lse.
+template <int D>
+__global__ void __launch_bounds__(128) fwd_merge_kernel(const FwdParams p) {
+  constexpr int TPR = D / 8;      // threads per row
+  constexpr int RPC = 128 / TPR;  // rows per CTA
+  const int ti = blockIdx.x;
+  const int row = blockIdx.y * RPC + threadIdx.x / TPR, seg = threadIdx.x % TPR;
+  const int unit = p.n_full + ti;
+  const int qt = unit % p.n_qtiles, h = unit / p.n_qtiles;
+  const int q_local = qt * kTile + row;
+  if (row >= kTile || q_local >= p.C) return;
+  const size_t base = static_cast<size_t>(ti) * p.n_split;
+  float mx = -INFINITY;
+  for (int k = 0; k < p.n_split; ++k) mx = fmaxf(mx, p.part_lse[(base + k) * kTile + row]);
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  float den = 0.f;
+  if (mx != -INFINITY) {
+    for (int k = 0; k < p.n_split; ++k) {
+      const float lk = p.part_lse[(base + k) * kTile + row];
+      if (lk == -INFINITY) continue;
+      const float wk = expf(lk - mx);
+      den += wk;
+      const float4* src =
+          reinterpret_cast<const float4*>(p.part_o + ((base + k) * kTile + row) * D + seg * 8);
+      const float4 a0 = src[0], a1 = src[1];
+      acc[0] = fmaf(wk, a0.x, acc[0]);
+      acc[1] = fmaf(wk, a0.y, acc[1]);
+      acc[2] = fmaf(wk, a0.z, acc[2]);
+      acc[3] = fmaf(wk, a0.w, acc[3]);
+      acc[4] = fmaf(wk, a1.x, acc[4]);
+      acc[5] = fmaf(wk, a1.y, acc[5]);
+      acc[6] = fmaf(wk, a1.z, acc[6]);
+      acc[7] = fmaf(wk, a1.w, acc[7]);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint32_t pk[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D + seg * 8) =
+      make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  if (seg == 0)
+    p.lse[static_cast<size_t>(h) * p.C + q_local] = mx == -INFINITY ? -INFINITY : mx + logf(den);
+}
+
+int sm_count(int device) {
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
 }
 
 template <int D>
@@ -476,12 +575,41 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.o_acc = a->o_acc;
   p.masks = a->lists_per_qtile == 2 ? a->past_masks : nullptr;
   p.lg_p = __builtin_ctz(static_cast<unsigned>(s.P));
-  dim3 grid(s.n_qtiles, s.Hq);
-  attn_fwd_kernel<D><<<grid, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
+  // one CTA per unit (one per SM); with a workspace the last, partial wave's
+  // units are split over the SMs it leaves free
+  const int units = s.n_qtiles * s.Hq;
+  int n_tail = 0;
+  p.n_qtiles = s.n_qtiles;
+  p.n_full = units;
+  p.n_split = 0;
+  p.part_o = a->fwd_ws;
+  p.part_lse = a->fwd_ws ? a->fwd_ws + static_cast<size_t>(kMaxFwdParts) * kTile * D : nullptr;
+  if (a->fwd_ws && a->segment == OOMB_SEG_WHOLE) {
+    const int ns = sm_count(pool->desc.device);
+    const int tail = units % ns;
+    if (tail > 0) {
+      const int parts = std::min(ns / tail, kMaxFwdParts / tail);
+      if (parts >= 2) {
+        n_tail = tail;
+        p.n_full = units - tail;
+        p.n_split = parts;
+      }
+    }
+  }
+  attn_fwd_kernel<D><<<p.n_full + n_tail * p.n_split, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
+  if (n_tail > 0) {
+    constexpr int rows_per_cta = 128 / (D / 8);
+    fwd_merge_kernel<D><<<dim3(n_tail, kTile / rows_per_cta), 128, 0, stream>>>(p);
+  }
   return check_launch();
 }
 
 }  // namespace
+
+extern "C" size_t oomb_chunk_attn_fwd_workspace_size(int32_t head_dim) {
+  if (head_dim != 64 && head_dim != 128) return 0;
+  return static_cast<size_t>(kMaxFwdParts) * kTile * (head_dim + 1) * sizeof(float);
+}
 
 extern "C" oomb_status oomb_chunk_attn_fwd(oomb_pool* pool, const oomb_attn_args* args,
                                            void* stream) {

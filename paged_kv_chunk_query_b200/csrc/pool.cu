@@ -260,6 +260,7 @@ oomb_status validate_attn(const oomb_pool* pool, const oomb_attn_args* a, bool b
   }
   if (!a->q || !a->o || !a->lse || !a->cur_pages) return OOMB_ERR_INVALID_ARG;
   if (!aligned16(a->q) || !aligned16(a->o)) return OOMB_ERR_INVALID_ARG;
+  if (!backward && a->fwd_ws && !aligned16(a->fwd_ws)) return OOMB_ERR_INVALID_ARG;
   if (!(a->softmax_scale > 0.f)) return OOMB_ERR_INVALID_ARG;
   if (backward) {
     if (!a->d_o || !a->dq || !a->delta_ws || !pool->grad) return OOMB_ERR_INVALID_ARG;

@@ -97,6 +97,8 @@ class OffloadRun:
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device)
                        for _ in range(n)]
+        # forward workspace (split last wave); every forward runs on the compute stream
+        self.fwd_ws = L.fwd_workspace(d, device)
         # every chunk's selection, copied back for inspection (not on the schedule's path)
         self.sel_hist = torch.zeros((N, Hkv, self.sel_max), dtype=torch.int32).pin_memory()
         self.cnt_hist = torch.zeros((N, Hkv), dtype=torch.int32).pin_memory()
@@ -166,7 +168,7 @@ class OffloadRun:
             past = self.past_dev[b] if c else None
             cnt = self.cnt_dev[b] if c else None
             L.chunk_attn_fwd(self.stage, x["q"], o, lse, past, cnt, self.cur_dev[b],
-                             w.softmax_scale, comp)
+                             w.softmax_scale, comp, fwd_ws=self.fwd_ws)
             if backward:
                 delta = self.deltas[b]
                 L.chunk_attn_bwd(self.stage, x["q"], o, lse, x["do"], dq, delta, past, cnt,

@@ -13,9 +13,12 @@ import paged_kv_chunk_query_b200 as pk
 
 
 class PagedRun:
-    def __init__(self, w, device="cuda", num_pages=None, alloc_seed=None):
+    def __init__(self, w, device="cuda", num_pages=None, alloc_seed=None, split_fwd=True):
         self.w = w
         self.dev = torch.device(device)
+        # forward workspace: the last partial wave of (query tile, head) units is
+        # split along its key tiles (every small test shape takes that path)
+        self.fwd_ws = pk.fwd_workspace(w.head_dim, self.dev) if split_fwd else None
         self.num_pages = num_pages or w.num_pages
         seed = w.alloc_seed if alloc_seed is None else alloc_seed
         self.pool = pk.pool_create(self.num_pages, w.page_size, w.num_kv_heads, w.head_dim,
@@ -67,7 +70,8 @@ class PagedRun:
         q = inp["q"].to(self.dev).contiguous()
         o = torch.empty_like(q)
         lse = torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32, device=self.dev)
-        pk.chunk_attn_fwd(self.pool, q, o, lse, past, counts, cur, w.softmax_scale)
+        pk.chunk_attn_fwd(self.pool, q, o, lse, past, counts, cur, w.softmax_scale,
+                          fwd_ws=self.fwd_ws)
         out = {"o": o, "lse": lse, "cur": cur, "past": past, "counts": counts}
         if backward:
             do = inp["do"].to(self.dev).contiguous()

@@ -152,6 +152,13 @@ def test_qsum_topk_workspace_size_formula():
     assert L.page_topk_qsum_workspace_size(4, -1) == 0
 
 
+def test_fwd_workspace_size_formula():
+    # 256 parts x 128 rows: normalised fp32 O (d values) and the LSE per row
+    assert L.chunk_attn_fwd_workspace_size(128) == 256 * 128 * (128 + 1) * 4
+    assert L.chunk_attn_fwd_workspace_size(64) == 256 * 128 * (64 + 1) * 4
+    assert L.chunk_attn_fwd_workspace_size(96) == 0
+
+
 def test_newer_entry_points_reject_host_pools_without_touching_cuda():
     """Block moves, list builders, batched / static Top-K and the projection
     check their pools' locations on the host first."""

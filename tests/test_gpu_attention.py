@@ -104,3 +104,29 @@ def test_page_lists_per_group_match_oracle(name):
     assert rel_l2(dq, ref["dq"]) <= BWD_REL
     assert rel_l2(dk, ref["dk"]) <= BWD_REL
     assert rel_l2(dv, ref["dv"]) <= BWD_REL
+
+
+# Units are (128-row query tile, query head); the forward runs one per SM.
+# 160 units on 148 SMs: 148 whole, the last 12 split 12 ways (n_full > 0);
+# 148 units fill the SMs exactly (no split even with a workspace).
+SPLIT_CASES = {
+    "units160_tail12": synth.Workload("u160", 80, 4, 64, 32, 256, 2, seed=21, shuffle_pages=True),
+    "units148_no_tail": synth.Workload("u148", 74, 2, 64, 32, 256, 2, seed=22),
+    "g7_d128_p64_ragged": CASES["g7_d128_p64_ragged"],
+}
+
+
+@pytest.mark.parametrize("split", [False, True])
+@pytest.mark.parametrize("name", list(SPLIT_CASES))
+def test_forward_split_last_wave_matches_oracle(name, split):
+    """With and without the forward workspace, the forward gives the oracle's O
+    and LSE: the split last wave (parts of a unit's key tiles, merged by
+    log-sum-exp) within the same tolerance as the whole units."""
+    w = SPLIT_CASES[name]
+    inp = synth.sequence_inputs(w)
+    ref = _oracle(w, inp, backward=False)
+    with PagedRun(w, split_fwd=split) as r:
+        outs = [r.chunk(c, synth.chunk_inputs(w, c), backward=False) for c in range(w.num_chunks)]
+        torch.cuda.synchronize()
+        assert r.status() == 0
+        _check_fwd(w, ref, outs)

@@ -28,7 +28,7 @@ def _run_chunk(r, w, c, past, cnt):
     q = ch["q"].cuda()
     o = torch.empty_like(q)
     lse = torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32, device="cuda")
-    pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale)
+    pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale, fwd_ws=r.fwd_ws)
     dq = torch.empty_like(q)
     delta = torch.empty_like(lse)
     pk.chunk_attn_bwd(r.pool, q, o, lse, ch["do"].cuda(), dq, delta, past, cnt, cur,

@@ -59,7 +59,7 @@ def _run_local(w, window, backward=True):
             q = inp["q"].to(DEV).contiguous()
             o = torch.empty_like(q)
             lse = torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32, device=DEV)
-            pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale)
+            pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale, fwd_ws=r.fwd_ws)
             out = {"o": o, "lse": lse}
             if backward:
                 do = inp["do"].to(DEV).contiguous()

@@ -121,7 +121,7 @@ def _run(w, sels, union=True):
             q = inp["q"].to(DEV).contiguous()
             o = torch.empty_like(q)
             lse = torch.empty((w.num_q_heads, C), dtype=torch.float32, device=DEV)
-            pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale,
+            pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale, fwd_ws=r.fwd_ws,
                               past_masks=masks)
             dq = torch.empty_like(q)
             pk.chunk_attn_bwd(r.pool, q, o, lse, inp["do"].to(DEV).contiguous(), dq,
@@ -252,6 +252,7 @@ def test_per_query_page_topk_then_attention():
             o = torch.empty_like(q)
             lse = torch.empty((w.num_q_heads, C), dtype=torch.float32, device=DEV)
             pk.chunk_attn_fwd(r.pool, q, o, lse, past, counts, cur, w.softmax_scale,
+                              fwd_ws=r.fwd_ws,
                               past_masks=masks)
             dq = torch.empty_like(q)
             pk.chunk_attn_bwd(r.pool, q, o, lse, ch["do"].to(DEV).contiguous(), dq,

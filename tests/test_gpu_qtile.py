@@ -51,7 +51,7 @@ def _run(w, sels, backward=True):
             q = inp["q"].to(DEV).contiguous()
             o = torch.empty_like(q)
             lse = torch.empty((w.num_q_heads, w.chunk_len), dtype=torch.float32, device=DEV)
-            pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale)
+            pk.chunk_attn_fwd(r.pool, q, o, lse, past, cnt, cur, w.softmax_scale, fwd_ws=r.fwd_ws)
             out = {"o": o, "lse": lse}
             if backward:
                 dq = torch.empty_like(q)
@@ -168,7 +168,8 @@ def test_per_qtile_topk_then_attention():
             cur = r.append(ch["k"], ch["v"])
             o = torch.empty_like(q)
             lse = torch.empty((w.num_q_heads, C), dtype=torch.float32, device=DEV)
-            pk.chunk_attn_fwd(r.pool, q, o, lse, past, counts, cur, w.softmax_scale)
+            pk.chunk_attn_fwd(r.pool, q, o, lse, past, counts, cur, w.softmax_scale,
+                              fwd_ws=r.fwd_ws)
             dq = torch.empty_like(q)
             pk.chunk_attn_bwd(r.pool, q, o, lse, ch["do"].to(DEV).contiguous(), dq,
                               torch.empty_like(lse), past, counts, cur, w.softmax_scale)

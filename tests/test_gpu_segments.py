@@ -65,7 +65,7 @@ def _run_segmented(w, seg_pages, empty_last=False):
                 lists.append((mode, ids, cnt))
             for mode, ids, cnt in lists:
                 pk.chunk_attn_fwd(r.pool, q, o, lse, ids, cnt, cur, w.softmax_scale,
-                                  segment=mode, o_acc=o_acc)
+                                  fwd_ws=r.fwd_ws, segment=mode, o_acc=o_acc)
             for mode, ids, cnt in lists:
                 pk.chunk_attn_bwd(r.pool, q, o, lse, do, dq, delta, ids, cnt, cur,
                                   w.softmax_scale, segment=mode, o_acc=o_acc, dq_acc=dq_acc)
@@ -118,8 +118,9 @@ def test_segment_arguments_are_checked():
         q = inp["q"].to(DEV).contiguous()
         o, lse = torch.empty_like(q), torch.empty((4, 128), dtype=torch.float32, device=DEV)
         with pytest.raises(pk.OombError):     # a segment without the fp32 running output
-            pk.chunk_attn_fwd(r.pool, q, o, lse, None, None, cur, w.softmax_scale,
+            pk.chunk_attn_fwd(r.pool, q, o, lse, None, None, cur, w.softmax_scale, fwd_ws=r.fwd_ws,
                               segment=pk.SEG_FIRST)
         with pytest.raises(pk.OombError):     # mode out of range
-            pk.chunk_attn_fwd(r.pool, q, o, lse, None, None, cur, w.softmax_scale, segment=7,
+            pk.chunk_attn_fwd(r.pool, q, o, lse, None, None, cur, w.softmax_scale,
+                              fwd_ws=r.fwd_ws, segment=7,
                               o_acc=torch.empty((128, 4, 64), dtype=torch.float32, device=DEV))
