@@ -549,7 +549,9 @@ def e2e_dense(w, steps, device):
     """Same dense workload through the public API with host buffers: every
     chunk's Q, K, V, dO are copied from pinned host memory and O, LSE, dQ plus
     the final gradient pool are read back, inside the timed region.  Copies run
-    on a copy stream, overlapped with the previous chunk's compute."""
+    on a copy stream, overlapped with the previous chunk's compute; each
+    chunk's dQ runs beside its dK/dV on a second stream (the backward's
+    step calls), as in the device-timed step."""
     import paged_kv_chunk_query_b200 as pk
     from paged_kv_chunk_query_b200 import synth
     N, C, Hq, Hkv, d, P = (w.num_chunks, w.chunk_len, w.num_q_heads, w.num_kv_heads,
@@ -575,13 +577,16 @@ def e2e_dense(w, steps, device):
         dev_out = [(torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device),
                     torch.empty((Hq, C), dtype=torch.float32, device=device),
                     torch.empty((C, Hq, d), dtype=torch.bfloat16, device=device)) for _ in range(2)]
-        delta = torch.empty((Hq, C), dtype=torch.float32, device=device)
+        # one delta per buffer parity: chunk c's dQ (side stream) may still read its
+        # delta while chunk c+1's preprocess runs
+        deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(2)]
         fwd_ws = pk.fwd_workspace(d, device)
         past = [None] + [pt[:c * ppc].repeat(Hkv, 1).contiguous() for c in range(1, N)]
         cnt = [None] + [torch.full((Hkv,), c * ppc, dtype=torch.int32, device=device)
                         for c in range(1, N)]
         comp = torch.cuda.current_stream()
         copy = torch.cuda.Stream(device=device)
+        side = torch.cuda.Stream(device=device)   # each chunk's dQ beside its dK/dV
         h2d = sum(t.numel() * t.element_size() for t in host_in[0].values()) * N
         d2h = (sum(t.numel() * t.element_size() for t in (host_o[0], host_lse[0], host_dq[0])) * N
                + host_grad.numel() * 4)
@@ -589,6 +594,7 @@ def e2e_dense(w, steps, device):
         def one_step():
             in_ready = [torch.cuda.Event() for _ in range(N)]
             out_ready = [torch.cuda.Event() for _ in range(N)]
+            dq_done = [torch.cuda.Event() for _ in range(N)]
             out_free = [torch.cuda.Event() for _ in range(N)]
             with torch.cuda.stream(copy):
                 for k, v in host_in[0].items():
@@ -598,8 +604,9 @@ def e2e_dense(w, steps, device):
                 buf = c % 2
                 if c + 1 < N:
                     with torch.cuda.stream(copy):
-                        if c >= 1:
-                            copy.wait_event(out_ready[c - 1])  # inputs buffer (c+1)%2 was chunk c-1's
+                        if c >= 1:  # inputs buffer (c+1)%2 was chunk c-1's
+                            copy.wait_event(out_ready[c - 1])
+                            copy.wait_event(dq_done[c - 1])
                         for k, v in host_in[c + 1].items():
                             dev_in[(c + 1) % 2][k].copy_(v, non_blocking=True)
                         in_ready[c + 1].record(copy)
@@ -612,11 +619,18 @@ def e2e_dense(w, steps, device):
                 pk.kv_append(pool, cur, x["k"], x["v"], comp)
                 pk.chunk_attn_fwd(pool, x["q"], o, lse, past[c], cnt[c], cur, w.softmax_scale, comp,
                                   fwd_ws=fwd_ws)
-                pk.chunk_attn_bwd(pool, x["q"], o, lse, x["do"], dq, delta, past[c], cnt[c], cur,
-                                  w.softmax_scale, comp)
+                delta = deltas[buf]
+                bwd = (pool, x["q"], o, lse, x["do"], dq, delta, past[c], cnt[c], cur,
+                       w.softmax_scale)
+                pk.chunk_attn_bwd(*bwd, comp, step=pk.BWD_PREPROCESS)
+                side.wait_stream(comp)
+                pk.chunk_attn_bwd(*bwd, side, step=pk.BWD_DQ)
+                dq_done[c].record(side)
+                pk.chunk_attn_bwd(*bwd, comp, step=pk.BWD_DKDV)
                 out_ready[c].record(comp)
                 with torch.cuda.stream(copy):
                     copy.wait_event(out_ready[c])
+                    copy.wait_event(dq_done[c])
                     host_o[c].copy_(o, non_blocking=True)
                     host_lse[c].copy_(lse, non_blocking=True)
                     host_dq[c].copy_(dq, non_blocking=True)

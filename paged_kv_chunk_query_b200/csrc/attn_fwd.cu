@@ -467,53 +467,61 @@ __global__ void __launch_bounds__(224, 1)
   }
 }
 
-// The parts of the split units merged: grid (n_tail, kTile / rows per CTA),
-// 128 threads, a thread 8 consecutive d of one row.  For each row
+// The parts of the split units merged: grid (n_tail, kTile / kMergeRows<D>),
+// 128 threads, a thread 4 consecutive d of one row.  For each row
 //   LSE = ln sum_k e^LSE_k,  O = sum_k e^(LSE_k - LSE) O_k
 // over the unit's n_split parts in part order (a part whose keys were all
-// masked for the row has LSE_k = -inf and weight 0); writes o (bf16) and lse.
+// masked for the row has LSE_k = -inf and weight 0; its O is written as 0);
+// writes o (bf16) and lse.  Parts are read in batches of 4 with every load of
+// a batch issued before its first use.
+template <int D>
+constexpr int kMergeRows = 128 / (D / 4);  // rows per merge CTA
+
 template <int D>
 __global__ void __launch_bounds__(128) fwd_merge_kernel(const FwdParams p) {
-  constexpr int TPR = D / 8;      // threads per row
-  constexpr int RPC = 128 / TPR;  // rows per CTA
+  constexpr int TPR = D / 4;  // threads per row
+  constexpr int U = 4;        // parts per batch
   const int ti = blockIdx.x;
-  const int row = blockIdx.y * RPC + threadIdx.x / TPR, seg = threadIdx.x % TPR;
+  const int row = blockIdx.y * kMergeRows<D> + threadIdx.x / TPR, seg = threadIdx.x % TPR;
   const int unit = p.n_full + ti;
   const int qt = unit % p.n_qtiles, h = unit / p.n_qtiles;
   const int q_local = qt * kTile + row;
   if (row >= kTile || q_local >= p.C) return;
-  const size_t base = static_cast<size_t>(ti) * p.n_split;
+  const int n = p.n_split;
+  const size_t base = static_cast<size_t>(ti) * n;
+  // part k of this row: LSE at lse_k[k * kTile], O at o_k[k * kPartStride]
+  const float* lse_k = p.part_lse + base * kTile + row;
+  const float4* o_k = reinterpret_cast<const float4*>(p.part_o + (base * kTile + row) * D) + seg;
+  constexpr size_t kPartStride = static_cast<size_t>(kTile) * D / 4;
   float mx = -INFINITY;
-  for (int k = 0; k < p.n_split; ++k) mx = fmaxf(mx, p.part_lse[(base + k) * kTile + row]);
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < n; ++k) mx = fmaxf(mx, lse_k[static_cast<size_t>(k) * kTile]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
   if (mx != -INFINITY) {
-    for (int k = 0; k < p.n_split; ++k) {
-      const float lk = p.part_lse[(base + k) * kTile + row];
-      if (lk == -INFINITY) continue;
-      const float wk = expf(lk - mx);
-      den += wk;
-      const float4* src =
-          reinterpret_cast<const float4*>(p.part_o + ((base + k) * kTile + row) * D + seg * 8);
-      const float4 a0 = src[0], a1 = src[1];
-      acc[0] = fmaf(wk, a0.x, acc[0]);
-      acc[1] = fmaf(wk, a0.y, acc[1]);
-      acc[2] = fmaf(wk, a0.z, acc[2]);
-      acc[3] = fmaf(wk, a0.w, acc[3]);
-      acc[4] = fmaf(wk, a1.x, acc[4]);
-      acc[5] = fmaf(wk, a1.y, acc[5]);
-      acc[6] = fmaf(wk, a1.z, acc[6]);
-      acc[7] = fmaf(wk, a1.w, acc[7]);
+    for (int k0 = 0; k0 < n; k0 += U) {
+      float lk[U];
+      float4 a[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int k = min(k0 + u, n - 1);  // past the last part: a repeat, weight 0 below
+        lk[u] = lse_k[static_cast<size_t>(k) * kTile];
+        a[u] = o_k[k * kPartStride];
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float wk = (k0 + u < n && lk[u] != -INFINITY) ? expf(lk[u] - mx) : 0.f;
+        den += wk;
+        acc.x = fmaf(wk, a[u].x, acc.x);
+        acc.y = fmaf(wk, a[u].y, acc.y);
+        acc.z = fmaf(wk, a[u].z, acc.z);
+        acc.w = fmaf(wk, a[u].w, acc.w);
+      }
     }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  uint32_t pk[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-  *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D + seg * 8) =
-      make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  *reinterpret_cast<uint2*>(p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D + seg * 4) =
+      make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
   if (seg == 0)
     p.lse[static_cast<size_t>(h) * p.C + q_local] = mx == -INFINITY ? -INFINITY : mx + logf(den);
 }
@@ -598,8 +606,7 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   }
   attn_fwd_kernel<D><<<p.n_full + n_tail * p.n_split, 224, Cfg::kSmem, stream>>>(p, qmap, kvmap);
   if (n_tail > 0) {
-    constexpr int rows_per_cta = 128 / (D / 8);
-    fwd_merge_kernel<D><<<dim3(n_tail, kTile / rows_per_cta), 128, 0, stream>>>(p);
+    fwd_merge_kernel<D><<<dim3(n_tail, kTile / kMergeRows<D>), 128, 0, stream>>>(p);
   }
   return check_launch();
 }
