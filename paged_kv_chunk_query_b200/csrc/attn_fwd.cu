@@ -24,6 +24,12 @@
 // only moved when a tile's maximum exceeds it by more than 8 (a factor 256),
 // so O is rescaled rarely; the final O / l and LSE = ln2 * (m + log2 l) are
 // exact whichever maximum was used.
+//
+// Grid: one CTA per (query tile, head) unit, one CTA per SM.  When the units
+// do not fill whole waves and the caller gives a workspace, the units of the
+// last wave are split along their key tiles over the SMs that wave would
+// leave idle; each part writes a normalised O and its LSE, and
+// fwd_merge_kernel combines them by log-sum-exp.
 #include <algorithm>
 
 #include "internal.h"
