@@ -317,7 +317,6 @@ class Run:
             b.record(st)
             timers.setdefault(name, []).append((a, b))
 
-        ppc = w.pages_per_chunk
         S.wait_stream(M)
         F.wait_stream(M)
         timed("append", lambda: pk.kv_append(self.pool, self.cur[0], self.inputs[0]["k"],
@@ -381,7 +380,6 @@ class Run:
             b.record(st)
             timers.setdefault(name, []).append((a, b))
 
-        ppc = w.pages_per_chunk
         if side is not stream:
             side.wait_stream(stream)
         early = self.early_select and (self.sparse or self.local)
@@ -929,7 +927,7 @@ def oracle_sample(w, rows, seed_chunk=None):
     from oracle.attention import chunk_backward, chunk_forward
     from paged_kv_chunk_query_b200 import synth
     c = w.num_chunks // 2 if seed_chunk is None else seed_chunk
-    C, P = w.chunk_len, w.page_size
+    C = w.chunk_len
     ch = synth.chunk_inputs(w, c)
     q = ch["q"][:rows].float().numpy().astype(np.float64)
     do = ch["do"][:rows].float().numpy().astype(np.float64)
@@ -1154,7 +1152,7 @@ def main():
         ms_s, kt_s = time_steps(sp, a.steps, a.warmup, dist_on, device)
         sparse_status = pk.get_device_status(sp.pool)
         topk_bytes = 0.0
-        C, Hq, Hkv, d, P = ws.chunk_len, ws.num_q_heads, ws.num_kv_heads, ws.head_dim, ws.page_size
+        C, Hq, Hkv, d = ws.chunk_len, ws.num_q_heads, ws.num_kv_heads, ws.head_dim
         for c in range(1, ws.num_chunks):
             n_past = c * ws.pages_per_chunk
             topk_bytes += C * Hq * d * 2 + n_past * (Hkv * d * 4 + 4) + Hkv * (ws.top_k + ws.n_recent) * 8

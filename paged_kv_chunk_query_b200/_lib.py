@@ -81,7 +81,7 @@ def load() -> ctypes.CDLL:
         raise ImportError(f"{LIB_PATH} is missing: build it with "
                           "`python -m paged_kv_chunk_query_b200.build` (no CPU fallback exists)")
     lib = ctypes.CDLL(LIB_PATH)
-    vp, i32, u64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_float
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
     sig = {
         "oomb_pool_create": [ctypes.POINTER(PoolDesc), ctypes.POINTER(vp)],
         "oomb_pool_destroy": [vp],
@@ -464,16 +464,20 @@ def page_topk_static(pool, q, page_table, n_past, top_k, n_recent, out_logical, 
 
 
 def _host_i32(blocks):
+    """A host int32 copy of a block list (list, array or tensor, on any device)
+    and its pointer; the C side reads these lists on the host."""
     if isinstance(blocks, np.ndarray):
         t = torch.from_numpy(np.ascontiguousarray(blocks, dtype=np.int32))
     else:
-        t = torch.as_tensor(blocks, dtype=torch.int32).contiguous()
+        t = torch.as_tensor(blocks, dtype=torch.int32).cpu().contiguous()
     return t, t.data_ptr()
 
 
 def page_prefetch(host_pool, device_pool, src_blocks, dst_blocks, stream=None, done_event=None):
     s, sp = _host_i32(src_blocks)
-    d, dp = _host_i32(dst_blocks)
+    d, dp = _host_i32(dst_blocks)  # d keeps the array behind dp alive
+    if d.numel() != s.numel():
+        raise ValueError("src_blocks and dst_blocks must have the same length")
     ev = _event_handle(done_event, stream)
     _check(load().oomb_page_prefetch(host_pool, device_pool, sp, dp, s.numel(), _stream(stream),
                                      ev), "oomb_page_prefetch")
@@ -481,7 +485,9 @@ def page_prefetch(host_pool, device_pool, src_blocks, dst_blocks, stream=None, d
 
 def grad_writeback(device_pool, host_pool, src_blocks, dst_blocks, stream=None):
     s, sp = _host_i32(src_blocks)
-    d, dp = _host_i32(dst_blocks)
+    d, dp = _host_i32(dst_blocks)  # d keeps the array behind dp alive
+    if d.numel() != s.numel():
+        raise ValueError("src_blocks and dst_blocks must have the same length")
     _check(load().oomb_grad_writeback(device_pool, host_pool, sp, dp, s.numel(),
                                       _stream(stream)), "oomb_grad_writeback")
 

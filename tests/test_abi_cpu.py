@@ -6,7 +6,9 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
+import torch
 
 import paged_kv_chunk_query_b200._lib as L
 from oracle.pool import PoolModel
@@ -150,6 +152,18 @@ def test_qsum_topk_workspace_size_formula():
     assert L.page_topk_qsum_workspace_size(2, 0) == a256(2 * 4) + a256(2 * 2 * 8)
     assert L.page_topk_qsum_workspace_size(0, 10) == 0
     assert L.page_topk_qsum_workspace_size(4, -1) == 0
+
+
+def test_host_block_lists_checked_before_the_call():
+    """Block lists are copied to the host and must pair up one to one; a
+    mismatch is refused before the library is called."""
+    with pytest.raises(ValueError):
+        L.page_prefetch(None, None, [1, 2, 3], [4, 5])
+    with pytest.raises(ValueError):
+        L.grad_writeback(None, None, np.arange(4, dtype=np.int64), [0])
+    t, ptr = L._host_i32(torch.arange(5, dtype=torch.int64))
+    assert t.dtype == torch.int32 and not t.is_cuda and ptr == t.data_ptr()
+    assert t.tolist() == [0, 1, 2, 3, 4]
 
 
 def test_fwd_workspace_size_formula():
