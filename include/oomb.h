@@ -180,9 +180,10 @@ typedef struct oomb_attn_args {
    * bytes, 16-byte aligned; NULL: none).  The forward runs one CTA per (128-row
    * query tile, query head) and one CTA per SM; when the number of such units is
    * not a multiple of the SM count, the units of the last, partial wave are split
-   * along their key tiles over the free SMs (whole-key-set calls only), each part
-   * writes a normalised partial O and its LSE here, and a second launch merges
-   * them (LSE = ln sum_k e^LSE_k, O = sum_k e^(LSE_k - LSE) O_k).  Without it the
+   * along their key tiles over the free SMs, each part writes a normalised
+   * partial O and its LSE here, and a second launch merges them (LSE = ln sum_k
+   * e^LSE_k, O = sum_k e^(LSE_k - LSE) O_k) and, for a segmented call, merges
+   * that with the running o_acc / lse as a whole unit would.  Without it the
    * last wave runs its few units alone.  The backward ignores it.  Calls sharing
    * a workspace must be ordered (one stream). */
   float* fwd_ws;

@@ -381,7 +381,9 @@ __global__ void __launch_bounds__(224, 1)
       float* lse_ptr = p.lse + static_cast<size_t>(h) * p.C + q_local;
       // merge with the running (o_acc, lse) of earlier segments:
       //   LSE = ln(e^LSE_old + e^LSE_s), O = e^(LSE_old - LSE) O_old + e^(LSE_s - LSE) O_s
-      const bool merge = p.seg == OOMB_SEG_NEXT || p.seg == OOMB_SEG_LAST;
+      // (a part of a split unit leaves that to fwd_merge_kernel)
+      const bool as_part = part >= 0;
+      const bool merge = (p.seg == OOMB_SEG_NEXT || p.seg == OOMB_SEG_LAST) && !as_part;
       float w_o = 0.f, w_s = 1.f, lse_new = lse_s;
       if (merge && valid) {
         const float lse_o = *lse_ptr;
@@ -402,7 +404,6 @@ __global__ void __launch_bounds__(224, 1)
       const bool write_bf16 = p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST;
       // a part of a split unit: its normalised O and LSE into the workspace
       // (every row; the merge writes the valid ones)
-      const bool as_part = part >= 0;
       const size_t prow = as_part ? static_cast<size_t>(cid - p.n_full) * kTile + r : 0;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -477,8 +478,11 @@ __global__ void __launch_bounds__(224, 1)
 // 128 threads, a thread 4 consecutive d of one row.  For each row
 //   LSE = ln sum_k e^LSE_k,  O = sum_k e^(LSE_k - LSE) O_k
 // over the unit's n_split parts in part order (a part whose keys were all
-// masked for the row has LSE_k = -inf and weight 0; its O is written as 0);
-// writes o (bf16) and lse.  Parts are read in batches of 4 with every load of
+// masked for the row has LSE_k = -inf and weight 0; its O is written as 0).
+// That is the call's result; a segmented call then merges it with the
+// running (o_acc, lse) as the forward's epilogue does, and the row is written
+// as o (bf16: whole key set, last segment) or o_acc (fp32: first and middle
+// segments) with its lse.  Parts are read in batches of 4 with every load of
 // a batch issued before its first use.
 template <int D>
 constexpr int kMergeRows = 128 / (D / 4);  // rows per merge CTA
@@ -492,7 +496,9 @@ __global__ void __launch_bounds__(128) fwd_merge_kernel(const FwdParams p) {
   const int unit = p.n_full + ti;
   const int qt = unit % p.n_qtiles, h = unit / p.n_qtiles;
   const int q_local = qt * kTile + row;
-  if (row >= kTile || q_local >= p.C) return;
+  // rows past the chunk's end are merged too (their parts exist) but neither
+  // read nor written; every lane stays to the warp barrier below
+  const bool active = q_local < p.C;
   const int n = p.n_split;
   const size_t base = static_cast<size_t>(ti) * n;
   // part k of this row: LSE at lse_k[k * kTile], O at o_k[k * kPartStride]
@@ -525,11 +531,43 @@ __global__ void __launch_bounds__(128) fwd_merge_kernel(const FwdParams p) {
       }
     }
   }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  *reinterpret_cast<uint2*>(p.o + (static_cast<size_t>(q_local) * p.Hq + h) * D + seg * 4) =
-      make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-  if (seg == 0)
-    p.lse[static_cast<size_t>(h) * p.C + q_local] = mx == -INFINITY ? -INFINITY : mx + logf(den);
+  // this call's result for the row: O_s = acc / den, LSE_s
+  const float lse_s = mx == -INFINITY ? -INFINITY : mx + logf(den);
+  float w_s = den > 0.f ? 1.f / den : 0.f, w_o = 0.f, lse_out = lse_s;
+  float* lse_ptr = p.lse + static_cast<size_t>(h) * p.C + q_local;
+  const size_t ridx = (static_cast<size_t>(q_local) * p.Hq + h) * D + seg * 4;
+  if (p.seg == OOMB_SEG_NEXT || p.seg == OOMB_SEG_LAST) {
+    // merged with the running (o_acc, lse) of earlier segments, as the
+    // forward's own epilogue does for a whole unit
+    const float lse_o = active ? *lse_ptr : -INFINITY;
+    const float m2 = fmaxf(lse_o, lse_s);
+    if (m2 == -INFINITY) {
+      lse_out = -INFINITY;
+      w_s = 0.f;
+    } else {
+      const float eo = lse_o == -INFINITY ? 0.f : expf(lse_o - m2);
+      const float es = lse_s == -INFINITY ? 0.f : expf(lse_s - m2);
+      lse_out = m2 + logf(eo + es);
+      w_o = eo / (eo + es);
+      w_s *= es / (eo + es);
+    }
+  }
+  float4 x = make_float4(acc.x * w_s, acc.y * w_s, acc.z * w_s, acc.w * w_s);
+  if (active && w_o > 0.f) {
+    const float4 a4 = *reinterpret_cast<const float4*>(p.o_acc + ridx);
+    x = make_float4(fmaf(a4.x, w_o, x.x), fmaf(a4.y, w_o, x.y), fmaf(a4.z, w_o, x.z),
+                    fmaf(a4.w, w_o, x.w));
+  }
+  if (active) {
+    if (p.seg == OOMB_SEG_WHOLE || p.seg == OOMB_SEG_LAST)
+      *reinterpret_cast<uint2*>(p.o + ridx) =
+          make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+    else
+      *reinterpret_cast<float4*>(p.o_acc + ridx) = x;
+  }
+  // every lane of the row has read the old lse before it is replaced
+  __syncwarp();
+  if (active && seg == 0) *lse_ptr = lse_out;
 }
 
 int sm_count(int device) {
@@ -598,7 +636,7 @@ oomb_status launch_fwd(oomb_pool* pool, const oomb_attn_args* a, const AttnShape
   p.n_split = 0;
   p.part_o = a->fwd_ws;
   p.part_lse = a->fwd_ws ? a->fwd_ws + static_cast<size_t>(kMaxFwdParts) * kTile * D : nullptr;
-  if (a->fwd_ws && a->segment == OOMB_SEG_WHOLE) {
+  if (a->fwd_ws) {
     const int ns = sm_count(pool->desc.device);
     const int tail = units % ns;
     if (tail > 0) {

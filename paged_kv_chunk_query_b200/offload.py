@@ -334,6 +334,8 @@ class DenseOffloadRun:
         # while chunk c+1 runs, so these alternate by chunk parity
         self.side = torch.cuda.Stream(device=device)
         self.deltas = [torch.empty((Hq, C), dtype=torch.float32, device=device) for _ in range(2)]
+        # forward workspace (split last wave of each segment call; one stream)
+        self.fwd_ws = L.fwd_workspace(d, device)
         self.h2d_bytes = self.d2h_bytes = 0
 
     def close(self):
@@ -439,7 +441,8 @@ class DenseOffloadRun:
                 past, cnt = (self.slot_lists[slot], self.counts[n]) if n else (None, None)
                 if kind == "fwd":
                     L.chunk_attn_fwd(self.stage, x["q"], o, lse, past, cnt, cur,
-                                     w.softmax_scale, comp, segment=mode, o_acc=self.o_acc)
+                                     w.softmax_scale, comp, segment=mode, o_acc=self.o_acc,
+                                     fwd_ws=self.fwd_ws)
                     done = torch.cuda.Event()
                     done.record(comp)
                     slot_used[slot] = (done,)

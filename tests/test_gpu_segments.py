@@ -38,10 +38,10 @@ def _segments(n_past, seg_pages, empty_last):
     return list(zip(modes, bounds))
 
 
-def _run_segmented(w, seg_pages, empty_last=False):
+def _run_segmented(w, seg_pages, empty_last=False, split_fwd=True):
     Hkv, C, Hq, d = w.num_kv_heads, w.chunk_len, w.num_q_heads, w.head_dim
     outs = []
-    with PagedRun(w) as r:
+    with PagedRun(w, split_fwd=split_fwd) as r:
         o_acc = torch.empty((C, Hq, d), dtype=torch.float32, device=DEV)
         dq_acc = torch.empty_like(o_acc)
         for c in range(w.num_chunks):
@@ -84,16 +84,20 @@ def _whole(w):
     return outs, dk, dv
 
 
+@pytest.mark.parametrize("split_fwd", [True, False], ids=["split_last_wave", "whole_units"])
 @pytest.mark.parametrize("w,seg_pages,empty_last", [
     (synth.Workload("sg7", 14, 2, 128, 64, 320, 4, seed=71, shuffle_pages=True), 3, False),
     (synth.Workload("sg7e", 14, 2, 128, 64, 320, 4, seed=72, shuffle_pages=True), 4, True),
     (synth.Workload("sg2", 4, 2, 64, 32, 256, 4, seed=73), 5, False),
 ], ids=["g7_d128_seg3", "g7_d128_seg4_empty_last", "g2_d64_seg5"])
-def test_segmented_matches_oracle_and_whole(w, seg_pages, empty_last):
+def test_segmented_matches_oracle_and_whole(w, seg_pages, empty_last, split_fwd):
+    """With the forward workspace every segment call of these small shapes
+    splits its units (a partial wave) and merges the parts into the running
+    o_acc / LSE in the merge launch; without it the units run whole."""
     inp = synth.sequence_inputs(w)
     ref = run_sequence(inp["q"], inp["k"], inp["v"], inp["do"], w.chunk_len, w.page_size,
                        w.softmax_scale)
-    outs, dk, dv = _run_segmented(w, seg_pages, empty_last)
+    outs, dk, dv = _run_segmented(w, seg_pages, empty_last, split_fwd)
     whole, dk_w, dv_w = _whole(w)
     C = w.chunk_len
     for c, (out, wo) in enumerate(zip(outs, whole)):
