@@ -1099,6 +1099,7 @@ def main():
     dense_status = pk.get_device_status(dense.pool)
     step_flops = dense.step_flops
     launches_dense = dense.launches_per_step
+    fwd_merge = dense.fwd_merge
     value = whole_job_rate(step_flops, ms, world) / 1e12
     tokens = whole_job_rate(w.context, ms, world)
     kernel_flops = {k: sum(v) for k, v in dense.flops.items()}
@@ -1320,6 +1321,9 @@ def main():
                    "heads": f"{w.num_q_heads}q/{w.num_kv_heads}kv", "head_dim": w.head_dim,
                    "page_table": "shuffled" if w.shuffle_pages else "identity",
                    "parallelism": f"replicas{world}",
+                   "fwd_schedule": "one CTA per (128-row query tile, head); the last partial "
+                   "wave split along its key tiles over the idle SMs, merged by a second launch"
+                   if fwd_merge else "one CTA per (128-row query tile, head)",
                    "bwd_schedule": "serial" if a.serial_bwd else
                    "dQ on a second stream beside dK/dV; next chunk's append issued early",
                    "l2": "inputs larger than L2 (Q+dO 3.5 GiB, KV pool 512 MiB, grad pool 1 GiB)"},
