@@ -33,9 +33,10 @@
 // The select (up to 4,096 past pages: keys in registers, 16 contiguous pages
 //   per thread): a 256-bucket histogram of the fp32 score on a linear scale
 //   between the candidates' minimum and maximum finds the bucket of the K-th
-//   largest key, exact 8-bit radix passes over the 64-bit keys of that bucket
-//   finish it, and one CTA-wide scan compacts the kept ids in ascending
-//   order; beyond 4,096 pages, 8-bit passes over the keys re-read from L2.
+//   largest key; one warp ranks that bucket's keys when there are at most 64
+//   of them, exact 8-bit radix passes over them otherwise; one CTA-wide scan
+//   compacts the kept ids in ascending order; beyond 4,096 pages, 8-bit
+//   passes over the keys re-read from L2.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -195,12 +196,18 @@ __device__ __forceinline__ uint32_t order_f32(float f) {
 
 // ---------------------------------------------------------------- select
 // Shared state of one CTA's radix select (256 bins, 8 warps of bin scan).
+// A boundary bucket of at most this many keys is ranked by one warp instead
+// of by radix passes.
+constexpr int kSmallBucket = 64;
+
 struct RadixShared {
   unsigned int hist[256];
   unsigned int warp_tot[8];
   int warp_cnt[32];
   unsigned long long kth;
   int need, done;
+  unsigned int n_small;                   // boundary-bucket keys gathered so far
+  unsigned long long small[kSmallBucket];  // and the keys
 };
 
 // One radix step's bin search, once hist[] holds the counts, by the 8-bit
@@ -407,6 +414,7 @@ __device__ void select_pages_regs(const unsigned long long* keys,
     if (t == 0) {
       sh.need = k_eff;
       sh.done = 0;
+      sh.n_small = 0u;
     }
     sh.hist[t] = 0u;
     __syncthreads();
@@ -437,7 +445,27 @@ __device__ void select_pages_regs(const unsigned long long* keys,
           khi = max(khi, kv[j]);
         }
       }
-    if (!bucket_whole) {
+    const unsigned int n_member = sh.hist[B];  // uniform: read after the pick's barrier
+    if (!bucket_whole && n_member <= static_cast<unsigned int>(kSmallBucket)) {
+      // exact K-th key among the boundary bucket's few keys (at least two, all
+      // distinct): gathered into shared memory, then the key that exactly
+      // need - 1 others exceed, found by one warp
+#pragma unroll
+      for (int j = 0; j < KPT; ++j)
+        if ((member_bits >> j) & 1u) sh.small[atomicAdd(&sh.n_small, 1u)] = kv[j];
+      __syncthreads();
+      if (warp == 0) {
+        const int need = sh.need;
+        for (int i = lane; i < static_cast<int>(n_member); i += 32) {
+          const unsigned long long x = sh.small[i];
+          int greater = 0;
+          for (int m = 0; m < static_cast<int>(n_member); ++m) greater += sh.small[m] > x;
+          if (greater == need - 1) sh.kth = x;
+        }
+      }
+      __syncthreads();
+      kth = sh.kth;
+    } else if (!bucket_whole) {
       // exact K-th key among the boundary bucket's keys (at least two of
       // them, all distinct): 8-bit digits from the highest differing bit
 #pragma unroll
